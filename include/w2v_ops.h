@@ -1,0 +1,52 @@
+/*
+ * w2v_ops.h — single-kernel entry points of the same library, for kernel-level
+ * parity tests on shapes the whole model does not reach (odd M, N tails,
+ * varying K) and for the bounded-wait error path.  Same conventions as w2v.h:
+ * plain device pointers owned by the caller, cudaStream_t as void*, int status
+ * return, asynchronous on the stream.  `err_dev` is a caller-owned device int
+ * that a kernel ORs a nonzero code into when one of its bounded waits gives up.
+ */
+#ifndef W2V_OPS_H
+#define W2V_OPS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* out[M][N] = act(A[M][K] * B[N][K]^T + bias) + residual  on the tcgen05 GEMM.
+ * A, B: fp16 row-major (B in the PyTorch Linear layout [out, in]); K a multiple
+ * of 64; bias fp32 [N] or NULL; residual [M][N] fp16 (res_f32 = 0) or fp32
+ * (res_f32 = 1) or NULL; out [M][N] fp16 or fp32 (out_f32); act 0 none,
+ * 1 exact GELU, 2 tanh GELU.  This is the contraction of every projection in
+ * the encoder blocks (README "Recipe" table: q/k/v/out projections,
+ * intermediate_dense, output_dense) and of the CTC head.  bn = 0 picks the
+ * tile width; 32/64/128/256 forces it. */
+int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, const float* bias, const void* residual,
+                int res_f32, void* out, int out_f32, int act, int bn, int* err_dev, void* stream);
+
+/* O = softmax(Q K^T / 8) V per (clip, head) with no mask (plain SDPA, LiteRT
+ * discussion fourth rewrite), head dim 64.  q, k: fp16 [batch][T][H*64];
+ * vt: fp16 [batch][H][64][t_pad] (V transposed per head, t_pad >= T, a multiple
+ * of 8); out: fp16 [batch][T][H*64]. */
+int w2v_op_attention(const void* q, const void* k, const void* vt, void* out, int batch, int T, int H, int t_pad,
+                     int* err_dev, void* stream);
+
+/* y = act(LN(x) * gamma + beta) per row over `cols` (256, 512, 768 or 1024)
+ * channels, biased variance, fp32 statistics.  x fp16 (in_f32 = 0) or fp32;
+ * y fp16. */
+int w2v_op_layernorm(const void* x, int in_f32, void* y, int rows, int cols, const float* gamma, const float* beta,
+                     float eps, int act, void* stream);
+
+/* Launches a kernel whose mbarrier wait can never complete; the bounded wait
+ * gives up after limit_ns and ORs a nonzero code into *err_dev.  Used to test
+ * that the timeout path reports instead of hanging. */
+int w2v_op_wait_probe(int* err_dev, uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W2V_OPS_H */

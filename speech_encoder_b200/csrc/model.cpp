@@ -1,0 +1,1037 @@
+// C ABI of the wav2vec2 CTC forward pass: configuration checks, weight
+// manifest and device layouts, workspace, the per-shape launch plan (tensor
+// maps and tile choices) and the kernel sequence, optionally recorded once per
+// shape as a CUDA graph.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "w2v.h"
+#include "w2v_internal.h"
+#include "w2v_ops.h"
+
+using namespace w2v;
+
+namespace {
+
+constexpr int kC = 512;
+constexpr int kKern[7] = {10, 3, 3, 3, 3, 2, 2};
+constexpr int kStride[7] = {5, 2, 2, 2, 2, 2, 2};
+constexpr int kPosK = 128;
+constexpr int kPosG = 16;
+
+int conv_len(int n, int k, int s) { return n >= k ? (n - k) / s + 1 : 0; }
+
+int frames_of(int n) {
+  int t = n;
+  for (int i = 0; i < 7; ++i) t = conv_len(t, kKern[i], kStride[i]);
+  return t;
+}
+
+struct Entry {
+  std::string name;
+  int ndim;
+  int64_t shape[3];
+  size_t offset;
+  size_t count;
+};
+
+bool check_cfg(const w2v_config* c, std::string* why) {
+  auto bad = [&](const char* m) {
+    if (why) *why = m;
+    return false;
+  };
+  if (!c) return bad("config is NULL");
+  if (c->d_model <= 0 || c->d_model % 256 != 0 || c->d_model > 1024) return bad("d_model must be a multiple of 256, <= 1024");
+  if (c->n_heads <= 0 || c->d_model != 64 * c->n_heads) return bad("d_model / n_heads must be 64");
+  if (c->n_layers < 0 || c->n_layers > 256) return bad("n_layers out of range");
+  if (c->d_ffn <= 0 || c->d_ffn % 64 != 0) return bad("d_ffn must be a positive multiple of 64");
+  if (c->vocab <= 0 || c->vocab > 65536) return bad("vocab out of range");
+  if (c->blank_id < 0 || c->blank_id >= c->vocab) return bad("blank_id out of range");
+  if (c->conv_norm != 0 && c->conv_norm != 1) return bad("conv_norm must be 0 (group) or 1 (layer)");
+  if (c->conv_bias != 0 && c->conv_bias != 1) return bad("conv_bias must be 0 or 1");
+  if (c->stable_layer_norm != 0 && c->stable_layer_norm != 1) return bad("stable_layer_norm must be 0 or 1");
+  if (c->gelu_tanh != 0 && c->gelu_tanh != 1) return bad("gelu_tanh must be 0 or 1");
+  if (c->max_samples < 400 || c->max_samples > 64 * 1024 * 1024) return bad("max_samples out of range");
+  if (c->max_batch < 1 || c->max_batch > 4096) return bad("max_batch out of range");
+  if (!(c->ln_eps > 0.f) || !std::isfinite(c->ln_eps)) return bad("ln_eps must be positive");
+  return true;
+}
+
+std::vector<Entry> manifest(const w2v_config& c) {
+  std::vector<Entry> m;
+  size_t off = 0;
+  auto add = [&](const std::string& n, std::initializer_list<int64_t> s) {
+    Entry e;
+    e.name = n;
+    e.ndim = static_cast<int>(s.size());
+    size_t cnt = 1;
+    int i = 0;
+    for (int64_t v : s) {
+      e.shape[i++] = v;
+      cnt *= static_cast<size_t>(v);
+    }
+    for (; i < 3; ++i) e.shape[i] = 0;
+    e.offset = off;
+    e.count = cnt;
+    off += cnt;
+    m.push_back(e);
+  };
+  const int d = c.d_model, F = c.d_ffn, V = c.vocab;
+  for (int i = 0; i < 7; ++i) {
+    const std::string p = "conv" + std::to_string(i);
+    add(p + ".weight", {kC, i == 0 ? 1 : kC, kKern[i]});
+    if (c.conv_bias) add(p + ".bias", {kC});
+    if (c.conv_norm == 1 || i == 0) {
+      add(p + ".norm.weight", {kC});
+      add(p + ".norm.bias", {kC});
+    }
+  }
+  add("fp.norm.weight", {kC});
+  add("fp.norm.bias", {kC});
+  add("fp.proj.weight", {d, kC});
+  add("fp.proj.bias", {d});
+  add("pos_conv.weight", {d, d / kPosG, kPosK});
+  add("pos_conv.bias", {d});
+  add("enc.norm.weight", {d});
+  add("enc.norm.bias", {d});
+  for (int l = 0; l < c.n_layers; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    for (const char* nm : {"q", "k", "v", "out"}) {
+      add(p + "attn." + nm + ".weight", {d, d});
+      add(p + "attn." + nm + ".bias", {d});
+    }
+    add(p + "attn_norm.weight", {d});
+    add(p + "attn_norm.bias", {d});
+    add(p + "ffn.in.weight", {F, d});
+    add(p + "ffn.in.bias", {F});
+    add(p + "ffn.out.weight", {d, F});
+    add(p + "ffn.out.bias", {d});
+    add(p + "ffn_norm.weight", {d});
+    add(p + "ffn_norm.bias", {d});
+  }
+  add("lm_head.weight", {V, d});
+  add("lm_head.bias", {V});
+  return m;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct LayerDev {
+  __half *wqkv = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr;
+  float *bqkv = nullptr, *bo = nullptr, *b1 = nullptr, *b2 = nullptr;
+  float *ln1g = nullptr, *ln1b = nullptr, *ln2g = nullptr, *ln2b = nullptr;
+};
+
+struct Plan {
+  int n = 0, batch = 0;
+  int T[7] = {};
+  int Tpad[7] = {};
+  int Tf = 0, t_pad = 0, rows = 0;
+  CUtensorMap convA[7], convB[7];
+  GemmShape convS[7];
+  int convBN[7] = {};
+  CUtensorMap projA, projB;
+  GemmShape projS;
+  int projBN = 0;
+  CUtensorMap posX;
+  CUtensorMap aH, aAO, aF;
+  std::vector<CUtensorMap> qkvB, oB, f1B, f2B;
+  GemmShape qkvS, oS, f1S, f2S;
+  int qkvBN = 0, oBN = 0, f1BN = 0, f2BN = 0;
+  CUtensorMap attQ, attK, attVt;
+  CUtensorMap lmB;
+  GemmShape lmS;
+  int lmBN = 0;
+};
+
+}  // namespace
+
+struct w2v_model {
+  w2v_config cfg{};
+  int device = 0;
+  std::string err;
+  void* wmem = nullptr;
+  void* ws = nullptr;
+  // weights
+  float *c0w = nullptr, *c0b = nullptr, *c0g = nullptr, *c0beta = nullptr;
+  __half* cw[7] = {};
+  float* cb[7] = {};
+  float* cg[7] = {};
+  float* cbeta[7] = {};
+  float *fpg = nullptr, *fpb = nullptr;
+  __half* wp = nullptr;
+  float* bp = nullptr;
+  __half* wpos = nullptr;
+  float* bpos = nullptr;
+  float *encg = nullptr, *encb = nullptr;
+  std::vector<LayerDev> L;
+  __half* wlm = nullptr;
+  float* blm = nullptr;
+  // workspace
+  __half *act_a = nullptr, *act_b = nullptr, *ln512 = nullptr, *x = nullptr, *h = nullptr, *q = nullptr,
+         *k = nullptr, *vt = nullptr, *ao = nullptr, *f = nullptr;
+  float* r = nullptr;
+  double* gn_acc = nullptr;
+  int* err_word = nullptr;
+  int32_t* ids = nullptr;
+  int max_rows = 0;
+  std::map<std::pair<int, int>, std::unique_ptr<Plan>> plans;
+  std::map<std::tuple<int, int, const void*, void*>, cudaGraphExec_t> graphs;
+  std::map<std::tuple<int, int, const void*, void*>, int> graph_launches;
+  cudaStream_t cap_stream = nullptr;
+  const Plan* last_plan = nullptr;
+  int last_launches = 0;
+  // staging buffers of w2v_transcribe (allocated on its first call)
+  float* pcm_stage = nullptr;
+  float* logits_stage = nullptr;
+  int32_t* tok_stage = nullptr;
+  int32_t* ntok_stage = nullptr;
+};
+
+namespace {
+
+int fail(w2v_model* m, int code, const char* fmt, ...) {
+  if (m) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    m->err = buf;
+  }
+  return code;
+}
+
+#define CUDA_OR(m, expr)                                                                             \
+  do {                                                                                               \
+    cudaError_t e_ = (expr);                                                                         \
+    if (e_ != cudaSuccess) return fail((m), W2V_ECUDA, "%s: %s (%s:%d)", #expr, cudaGetErrorString(e_), \
+                                       __FILE__, __LINE__);                                          \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 2-D fp16 matrix [rows][cols] (row-major) as a TMA map with box {64, box_rows}, 128-byte swizzle.
+cudaError_t map_matrix(CUtensorMap* t, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t str[1] = {static_cast<uint64_t>(cols) * 2};
+  const uint32_t box[2] = {64, static_cast<uint32_t>(box_rows)};
+  return make_tmap_f16(t, base, 2, dims, str, box, true);
+}
+
+// GEMM A operand: {cols, rows, batch} with a batch stride, box {64, 128, 1}.
+cudaError_t map_a(CUtensorMap* t, const void* base, int64_t cols, int64_t rows, int64_t row_stride_elems, int batch,
+                  int64_t batch_stride_elems) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)};
+  const uint64_t str[2] = {static_cast<uint64_t>(row_stride_elems) * 2, static_cast<uint64_t>(batch_stride_elems) * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return make_tmap_f16(t, base, 3, dims, str, box, true);
+}
+
+int build_plan(w2v_model* m, int n, int batch, Plan* p) {
+  const w2v_config& c = m->cfg;
+  const int d = c.d_model, F = c.d_ffn, V = c.vocab, H = c.n_heads;
+  p->n = n;
+  p->batch = batch;
+  p->T[0] = conv_len(n, kKern[0], kStride[0]);
+  for (int i = 1; i < 7; ++i) p->T[i] = conv_len(p->T[i - 1], kKern[i], kStride[i]);
+  for (int i = 0; i < 7; ++i) p->Tpad[i] = (p->T[i] + 1) & ~1;
+  p->Tf = p->T[6];
+  p->Tpad[6] = p->Tf;  // the last conv layer writes packed rows
+  p->t_pad = (p->Tf + 7) & ~7;
+  p->rows = batch * p->Tf;
+  if (p->Tf < 1) return fail(m, W2V_ESHAPE, "n_samples=%d gives no frame", n);
+
+  for (int i = 1; i < 7; ++i) {
+    const __half* in = ((i - 1) % 2 == 0) ? m->act_a : m->act_b;
+    const int K = kKern[i] * kC;
+    CUDA_OR(m, map_a(&p->convA[i], in, 2 * kC, p->Tpad[i - 1] / 2, 2 * kC, batch,
+                     static_cast<int64_t>(p->Tpad[i - 1]) * kC));
+    GemmShape s;
+    s.M = p->T[i];
+    s.N = kC;
+    s.K = K;
+    s.a_kwrap = 2 * kC;
+    s.batch = batch;
+    p->convS[i] = s;
+    p->convBN[i] = gemm_pick_bn(s);
+    CUDA_OR(m, map_matrix(&p->convB[i], m->cw[i], kC, K, p->convBN[i]));
+  }
+  const int rows = p->rows;
+  {
+    CUDA_OR(m, map_a(&p->projA, m->ln512, kC, rows, kC, 1, 0));
+    GemmShape s;
+    s.M = rows; s.N = d; s.K = kC; s.a_kwrap = kC; s.batch = 1;
+    p->projS = s;
+    p->projBN = gemm_pick_bn(s);
+    CUDA_OR(m, map_matrix(&p->projB, m->wp, d, kC, p->projBN));
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(p->Tf), static_cast<uint64_t>(batch)};
+    const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(p->Tf) * d * 2};
+    const uint32_t box[3] = {8, 256, 1};
+    CUDA_OR(m, make_tmap_f16(&p->posX, m->x, 3, dims, str, box, false));
+  }
+  CUDA_OR(m, map_a(&p->aH, m->h, d, rows, d, 1, 0));
+  CUDA_OR(m, map_a(&p->aAO, m->ao, d, rows, d, 1, 0));
+  CUDA_OR(m, map_a(&p->aF, m->f, F, rows, F, 1, 0));
+  auto shp = [&](int N, int K) {
+    GemmShape s;
+    s.M = rows; s.N = N; s.K = K; s.a_kwrap = K; s.batch = 1;
+    return s;
+  };
+  p->qkvS = shp(3 * d, d);
+  p->oS = shp(d, d);
+  p->f1S = shp(F, d);
+  p->f2S = shp(d, F);
+  p->qkvBN = gemm_pick_bn(p->qkvS);
+  p->oBN = gemm_pick_bn(p->oS);
+  p->f1BN = gemm_pick_bn(p->f1S);
+  p->f2BN = gemm_pick_bn(p->f2S);
+  p->qkvB.resize(c.n_layers);
+  p->oB.resize(c.n_layers);
+  p->f1B.resize(c.n_layers);
+  p->f2B.resize(c.n_layers);
+  for (int l = 0; l < c.n_layers; ++l) {
+    CUDA_OR(m, map_matrix(&p->qkvB[l], m->L[l].wqkv, 3 * d, d, p->qkvBN));
+    CUDA_OR(m, map_matrix(&p->oB[l], m->L[l].wo, d, d, p->oBN));
+    CUDA_OR(m, map_matrix(&p->f1B[l], m->L[l].w1, F, d, p->f1BN));
+    CUDA_OR(m, map_matrix(&p->f2B[l], m->L[l].w2, d, F, p->f2BN));
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(p->Tf), static_cast<uint64_t>(batch)};
+    const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(p->Tf) * d * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    CUDA_OR(m, make_tmap_f16(&p->attQ, m->q, 3, dims, str, box, true));
+    CUDA_OR(m, make_tmap_f16(&p->attK, m->k, 3, dims, str, box, true));
+    const uint64_t vd[2] = {static_cast<uint64_t>(p->Tf), static_cast<uint64_t>(batch) * H * 64};
+    const uint64_t vs[1] = {static_cast<uint64_t>(p->t_pad) * 2};
+    const uint32_t vb[2] = {64, 64};
+    CUDA_OR(m, make_tmap_f16(&p->attVt, m->vt, 2, vd, vs, vb, true));
+  }
+  p->lmS = shp(V, d);
+  p->lmBN = gemm_pick_bn(p->lmS);
+  CUDA_OR(m, map_matrix(&p->lmB, m->wlm, V, d, p->lmBN));
+  return W2V_OK;
+}
+
+int get_plan(w2v_model* m, int n, int batch, const Plan** out) {
+  auto key = std::make_pair(n, batch);
+  auto it = m->plans.find(key);
+  if (it != m->plans.end()) {
+    *out = it->second.get();
+    return W2V_OK;
+  }
+  std::unique_ptr<Plan> p(new Plan());
+  int rc = build_plan(m, n, batch, p.get());
+  if (rc != W2V_OK) return rc;
+  *out = p.get();
+  m->plans[key] = std::move(p);
+  return W2V_OK;
+}
+
+// Optional per-launch instrumentation: counts launches and, when timing,
+// brackets each launch with a CUDA event pair and records its algorithmic
+// cost (FLOPs and the bytes it must move at minimum).
+struct Prof {
+  bool timing = false;
+  int launches = 0;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  struct Rec {
+    int klass;
+    double flops, bytes;
+    cudaEvent_t e0, e1;
+  };
+  std::vector<Rec> recs;
+  cudaEvent_t next() {
+    if (used == pool.size()) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+  ~Prof() {
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+
+#define LAUNCH(KL, FL, BY, EXPR)                                             \
+  do {                                                                       \
+    cudaEvent_t e0_ = nullptr;                                               \
+    if (prof && prof->timing) {                                              \
+      e0_ = prof->next();                                                    \
+      cudaEventRecord(e0_, st);                                              \
+    }                                                                        \
+    CUDA_OR(m, (EXPR));                                                      \
+    if (prof) {                                                              \
+      prof->launches++;                                                      \
+      if (prof->timing) {                                                    \
+        cudaEvent_t e1_ = prof->next();                                      \
+        cudaEventRecord(e1_, st);                                            \
+        prof->recs.push_back({(KL), double(FL), double(BY), e0_, e1_});      \
+      }                                                                      \
+    }                                                                        \
+  } while (0)
+
+// Queues the whole forward pass on `st`.
+int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits, cudaStream_t st, Prof* prof) {
+  const w2v_config& c = m->cfg;
+  const int d = c.d_model, F = c.d_ffn, V = c.vocab, H = c.n_heads, B = p.batch;
+  const int act = c.gelu_tanh ? 2 : 1;
+  const float eps = c.ln_eps;
+  const int rows = p.rows;
+  const double R = rows, D = d, FF = F, VV = V;
+
+  // --- conv feature encoder
+  if (c.conv_norm == 0) {
+    CUDA_OR(m, cudaMemsetAsync(m->gn_acc, 0, sizeof(double) * 65 * B, st));
+    LAUNCH(W2V_K_GN_MOMENTS, 130.0 * p.T[0] * B, 4.0 * p.n * B,
+           launch_gn_moments(pcm, p.n, B, p.T[0], m->gn_acc, st));
+  }
+  LAUNCH(W2V_K_CONV0, 2.0 * 10 * kC * p.T[0] * B, 4.0 * p.n * B + 2.0 * kC * p.T[0] * B,
+         launch_conv0(pcm, p.n, B, p.T[0], p.Tpad[0], m->c0w, m->c0b, m->c0g, m->c0beta, m->gn_acc, c.conv_norm,
+                      eps, act, m->act_a, st));
+  for (int i = 1; i < 7; ++i) {
+    __half* out = (i % 2 == 0) ? m->act_a : m->act_b;
+    GemmEpilogue e;
+    e.bias = m->cb[i];
+    e.out = out;
+    e.ldo = kC;
+    e.out_batch_stride = static_cast<int64_t>(p.Tpad[i]) * kC;
+    e.act = (c.conv_norm == 0) ? act : 0;
+    const double K = p.convS[i].K;
+    LAUNCH(W2V_K_CONV_GEMM, 2.0 * p.T[i] * kC * K * B,
+           2.0 * kC * (p.T[i - 1] + p.T[i]) * B + 2.0 * kC * K,
+           launch_gemm(p.convA[i], p.convB[i], p.convS[i], p.convBN[i], e, m->err_word, st));
+    if (c.conv_norm == 1)
+      LAUNCH(W2V_K_CONV_LN, 0.0, 4.0 * kC * p.Tpad[i] * B,
+             launch_layernorm(out, 0, out, B * p.Tpad[i], kC, m->cg[i], m->cbeta[i], eps, act, st));
+  }
+  const __half* conv_out = m->act_a;  // layer 6 (even) writes act_a, packed [B*Tf][512]
+
+  // --- feature projection: LN(512) then Linear 512 -> d
+  LAUNCH(W2V_K_FP_LN, 0.0, 4.0 * kC * R, launch_layernorm(conv_out, 0, m->ln512, rows, kC, m->fpg, m->fpb, eps, 0, st));
+  {
+    GemmEpilogue e;
+    e.bias = m->bp;
+    e.out = m->x;
+    e.ldo = d;
+    LAUNCH(W2V_K_PROJ_GEMM, 2.0 * R * D * kC, 2.0 * R * kC + 2.0 * D * kC + 2.0 * R * D,
+           launch_gemm(p.projA, p.projB, p.projS, p.projBN, e, m->err_word, st));
+  }
+  // --- positional conv + residual -> r (fp32)
+  LAUNCH(W2V_K_POSCONV, 2.0 * R * D * (D / 16) * 128, 2.0 * R * D + 2.0 * D * (D / 16) * 128 + 4.0 * R * D,
+         launch_posconv(p.posX, m->x, m->wpos, m->bpos, p.Tf, B, d, act, m->r, m->err_word, st));
+
+  // --- encoder blocks
+  const bool stable = c.stable_layer_norm != 0;
+  const double ln_bytes = 6.0 * R * D;  // fp32 in, fp16 out
+  if (!stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, m->encg, m->encb, eps, 0, st));
+  const double res_bytes = (stable ? 4.0 : 2.0) * R * D;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const LayerDev& w = m->L[l];
+    if (stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, w.ln1g, w.ln1b, eps, 0, st));
+    {
+      GemmEpilogue e;
+      e.bias = w.bqkv;
+      e.out = m->q;
+      e.ldo = d;
+      e.qkv_d = d;
+      e.out_k = m->k;
+      e.vt = m->vt;
+      e.t_pad = p.t_pad;
+      e.n_heads = H;
+      e.t_len = p.Tf;
+      LAUNCH(W2V_K_QKV_GEMM, 2.0 * R * 3 * D * D, 2.0 * R * D + 6.0 * D * D + 6.0 * R * D,
+             launch_gemm(p.aH, p.qkvB[l], p.qkvS, p.qkvBN, e, m->err_word, st));
+    }
+    LAUNCH(W2V_K_ATTENTION, 4.0 * B * double(p.Tf) * p.Tf * D, 8.0 * R * D,
+           launch_attention(p.attQ, p.attK, p.attVt, p.Tf, B, H, m->ao, m->err_word, st));
+    {
+      GemmEpilogue e;
+      e.bias = w.bo;
+      if (stable) {
+        e.residual = m->r;
+        e.res_f32 = 1;
+      } else {
+        e.residual = m->h;
+        e.res_f32 = 0;
+      }
+      e.ldr = d;
+      e.out = m->r;
+      e.out_f32 = 1;
+      e.ldo = d;
+      LAUNCH(W2V_K_OUT_GEMM, 2.0 * R * D * D, 2.0 * R * D + 2.0 * D * D + res_bytes + 4.0 * R * D,
+             launch_gemm(p.aAO, p.oB[l], p.oS, p.oBN, e, m->err_word, st));
+    }
+    LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes,
+           launch_layernorm(m->r, 1, m->h, rows, d, stable ? w.ln2g : w.ln1g, stable ? w.ln2b : w.ln1b, eps, 0, st));
+    {
+      GemmEpilogue e;
+      e.bias = w.b1;
+      e.act = act;
+      e.out = m->f;
+      e.ldo = F;
+      LAUNCH(W2V_K_FFN1_GEMM, 2.0 * R * FF * D, 2.0 * R * D + 2.0 * FF * D + 2.0 * R * FF,
+             launch_gemm(p.aH, p.f1B[l], p.f1S, p.f1BN, e, m->err_word, st));
+    }
+    {
+      GemmEpilogue e;
+      e.bias = w.b2;
+      if (stable) {
+        e.residual = m->r;
+        e.res_f32 = 1;
+      } else {
+        e.residual = m->h;
+        e.res_f32 = 0;
+      }
+      e.ldr = d;
+      e.out = m->r;
+      e.out_f32 = 1;
+      e.ldo = d;
+      LAUNCH(W2V_K_FFN2_GEMM, 2.0 * R * D * FF, 2.0 * R * FF + 2.0 * D * FF + res_bytes + 4.0 * R * D,
+             launch_gemm(p.aF, p.f2B[l], p.f2S, p.f2BN, e, m->err_word, st));
+    }
+    if (!stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, w.ln2g, w.ln2b, eps, 0, st));
+  }
+  if (stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, m->encg, m->encb, eps, 0, st));
+
+  // --- CTC head, fp32 logits
+  {
+    GemmEpilogue e;
+    e.bias = m->blm;
+    e.out = logits;
+    e.out_f32 = 1;
+    e.ldo = V;
+    LAUNCH(W2V_K_LM_HEAD, 2.0 * R * VV * D, 2.0 * R * D + 2.0 * VV * D + 4.0 * R * VV,
+           launch_gemm(p.aH, p.lmB, p.lmS, p.lmBN, e, m->err_word, st));
+  }
+  return W2V_OK;
+}
+
+int enqueue_ctc(w2v_model* m, const float* logits, int batch, int T, int t_valid, int32_t* tokens, int32_t* n_tokens,
+                cudaStream_t st, Prof* prof) {
+  const double rows = double(batch) * T;
+  LAUNCH(W2V_K_ARGMAX, 0.0, 4.0 * rows * m->cfg.vocab + 4.0 * rows,
+         launch_argmax(logits, batch * T, m->cfg.vocab, m->ids, st));
+  LAUNCH(W2V_K_CTC_COLLAPSE, 0.0, 8.0 * double(batch) * t_valid,
+         launch_ctc_collapse(m->ids, batch, T, t_valid, m->cfg.blank_id, tokens, n_tokens, st));
+  return W2V_OK;
+}
+
+__half to_half(float v) { return __float2half_rn(v); }
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" int w2v_num_frames(int n_samples) { return n_samples >= 400 ? (n_samples - 400) / 320 + 1 : 0; }
+
+extern "C" size_t w2v_weight_count(const w2v_config* cfg) {
+  if (!check_cfg(cfg, nullptr)) return 0;
+  auto mf = manifest(*cfg);
+  return mf.back().offset + mf.back().count;
+}
+
+extern "C" int w2v_weight_num_entries(const w2v_config* cfg) {
+  if (!check_cfg(cfg, nullptr)) return -1;
+  return static_cast<int>(manifest(*cfg).size());
+}
+
+extern "C" int w2v_weight_entry(const w2v_config* cfg, int index, char* name, size_t name_len, int* ndim,
+                                int64_t shape[3], size_t* offset) {
+  if (!check_cfg(cfg, nullptr)) return W2V_EINVAL;
+  auto mf = manifest(*cfg);
+  if (index < 0 || index >= static_cast<int>(mf.size())) return W2V_EINVAL;
+  const Entry& e = mf[index];
+  if (name && name_len) {
+    std::snprintf(name, name_len, "%s", e.name.c_str());
+  }
+  if (ndim) *ndim = e.ndim;
+  if (shape)
+    for (int i = 0; i < 3; ++i) shape[i] = e.shape[i];
+  if (offset) *offset = e.offset;
+  return W2V_OK;
+}
+
+extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size_t n_floats, w2v_model** out) {
+  if (!out) return W2V_EINVAL;
+  *out = nullptr;
+  std::string why;
+  if (!check_cfg(cfg, &why)) {
+    std::fprintf(stderr, "w2v_create: %s\n", why.c_str());
+    return W2V_EINVAL;
+  }
+  if (!host_weights) return W2V_EINVAL;
+  auto mf = manifest(*cfg);
+  const size_t total = mf.back().offset + mf.back().count;
+  if (n_floats != total) {
+    std::fprintf(stderr, "w2v_create: weight blob has %zu floats, expected %zu\n", n_floats, total);
+    return W2V_ESHAPE;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W2V_EDEVICE;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return W2V_EDEVICE;
+  if (prop.major != 10) {
+    std::fprintf(stderr, "w2v_create: device is sm_%d%d; this library is built for sm_100a\n", prop.major,
+                 prop.minor);
+    return W2V_EDEVICE;
+  }
+
+  if (gemm_prepare() != cudaSuccess || posconv_prepare() != cudaSuccess || attention_prepare() != cudaSuccess) {
+    std::fprintf(stderr, "w2v_create: cannot configure kernels: %s\n", cudaGetErrorString(cudaGetLastError()));
+    return W2V_ECUDA;
+  }
+  std::unique_ptr<w2v_model> m(new w2v_model());
+  m->cfg = *cfg;
+  m->device = dev;
+  const w2v_config& c = m->cfg;
+  const int d = c.d_model, F = c.d_ffn, V = c.vocab, NL = c.n_layers;
+  std::map<std::string, const Entry*> byname;
+  for (auto& e : mf) byname[e.name] = &e;
+  auto src = [&](const std::string& n) { return host_weights + byname.at(n)->offset; };
+
+  // ---------------------------------------------------------- weight arena
+  std::vector<uint8_t> host;  // staged device image
+  size_t cursor = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = round_up(cursor, 256);
+    cursor = o + bytes;
+    if (host.size() < cursor) host.resize(round_up(cursor, 1 << 20));
+    return o;
+  };
+  std::vector<std::pair<size_t, void**>> fix;  // offset -> member pointer
+  auto put_f32 = [&](void** dst, const float* s, size_t cnt) {
+    size_t o = take(cnt * 4);
+    std::memcpy(host.data() + o, s, cnt * 4);
+    fix.push_back({o, dst});
+  };
+  auto put_f32_zero = [&](void** dst, size_t cnt) {
+    size_t o = take(cnt * 4);
+    std::memset(host.data() + o, 0, cnt * 4);
+    fix.push_back({o, dst});
+  };
+  auto put_f16 = [&](void** dst, size_t cnt, auto&& gen) {
+    size_t o = take(cnt * 2);
+    __half* hp = reinterpret_cast<__half*>(host.data() + o);
+    for (size_t i = 0; i < cnt; ++i) hp[i] = to_half(gen(i));
+    fix.push_back({o, dst});
+  };
+
+  put_f32(reinterpret_cast<void**>(&m->c0w), src("conv0.weight"), kC * 10);
+  if (c.conv_bias)
+    put_f32(reinterpret_cast<void**>(&m->c0b), src("conv0.bias"), kC);
+  put_f32(reinterpret_cast<void**>(&m->c0g), src("conv0.norm.weight"), kC);
+  put_f32(reinterpret_cast<void**>(&m->c0beta), src("conv0.norm.bias"), kC);
+  for (int i = 1; i < 7; ++i) {
+    const std::string p = "conv" + std::to_string(i);
+    const float* w = src(p + ".weight");  // [co][ci][k]
+    const int k = kKern[i];
+    // GEMM B operand [co][j*512 + ci]: K ordered tap-major, channel-minor,
+    // matching the A operand's frame-pair view of the input.
+    put_f16(reinterpret_cast<void**>(&m->cw[i]), static_cast<size_t>(kC) * k * kC, [&](size_t idx) {
+      const size_t co = idx / (k * kC), rem = idx % (k * kC), j = rem / kC, ci = rem % kC;
+      return w[(co * kC + ci) * k + j];
+    });
+    if (c.conv_bias) put_f32(reinterpret_cast<void**>(&m->cb[i]), src(p + ".bias"), kC);
+    if (c.conv_norm == 1) {
+      put_f32(reinterpret_cast<void**>(&m->cg[i]), src(p + ".norm.weight"), kC);
+      put_f32(reinterpret_cast<void**>(&m->cbeta[i]), src(p + ".norm.bias"), kC);
+    }
+  }
+  put_f32(reinterpret_cast<void**>(&m->fpg), src("fp.norm.weight"), kC);
+  put_f32(reinterpret_cast<void**>(&m->fpb), src("fp.norm.bias"), kC);
+  {
+    const float* w = src("fp.proj.weight");
+    put_f16(reinterpret_cast<void**>(&m->wp), static_cast<size_t>(d) * kC, [&](size_t i) { return w[i]; });
+  }
+  put_f32(reinterpret_cast<void**>(&m->bp), src("fp.proj.bias"), d);
+  {
+    // Positional conv weight [c][i][j] (c = g*mg + n) -> per (g, j) an [mg x mg]
+    // block in the no-swizzle K-major core-matrix layout: element (n, i) at
+    // (i/8)*mg*8 + n*8 + i%8.
+    const int mg = d / kPosG;
+    const float* w = src("pos_conv.weight");
+    put_f16(reinterpret_cast<void**>(&m->wpos), static_cast<size_t>(kPosG) * kPosK * mg * mg, [&](size_t idx) {
+      const size_t blk = static_cast<size_t>(mg) * mg;
+      const size_t gj = idx / blk, e = idx % blk;
+      const size_t g = gj / kPosK, j = gj % kPosK;
+      const size_t ich = e / (static_cast<size_t>(mg) * 8), rem = e % (static_cast<size_t>(mg) * 8);
+      const size_t nn = rem / 8, i = ich * 8 + rem % 8;
+      return w[((g * mg + nn) * mg + i) * kPosK + j];
+    });
+  }
+  put_f32(reinterpret_cast<void**>(&m->bpos), src("pos_conv.bias"), d);
+  put_f32(reinterpret_cast<void**>(&m->encg), src("enc.norm.weight"), d);
+  put_f32(reinterpret_cast<void**>(&m->encb), src("enc.norm.bias"), d);
+  m->L.resize(NL);
+  for (int l = 0; l < NL; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    LayerDev& L = m->L[l];
+    const float* wq = src(p + "attn.q.weight");
+    const float* wk = src(p + "attn.k.weight");
+    const float* wv = src(p + "attn.v.weight");
+    const size_t dd = static_cast<size_t>(d) * d;
+    put_f16(reinterpret_cast<void**>(&L.wqkv), 3 * dd, [&](size_t i) {
+      return i < dd ? wq[i] : (i < 2 * dd ? wk[i - dd] : wv[i - 2 * dd]);
+    });
+    {
+      size_t o = take(3 * d * 4);
+      std::memcpy(host.data() + o, src(p + "attn.q.bias"), d * 4);
+      std::memcpy(host.data() + o + d * 4, src(p + "attn.k.bias"), d * 4);
+      std::memcpy(host.data() + o + 2 * d * 4, src(p + "attn.v.bias"), d * 4);
+      fix.push_back({o, reinterpret_cast<void**>(&L.bqkv)});
+    }
+    const float* wo = src(p + "attn.out.weight");
+    put_f16(reinterpret_cast<void**>(&L.wo), dd, [&](size_t i) { return wo[i]; });
+    put_f32(reinterpret_cast<void**>(&L.bo), src(p + "attn.out.bias"), d);
+    put_f32(reinterpret_cast<void**>(&L.ln1g), src(p + "attn_norm.weight"), d);
+    put_f32(reinterpret_cast<void**>(&L.ln1b), src(p + "attn_norm.bias"), d);
+    const float* w1 = src(p + "ffn.in.weight");
+    put_f16(reinterpret_cast<void**>(&L.w1), static_cast<size_t>(F) * d, [&](size_t i) { return w1[i]; });
+    put_f32(reinterpret_cast<void**>(&L.b1), src(p + "ffn.in.bias"), F);
+    const float* w2 = src(p + "ffn.out.weight");
+    put_f16(reinterpret_cast<void**>(&L.w2), static_cast<size_t>(F) * d, [&](size_t i) { return w2[i]; });
+    put_f32(reinterpret_cast<void**>(&L.b2), src(p + "ffn.out.bias"), d);
+    put_f32(reinterpret_cast<void**>(&L.ln2g), src(p + "ffn_norm.weight"), d);
+    put_f32(reinterpret_cast<void**>(&L.ln2b), src(p + "ffn_norm.bias"), d);
+  }
+  {
+    const float* w = src("lm_head.weight");
+    put_f16(reinterpret_cast<void**>(&m->wlm), static_cast<size_t>(V) * d, [&](size_t i) { return w[i]; });
+  }
+  put_f32(reinterpret_cast<void**>(&m->blm), src("lm_head.bias"), V);
+  (void)put_f32_zero;
+
+  const size_t wbytes = round_up(cursor, 256);
+  if (cudaMalloc(&m->wmem, wbytes) != cudaSuccess) return W2V_ENOMEM;
+  if (cudaMemcpy(m->wmem, host.data(), wbytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(m->wmem);
+    return W2V_ECUDA;
+  }
+  for (auto& fx : fix) *fx.second = static_cast<uint8_t*>(m->wmem) + fx.first;
+  std::vector<uint8_t>().swap(host);
+
+  // ------------------------------------------------------------ workspace
+  const int B = c.max_batch;
+  const int t0max = conv_len(c.max_samples, kKern[0], kStride[0]);
+  const size_t act_rows = static_cast<size_t>(B) * (t0max + 2) + 256;
+  const int tf = frames_of(c.max_samples);
+  const size_t rows = static_cast<size_t>(B) * tf + 256;
+  const size_t tpad = (tf + 7) & ~7;
+  cursor = 0;
+  std::vector<std::pair<size_t, void**>> wfix;
+  auto wtake = [&](void** dst, size_t bytes) {
+    size_t o = round_up(cursor, 1024);
+    cursor = o + bytes;
+    wfix.push_back({o, dst});
+  };
+  wtake(reinterpret_cast<void**>(&m->act_a), act_rows * kC * 2);
+  wtake(reinterpret_cast<void**>(&m->act_b), act_rows * kC * 2);
+  wtake(reinterpret_cast<void**>(&m->ln512), rows * kC * 2);
+  wtake(reinterpret_cast<void**>(&m->x), rows * d * 2);
+  wtake(reinterpret_cast<void**>(&m->h), rows * d * 2);
+  wtake(reinterpret_cast<void**>(&m->q), rows * d * 2);
+  wtake(reinterpret_cast<void**>(&m->k), rows * d * 2);
+  wtake(reinterpret_cast<void**>(&m->vt), static_cast<size_t>(B) * d * tpad * 2 + 4096);
+  wtake(reinterpret_cast<void**>(&m->ao), rows * d * 2);
+  wtake(reinterpret_cast<void**>(&m->f), rows * F * 2);
+  wtake(reinterpret_cast<void**>(&m->r), rows * d * 4);
+  wtake(reinterpret_cast<void**>(&m->gn_acc), static_cast<size_t>(B) * 65 * 8);
+  wtake(reinterpret_cast<void**>(&m->err_word), 256);
+  wtake(reinterpret_cast<void**>(&m->ids), 3 * rows * 4);  // ids, plus token scratch of the profiler
+  const size_t wsbytes = round_up(cursor, 1 << 20);
+  if (cudaMalloc(&m->ws, wsbytes) != cudaSuccess) {
+    cudaFree(m->wmem);
+    return W2V_ENOMEM;
+  }
+  for (auto& fx : wfix) *fx.second = static_cast<uint8_t*>(m->ws) + fx.first;
+  // Zero the whole workspace once: padding rows and columns are then finite.
+  if (cudaMemset(m->ws, 0, wsbytes) != cudaSuccess) {
+    cudaFree(m->ws);
+    cudaFree(m->wmem);
+    return W2V_ECUDA;
+  }
+  m->max_rows = static_cast<int>(B) * tf;
+  if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaFree(m->ws);
+    cudaFree(m->wmem);
+    return W2V_ECUDA;
+  }
+  *out = m.release();
+  return W2V_OK;
+}
+
+extern "C" int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev,
+                           void* stream) {
+  if (!m) return W2V_EINVAL;
+  if (!pcm_dev || !logits_dev) return fail(m, W2V_EINVAL, "null pointer");
+  if (!aligned16(pcm_dev) || !aligned16(logits_dev)) return fail(m, W2V_EINVAL, "pointers must be 16-byte aligned");
+  if (n_samples < 400) return fail(m, W2V_ESHAPE, "n_samples=%d < 400 (no frame)", n_samples);
+  if (n_samples > m->cfg.max_samples)
+    return fail(m, W2V_ESHAPE, "n_samples=%d > max_samples=%d", n_samples, m->cfg.max_samples);
+  if (batch < 1 || batch > m->cfg.max_batch)
+    return fail(m, W2V_ESHAPE, "batch=%d outside [1, %d]", batch, m->cfg.max_batch);
+  if (cudaSetDevice(m->device) != cudaSuccess) return fail(m, W2V_ECUDA, "cudaSetDevice failed");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Plan* p = nullptr;
+  int rc = get_plan(m, n_samples, batch, &p);
+  if (rc != W2V_OK) return rc;
+  m->last_plan = p;
+  if (!m->cfg.use_cuda_graph) {
+    Prof counter;
+    rc = enqueue_forward(m, *p, pcm_dev, logits_dev, st, &counter);
+    m->last_launches = counter.launches;
+    return rc;
+  }
+
+  auto key = std::make_tuple(n_samples, batch, static_cast<const void*>(pcm_dev), static_cast<void*>(logits_dev));
+  auto it = m->graphs.find(key);
+  if (it == m->graphs.end()) {
+    cudaGraph_t g = nullptr;
+    CUDA_OR(m, cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    Prof counter;
+    rc = enqueue_forward(m, *p, pcm_dev, logits_dev, m->cap_stream, &counter);
+    m->graph_launches[key] = counter.launches;
+    cudaError_t e = cudaStreamEndCapture(m->cap_stream, &g);
+    if (rc != W2V_OK) {
+      if (g) cudaGraphDestroy(g);
+      return rc;
+    }
+    if (e != cudaSuccess) return fail(m, W2V_ECUDA, "graph capture: %s", cudaGetErrorString(e));
+    cudaGraphExec_t ex = nullptr;
+    e = cudaGraphInstantiate(&ex, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return fail(m, W2V_ECUDA, "graph instantiate: %s", cudaGetErrorString(e));
+    it = m->graphs.emplace(key, ex).first;
+  }
+  CUDA_OR(m, cudaGraphLaunch(it->second, st));
+  m->last_launches = m->graph_launches[key];
+  return W2V_OK;
+}
+
+extern "C" int w2v_ctc_greedy(w2v_model* m, const float* logits_dev, int batch, int T, int t_valid,
+                              int32_t* tokens_dev, int32_t* n_tokens_dev, void* stream) {
+  if (!m) return W2V_EINVAL;
+  if (!logits_dev || !tokens_dev || !n_tokens_dev) return fail(m, W2V_EINVAL, "null pointer");
+  if (!aligned16(logits_dev) || !aligned16(tokens_dev) || !aligned16(n_tokens_dev))
+    return fail(m, W2V_EINVAL, "pointers must be 16-byte aligned");
+  if (batch < 1 || batch > m->cfg.max_batch) return fail(m, W2V_ESHAPE, "batch=%d outside [1, %d]", batch, m->cfg.max_batch);
+  if (T < 0 || static_cast<int64_t>(T) * batch > m->max_rows) return fail(m, W2V_ESHAPE, "T=%d too large", T);
+  if (t_valid < 0 || t_valid > T) return fail(m, W2V_ESHAPE, "t_valid=%d outside [0, T=%d]", t_valid, T);
+  CUDA_OR(m, cudaSetDevice(m->device));
+  return enqueue_ctc(m, logits_dev, batch, T, t_valid, tokens_dev, n_tokens_dev, static_cast<cudaStream_t>(stream),
+                     nullptr);
+}
+
+extern "C" int w2v_sync(w2v_model* m, void* stream) {
+  if (!m) return W2V_EINVAL;
+  CUDA_OR(m, cudaSetDevice(m->device));
+  CUDA_OR(m, cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int word = 0;
+  CUDA_OR(m, cudaMemcpy(&word, m->err_word, sizeof(int), cudaMemcpyDeviceToHost));
+  if (word) {
+    CUDA_OR(m, cudaMemset(m->err_word, 0, sizeof(int)));
+    return fail(m, W2V_ETIMEOUT, "a kernel's bounded wait gave up (code 0x%x)", word);
+  }
+  return W2V_OK;
+}
+
+extern "C" int w2v_debug_read(w2v_model* m, int which, void* dst_dev, size_t dst_bytes, size_t* bytes, void* stream) {
+  if (!m || !dst_dev) return W2V_EINVAL;
+  const Plan* p = m->last_plan;
+  if (!p) return fail(m, W2V_EINVAL, "no forward has run");
+  const size_t rows = static_cast<size_t>(p->rows);
+  const void* srcp = nullptr;
+  size_t sz = 0;
+  switch (which) {
+    case 0: srcp = m->act_a; sz = rows * kC * 2; break;
+    case 1: srcp = m->x; sz = rows * m->cfg.d_model * 2; break;
+    case 2: srcp = m->r; sz = rows * m->cfg.d_model * 4; break;
+    case 3: srcp = m->h; sz = rows * m->cfg.d_model * 2; break;
+    default: return fail(m, W2V_EINVAL, "unknown buffer %d", which);
+  }
+  if (bytes) *bytes = sz;
+  if (dst_bytes < sz) return fail(m, W2V_ESHAPE, "destination too small (%zu < %zu)", dst_bytes, sz);
+  CUDA_OR(m, cudaMemcpyAsync(dst_dev, srcp, sz, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return W2V_OK;
+}
+
+extern "C" int w2v_last_error(w2v_model* m, char* buf, size_t len) {
+  if (!m || !buf || !len) return W2V_EINVAL;
+  std::snprintf(buf, len, "%s", m->err.c_str());
+  return W2V_OK;
+}
+
+extern "C" void w2v_destroy(w2v_model* m) {
+  if (!m) return;
+  cudaSetDevice(m->device);
+  for (auto& g : m->graphs) cudaGraphExecDestroy(g.second);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  if (m->pcm_stage) cudaFree(m->pcm_stage);
+  if (m->logits_stage) cudaFree(m->logits_stage);
+  if (m->tok_stage) cudaFree(m->tok_stage);
+  if (m->ntok_stage) cudaFree(m->ntok_stage);
+  if (m->ws) cudaFree(m->ws);
+  if (m->wmem) cudaFree(m->wmem);
+  delete m;
+}
+
+extern "C" int w2v_last_launch_count(w2v_model* m) { return m ? m->last_launches : -1; }
+
+extern "C" const char* w2v_kernel_class_name(int klass) {
+  static const char* names[] = {"gn_moments", "conv0_norm_gelu", "conv_gemm", "conv_layernorm", "fp_layernorm",
+                                "proj_gemm", "posconv", "enc_layernorm", "qkv_gemm", "attention", "out_gemm",
+                                "ffn1_gemm", "ffn2_gemm", "lm_head_gemm", "argmax", "ctc_collapse"};
+  if (klass < 0 || klass >= static_cast<int>(sizeof(names) / sizeof(names[0]))) return "unknown";
+  return names[klass];
+}
+
+extern "C" int w2v_profile_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev,
+                                   void* stream, w2v_kernel_time* out, int max_out, int* n_out) {
+  if (!m || !out || !n_out) return W2V_EINVAL;
+  if (!pcm_dev || !logits_dev || !aligned16(pcm_dev) || !aligned16(logits_dev)) return fail(m, W2V_EINVAL, "bad pointer");
+  if (n_samples < 400 || n_samples > m->cfg.max_samples) return fail(m, W2V_ESHAPE, "n_samples=%d out of range", n_samples);
+  if (batch < 1 || batch > m->cfg.max_batch) return fail(m, W2V_ESHAPE, "batch=%d out of range", batch);
+  CUDA_OR(m, cudaSetDevice(m->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Plan* p = nullptr;
+  int rc = get_plan(m, n_samples, batch, &p);
+  if (rc != W2V_OK) return rc;
+  m->last_plan = p;
+  Prof prof;
+  prof.timing = true;
+  rc = enqueue_forward(m, *p, pcm_dev, logits_dev, st, &prof);
+  if (rc != W2V_OK) return rc;
+  rc = enqueue_ctc(m, logits_dev, batch, p->Tf, p->Tf, m->ids + static_cast<size_t>(batch) * p->Tf,
+                   m->ids + static_cast<size_t>(2) * batch * p->Tf, st, &prof);
+  if (rc != W2V_OK) return rc;
+  CUDA_OR(m, cudaStreamSynchronize(st));
+  int n = 0;
+  for (auto& r : prof.recs) {
+    if (n >= max_out) break;
+    float ms = 0.f;
+    CUDA_OR(m, cudaEventElapsedTime(&ms, r.e0, r.e1));
+    out[n].klass = r.klass;
+    out[n].ms = ms;
+    out[n].flops = r.flops;
+    out[n].bytes = r.bytes;
+    ++n;
+  }
+  *n_out = n;
+  m->last_launches = prof.launches;
+  return W2V_OK;
+}
+
+extern "C" int w2v_transcribe(w2v_model* m, const float* pcm_host, int n_samples, int batch, int t_valid,
+                              int32_t* tokens_host, int32_t* n_tokens_host, void* stream) {
+  if (!m) return W2V_EINVAL;
+  if (!pcm_host || !tokens_host || !n_tokens_host) return fail(m, W2V_EINVAL, "null pointer");
+  if (n_samples < 400 || n_samples > m->cfg.max_samples) return fail(m, W2V_ESHAPE, "n_samples=%d out of range", n_samples);
+  if (batch < 1 || batch > m->cfg.max_batch) return fail(m, W2V_ESHAPE, "batch=%d out of range", batch);
+  const int T = w2v_num_frames(n_samples);
+  if (t_valid < 0 || t_valid > T) return fail(m, W2V_ESHAPE, "t_valid=%d outside [0, %d]", t_valid, T);
+  CUDA_OR(m, cudaSetDevice(m->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!m->pcm_stage) {
+    const size_t ns = static_cast<size_t>(m->cfg.max_batch) * m->cfg.max_samples;
+    const size_t nl = static_cast<size_t>(m->max_rows) * m->cfg.vocab;
+    if (cudaMalloc(&m->pcm_stage, ns * 4) != cudaSuccess || cudaMalloc(&m->logits_stage, nl * 4) != cudaSuccess ||
+        cudaMalloc(&m->tok_stage, static_cast<size_t>(m->max_rows) * 4 + 16) != cudaSuccess ||
+        cudaMalloc(&m->ntok_stage, static_cast<size_t>(m->cfg.max_batch) * 4 + 16) != cudaSuccess)
+      return fail(m, W2V_ENOMEM, "staging buffers");
+  }
+  const size_t pcm_bytes = static_cast<size_t>(batch) * n_samples * 4;
+  CUDA_OR(m, cudaMemcpyAsync(m->pcm_stage, pcm_host, pcm_bytes, cudaMemcpyHostToDevice, st));
+  int rc = w2v_forward(m, m->pcm_stage, n_samples, batch, m->logits_stage, stream);
+  if (rc != W2V_OK) return rc;
+  rc = enqueue_ctc(m, m->logits_stage, batch, T, t_valid, m->tok_stage, m->ntok_stage, st, nullptr);
+  if (rc != W2V_OK) return rc;
+  CUDA_OR(m, cudaMemcpyAsync(n_tokens_host, m->ntok_stage, static_cast<size_t>(batch) * 4, cudaMemcpyDeviceToHost, st));
+  if (t_valid > 0)
+    CUDA_OR(m, cudaMemcpyAsync(tokens_host, m->tok_stage, static_cast<size_t>(batch) * t_valid * 4,
+                               cudaMemcpyDeviceToHost, st));
+  return w2v_sync(m, stream);
+}
+
+// ============================================================ op-level ABI
+
+extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, const float* bias, const void* residual,
+                           int res_f32, void* out, int out_f32, int act, int bn, int* err_dev, void* stream) {
+  if (!A || !B || !out || !err_dev) return W2V_EINVAL;
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0) return W2V_ESHAPE;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return W2V_EINVAL;
+  if (act < 0 || act > 2) return W2V_EINVAL;
+  if (gemm_prepare() != cudaSuccess) return W2V_ECUDA;
+  GemmShape s;
+  s.M = M; s.N = N; s.K = K; s.a_kwrap = K; s.batch = 1;
+  if (bn == 0) bn = gemm_pick_bn(s);
+  if (bn != 32 && bn != 64 && bn != 128 && bn != 256) return W2V_EINVAL;
+  CUtensorMap ta, tb;
+  if (map_a(&ta, A, K, M, K, 1, 0) != cudaSuccess) return W2V_ECUDA;
+  if (map_matrix(&tb, B, N, K, bn) != cudaSuccess) return W2V_ECUDA;
+  GemmEpilogue e;
+  e.bias = bias;
+  e.residual = residual;
+  e.res_f32 = res_f32;
+  e.ldr = N;
+  e.out = out;
+  e.out_f32 = out_f32;
+  e.ldo = N;
+  e.act = act;
+  return launch_gemm(ta, tb, s, bn, e, err_dev, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W2V_OK
+                                                                                                    : W2V_ECUDA;
+}
+
+extern "C" int w2v_op_attention(const void* q, const void* k, const void* vt, void* out, int batch, int T, int H,
+                                int t_pad, int* err_dev, void* stream) {
+  if (!q || !k || !vt || !out || !err_dev) return W2V_EINVAL;
+  if (batch < 1 || T < 1 || H < 1 || t_pad < T || t_pad % 8 != 0) return W2V_ESHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(out)) return W2V_EINVAL;
+  const int d = 64 * H;
+  CUtensorMap tq, tk, tv;
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(T), static_cast<uint64_t>(batch)};
+  const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(T) * d * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  if (make_tmap_f16(&tq, q, 3, dims, str, box, true) != cudaSuccess) return W2V_ECUDA;
+  if (make_tmap_f16(&tk, k, 3, dims, str, box, true) != cudaSuccess) return W2V_ECUDA;
+  const uint64_t vd[2] = {static_cast<uint64_t>(T), static_cast<uint64_t>(batch) * H * 64};
+  const uint64_t vs[1] = {static_cast<uint64_t>(t_pad) * 2};
+  const uint32_t vb[2] = {64, 64};
+  if (make_tmap_f16(&tv, vt, 2, vd, vs, vb, true) != cudaSuccess) return W2V_ECUDA;
+  if (attention_prepare() != cudaSuccess) return W2V_ECUDA;
+  return launch_attention(tq, tk, tv, T, batch, H, static_cast<__half*>(out), err_dev,
+                          static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? W2V_OK
+             : W2V_ECUDA;
+}
+
+extern "C" int w2v_op_layernorm(const void* x, int in_f32, void* y, int rows, int cols, const float* gamma,
+                                const float* beta, float eps, int act, void* stream) {
+  if (!x || !y || !gamma || !beta) return W2V_EINVAL;
+  if (rows < 0 || (cols != 256 && cols != 512 && cols != 768 && cols != 1024)) return W2V_ESHAPE;
+  if (!aligned16(x) || !aligned16(y)) return W2V_EINVAL;
+  return launch_layernorm(x, in_f32, static_cast<__half*>(y), rows, cols, gamma, beta, eps, act,
+                          static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? W2V_OK
+             : W2V_ECUDA;
+}
+
+extern "C" int w2v_op_wait_probe(int* err_dev, uint64_t limit_ns, void* stream) {
+  if (!err_dev) return W2V_EINVAL;
+  if (limit_ns > 5000000000ull) return W2V_EINVAL;
+  return launch_wait_timeout_probe(err_dev, limit_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W2V_OK
+                                                                                                         : W2V_ECUDA;
+}

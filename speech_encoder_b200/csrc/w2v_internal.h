@@ -1,0 +1,104 @@
+// Host-side declarations shared by the kernel launchers and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace w2v {
+
+// ---------------------------------------------------------------- tensor maps
+// Encodes a tiled TMA descriptor for a row-major fp16 tensor with up to 3
+// dimensions (dims[0] innermost).  strides_bytes[i] is the stride of dims[i+1].
+// Returns cudaSuccess or an error (bad alignment, driver entry point missing).
+cudaError_t make_tmap_f16(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
+// ----------------------------------------------------------------------- GEMM
+// D = A * B^T over fp16 operands with fp32 accumulation on tcgen05 and a fused
+// epilogue.  A is read through a 3-D tensor map {K-ish cols, rows, batch}: the
+// K block starting at k is fetched from column (k % a_kwrap) of row
+// (m0 + k / a_kwrap) — a_kwrap = K for an ordinary matrix, or the width of a
+// pair of frames for the stride-2 conv layers (implicit GEMM).
+struct GemmEpilogue {
+  const float* bias = nullptr;     // [N] or null
+  const void* residual = nullptr;  // [rows, ldr], fp16 or fp32 per res_f32, or null
+  int res_f32 = 0;
+  int64_t ldr = 0;
+  int64_t res_batch_stride = 0;    // elements between batch items
+  void* out = nullptr;             // [rows, ldo], fp16 or fp32 per out_f32
+  int out_f32 = 0;
+  int64_t ldo = 0;
+  int64_t out_batch_stride = 0;
+  int act = 0;                     // 0 none, 1 exact GELU, 2 tanh GELU
+  // QKV split: when qkv_d > 0 the N = 3*qkv_d columns go to three places:
+  // [0, d) -> out (Q, row-major, ldo), [d, 2d) -> out_k (K, row-major, ldo),
+  // [2d, 3d) -> vt laid out [batch][head][64][t_pad] (V transposed per head).
+  int qkv_d = 0;
+  void* out_k = nullptr;
+  void* vt = nullptr;
+  int t_pad = 0;
+  int n_heads = 0;
+  int t_len = 0;                   // frames per clip (rows are clip-major)
+};
+
+struct GemmShape {
+  int M = 0;        // valid rows per batch item
+  int N = 0;        // valid output columns
+  int K = 0;        // multiple of 64
+  int a_kwrap = 0;  // see above
+  int batch = 1;
+};
+
+// Chooses the N tile and launches.  tmA: {cols, rows, batch}, box {64,128,1};
+// tmB: {K, N}, box {64, bn} where bn = gemm_pick_bn(...).
+int gemm_pick_bn(const GemmShape& s);
+// Raise the dynamic shared-memory limits of the tcgen05 kernels (idempotent;
+// called before any launch or stream capture).
+cudaError_t gemm_prepare();
+cudaError_t posconv_prepare();
+cudaError_t attention_prepare();
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
+                        const GemmEpilogue& e, int* err, cudaStream_t st);
+
+// ------------------------------------------------------------------ frontend
+// Group layout: per-clip first and second moments of the conv-0 input windows
+// (10 taps, hop 5) accumulated into acc[b][65] (fp64; must be zero on entry).
+cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, double* acc, cudaStream_t st);
+// conv0 + norm + GELU -> fp16 [batch][clip_rows][512] (rows >= t0 untouched).
+//   group layout: per-channel GroupNorm from acc (over all t0 frames),
+//   layer layout: conv bias, per-frame LayerNorm over the 512 channels.
+cudaError_t launch_conv0(const float* pcm, int n, int batch, int t0, int clip_rows, const float* w0, const float* b0,
+                         const float* gamma, const float* beta, const double* acc, int layer_norm, float eps,
+                         int act, __half* out, cudaStream_t st);
+// Row LayerNorm over `cols` channels (512, 768 or 1024), fp16 or fp32 input,
+// fp16 output, optional GELU after the affine.
+cudaError_t launch_layernorm(const void* x, int in_f32, __half* y, int rows, int cols, const float* gamma,
+                             const float* beta, float eps, int act, cudaStream_t st);
+
+// ----------------------------------------------------------- positional conv
+// h[t, c] (fp32) = x[t, c] + GELU(bias[c] + sum_{j, i} x[t + j - 64, g*m + i] * W[c, i, j]),
+// grouped conv over 16 groups of m = d/16 channels, kernel 128.  x is read
+// through tmX {d, T, batch}, box {8, 256, 1}, no swizzle.  wpack holds the
+// weights pre-arranged per (group, tap) in the no-swizzle K-major core-matrix
+// layout that the tensor core reads directly.
+cudaError_t launch_posconv(const CUtensorMap& tmX, const __half* x, const __half* wpack, const float* bias, int T,
+                           int batch, int d, int act, float* h, int* err, cudaStream_t st);
+
+// ----------------------------------------------------------------- attention
+// O = softmax(Q K^T / 8) V per (clip, head), no mask, head dim 64.
+// tmQ/tmK: {d, T, batch} box {64,128,1} SW128; tmVt: {T, batch*H*64} box {64,64} SW128.
+cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt, int T,
+                             int batch, int H, __half* out, int* err, cudaStream_t st);
+
+// ----------------------------------------------------------------------- CTC
+cudaError_t launch_argmax(const float* logits, int rows, int V, int32_t* ids, cudaStream_t st);
+cudaError_t launch_ctc_collapse(const int32_t* ids, int batch, int T, int t_valid, int blank, int32_t* tokens,
+                                int32_t* n_tokens, cudaStream_t st);
+
+// A kernel whose bounded wait runs out on purpose (nothing ever arrives on its
+// barrier); it records kErrTest in *err and returns.
+cudaError_t launch_wait_timeout_probe(int* err, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace w2v

@@ -203,7 +203,7 @@ def workload(name: str) -> Workload:
 
 
 def small_shape(conv_norm="group", stable=False, conv_bias=False, gelu_tanh=False,
-                d_model=128, n_layers=2, n_heads=2, d_ffn=256, vocab=40) -> ModelShape:
+                d_model=256, n_layers=2, n_heads=4, d_ffn=512, vocab=40) -> ModelShape:
     """A reduced model for fast tests: real conv frontend, narrow encoder
     (head dim stays 64, pos-conv groups stay 16)."""
     return ModelShape("small", d_model, n_layers, n_heads, d_ffn, vocab, 0, conv_norm,

@@ -1,0 +1,203 @@
+"""Whole-model parity of the CUDA forward pass against the fp64 oracle, through
+the C ABI, on the same seeded PCM and random-init weights.
+
+Bar: frame count exact; logits max-abs <= 3e-2 and mean-abs <= 2e-3; per-frame
+argmax agreement >= 99.5% on frames whose oracle top-2 margin exceeds 0.1; the
+CTC kernel fed the oracle's own fp32 logits reproduces the oracle's tokens
+exactly (the decision is an fp32 compare on both sides)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import w2v_oracle as O
+from speech_encoder_b200 import w2v as B
+from synth import inputs as S
+
+import w2v_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+LAYOUTS = {
+    "group_post": dict(conv_norm="group", stable=False, conv_bias=False),
+    "group_post_tanh": dict(conv_norm="group", stable=False, conv_bias=False, gelu_tanh=True),
+    "layer_stable": dict(conv_norm="layer", stable=True, conv_bias=True),
+    "layer_stable_tanh": dict(conv_norm="layer", stable=True, conv_bias=True, gelu_tanh=True),
+    "group_post_bias": dict(conv_norm="group", stable=False, conv_bias=True),
+}
+
+
+def _run(model, pcm_np):
+    pcm = torch.from_numpy(np.ascontiguousarray(pcm_np, dtype=np.float32)).cuda()
+    logits = model.forward(pcm)
+    model.sync()
+    return logits.cpu().numpy()
+
+
+@pytest.mark.parametrize("layout", list(LAYOUTS))
+@pytest.mark.parametrize("n", [400, 16000, 41234])
+def test_small_model_matches_oracle(layout, n):
+    shape = S.small_shape(**LAYOUTS[layout])
+    model = U.make_model(shape, max_samples=48000, max_batch=2, seed=3, affine_noise=True)
+    pcm = np.stack([S.synth_pcm(n, 21), S.synth_pcm(n, 22)])
+    got = _run(model, pcm)
+    assert got.shape == (2, O.num_frames(n), shape.vocab)
+    for b in range(2):
+        ref = U.oracle_logits(shape, pcm[b], seed=3, affine_noise=True)
+        U.compare_logits(got[b], ref, f"{layout} n={n} clip {b}")
+    model.close()
+
+
+def test_small_model_stages_match_oracle():
+    # Intermediate activations (conv encoder output, projection, encoder output)
+    # of a 0-layer and a 2-layer model, to localise any disagreement.
+    for nl in (0, 2):
+        shape = S.small_shape(n_layers=nl)
+        model = U.make_model(shape, max_samples=48000, max_batch=1, seed=4, affine_noise=True)
+        pcm = S.synth_pcm(41234, 5)[None]
+        _run(model, pcm)
+        taps = {}
+        U.oracle_logits(shape, pcm[0], seed=4, affine_noise=True, taps=taps)
+        T = O.num_frames(41234)
+        conv = torch.empty(T, 512, dtype=torch.float16, device="cuda")
+        B.w2v_debug_read(model.handle, 0, conv)
+        proj = torch.empty(T, shape.d_model, dtype=torch.float16, device="cuda")
+        B.w2v_debug_read(model.handle, 1, proj)
+        fin = torch.empty(T, shape.d_model, dtype=torch.float16, device="cuda")
+        B.w2v_debug_read(model.handle, 3, fin)
+        torch.cuda.synchronize()
+        for nm, t, ref in (("conv", conv, taps["conv6"]), ("proj", proj, taps["proj"]), ("final", fin, taps["final"])):
+            d = np.abs(t.double().cpu().numpy() - ref)
+            scale = max(1.0, np.abs(ref).max())
+            assert d.max() <= 2e-2 * scale, (nl, nm, d.max(), scale)
+        if nl == 0:
+            r = torch.empty(T, shape.d_model, dtype=torch.float32, device="cuda")
+            B.w2v_debug_read(model.handle, 2, r)
+            torch.cuda.synchronize()
+            assert np.abs(r.double().cpu().numpy() - taps["posconv"]).max() < 2e-2 * max(1, np.abs(taps["posconv"]).max())
+        model.close()
+
+
+def test_graph_replay_equals_direct_launch_and_is_deterministic():
+    shape = S.small_shape()
+    pcm = S.synth_pcm(30000, 9)[None]
+    m1 = U.make_model(shape, 48000, 1, use_cuda_graph=False)
+    m2 = U.make_model(shape, 48000, 1, use_cuda_graph=True)
+    a = _run(m1, pcm)
+    b = _run(m2, pcm)
+    c = _run(m2, pcm)
+    assert np.array_equal(a, b) and np.array_equal(b, c)
+    m1.close()
+    m2.close()
+
+
+def test_forward_rejects_bad_shapes_without_launching():
+    shape = S.small_shape()
+    m = U.make_model(shape, 20000, 2)
+    pcm = torch.zeros(3, 20000, device="cuda")
+    lg = torch.zeros(3, 61, shape.vocab, device="cuda")
+    L = B.lib()
+    assert L.w2v_forward(m.handle, pcm.data_ptr(), 399, 1, lg.data_ptr(), None) == B.W2V_ESHAPE
+    assert L.w2v_forward(m.handle, pcm.data_ptr(), 20001, 1, lg.data_ptr(), None) == B.W2V_ESHAPE
+    assert L.w2v_forward(m.handle, pcm.data_ptr(), 16000, 3, lg.data_ptr(), None) == B.W2V_ESHAPE
+    assert L.w2v_forward(m.handle, pcm.data_ptr() + 4, 16000, 1, lg.data_ptr(), None) == B.W2V_EINVAL
+    tok = torch.zeros(2, 61, dtype=torch.int32, device="cuda")
+    nt = torch.zeros(2, dtype=torch.int32, device="cuda")
+    assert L.w2v_ctc_greedy(m.handle, lg.data_ptr(), 1, 49, 50, tok.data_ptr(), nt.data_ptr(), None) == B.W2V_ESHAPE
+    m.sync()
+    m.close()
+
+
+# ------------------------------------------------------------------ CTC kernel
+def test_ctc_kernel_reproduces_oracle_tokens_on_oracle_logits():
+    rng = np.random.default_rng(0)
+    for (T, V, t_valid) in [(799, 32, 799), (799, 32, 184), (1, 32, 1), (999, 2341, 999), (50, 5, 0), (3000, 8, 2999)]:
+        batch = 2
+        z = rng.normal(size=(batch, T, V)).astype(np.float32)
+        # long runs of repeats and blanks, plus exact ties, like CTC posteriors
+        ids = rng.integers(0, min(V, 4), size=(batch, T))
+        z[np.arange(batch)[:, None], np.arange(T)[None], ids] += 5.0
+        z[:, ::17, 1] = z[:, ::17, 2] = 50.0  # ties: lowest index (1) must win
+        shape = S.small_shape(vocab=V)
+        m = U.make_model(shape, 16000 if T < 49 else 320 * T + 400, batch)
+        lg = torch.from_numpy(z).cuda()
+        tok = torch.full((batch, max(t_valid, 1)), -1, dtype=torch.int32, device="cuda")
+        nt = torch.full((batch,), -1, dtype=torch.int32, device="cuda")
+        B.w2v_ctc_greedy(m.handle, lg, batch, T, t_valid, tok, nt)
+        m.sync()
+        for b in range(batch):
+            want = O.ctc_greedy(z[b], t_valid, 0)
+            n = int(nt[b])
+            assert n == len(want)
+            assert tok[b, :n].cpu().tolist() == want
+        m.close()
+
+
+# ------------------------------------------------------ the five workloads
+def _config_model(name, max_batch=1, max_samples=None):
+    w = S.workload(name)
+    ms = max_samples or max(p.shape[1] for p, _ in w.calls)
+    return w, U.make_model(w.model, ms, max_batch)
+
+
+def _tokens_check(model, logits_t, ref_logits_fp32, t_valid):
+    tok, nt = model.ctc_greedy(logits_t[None] if logits_t.dim() == 2 else logits_t, t_valid)
+    model.sync()
+    # identical argmax rows give identical collapses: decode the GPU logits on the host too
+    got_host = O.ctc_greedy(logits_t.cpu().numpy().reshape(-1, logits_t.shape[-1]), t_valid, 0)
+    assert tok[0, :int(nt[0])].cpu().tolist() == got_host
+
+
+def test_c0_base_1s():
+    w, m = _config_model("c0")
+    got = _run(m, w.calls[0][0])
+    assert got.shape == (1, 49, 32)
+    st = U.compare_logits(got[0], U.oracle_workload_clip("c0", 0, 0), "c0")
+    print("c0", st)
+    _tokens_check(m, torch.from_numpy(got[0]).cuda(), None, 49)
+    m.close()
+
+
+def test_c1_base_16s_window_tanh_and_padded_short_clip():
+    w, m = _config_model("c1")
+    full = _run(m, w.calls[0][0])
+    assert full.shape == (1, 799, 32)
+    print("c1 full", U.compare_logits(full[0], U.oracle_workload_clip("c1", 0, 0), "c1 full"))
+    short = _run(m, w.calls[1][0])
+    ref_short = U.oracle_workload_clip("c1", 1, 0)
+    print("c1 short", U.compare_logits(short[0], ref_short, "c1 short (all 799 frames)"))
+    t_valid = O.num_frames(59200)
+    assert t_valid == 184
+    U.compare_logits(short[0, :t_valid], ref_short[:t_valid], "c1 short valid frames")
+    _tokens_check(m, torch.from_numpy(short[0]).cuda(), None, t_valid)
+    m.close()
+
+
+def test_c2_base_batch16_sampled_clips():
+    w, m = _config_model("c2", max_batch=16)
+    got = _run(m, w.calls[0][0])
+    assert got.shape == (16, 499, 32)
+    for clip in (0, 7, 15):
+        print("c2", clip, U.compare_logits(got[clip], U.oracle_workload_clip("c2", 0, clip), f"c2 clip {clip}"))
+    # every clip's logits are finite and clips differ (no cross-clip mixing by construction of seeds)
+    assert np.isfinite(got).all()
+    m.close()
+
+
+def test_c3_large_stable_16s():
+    w, m = _config_model("c3")
+    got = _run(m, w.calls[0][0])
+    assert got.shape == (1, 799, 2341)
+    print("c3", U.compare_logits(got[0], U.oracle_workload_clip("c3", 0, 0), "c3"))
+    m.close()
+
+
+def test_c4_large_true_length_clips_sampled():
+    w, m = _config_model("c4", max_samples=320000)
+    lens = [p.shape[1] for p, _ in w.calls]
+    outs = [_run(m, p) for p, _ in w.calls]
+    for i, o in enumerate(outs):
+        assert o.shape == (1, O.num_frames(lens[i]), 2341)
+        assert np.isfinite(o).all()
+    for i in (int(np.argmin(lens)), int(np.argmax(lens))):
+        print("c4", i, lens[i], U.compare_logits(outs[i][0], U.oracle_workload_clip("c4", i, 0), f"c4 clip {i}"))
+    m.close()

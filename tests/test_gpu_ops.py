@@ -1,0 +1,142 @@
+"""Kernel-level parity through the C ABI: the tcgen05 GEMM (every tile width,
+every epilogue, ragged M/N tails), the row LayerNorm, the fused attention, and
+the bounded-wait error path.  References are computed in float64 on the host
+from the same fp16/fp32 inputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import w2v_oracle as O
+from speech_encoder_b200 import w2v as B
+
+pytestmark = pytest.mark.gpu
+
+
+def _err():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def _act_ref(x, act):
+    return O.gelu(x) if act == 1 else (O.gelu_tanh(x) if act == 2 else x)
+
+
+GEMM_CASES = [
+    # M, N, K, bn, act, residual, out_f32
+    (128, 64, 64, 64, 0, None, 0),
+    (1, 32, 64, 32, 0, None, 0),
+    (130, 96, 128, 64, 1, None, 0),
+    (799, 2304, 768, 128, 0, None, 0),
+    (799, 768, 3072, 64, 0, "f16", 1),
+    (799, 768, 768, 256, 0, "f32", 1),
+    (799, 3072, 768, 128, 2, None, 0),
+    (300, 2341, 1024, 256, 0, None, 1),
+    (257, 512, 1536, 256, 1, None, 0),
+    (7984, 768, 768, 256, 0, "f16", 1),
+    (49, 32, 768, 32, 0, None, 1),
+    (200, 200, 192, 128, 1, "f32", 0),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bn,act,res,out_f32", GEMM_CASES)
+def test_gemm_matches_fp64(M, N, K, bn, act, res, out_f32):
+    g = torch.Generator().manual_seed(M * 7 + N * 13 + K)
+    A = (torch.rand(M, K, generator=g) * 2 - 1).half()
+    W = ((torch.rand(N, K, generator=g) * 2 - 1) / np.sqrt(K) * 2).half()
+    bias = torch.randn(N, generator=g).float() * 0.1
+    ref = A.double().numpy() @ W.double().numpy().T + bias.double().numpy()
+    ref = _act_ref(ref, act)
+    resid = None
+    if res is not None:
+        resid = torch.randn(M, N, generator=g)
+        resid = resid.half() if res == "f16" else resid.float()
+        ref = ref + resid.double().numpy()
+    out = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.float16, device="cuda")
+    err = _err()
+    rc = B.w2v_op_gemm(A.cuda(), W.cuda(), M, N, K, bias.cuda(), None if resid is None else resid.cuda(),
+                       1 if res == "f32" else 0, out, out_f32, act, err, bn=bn)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    got = out.double().cpu().numpy()
+    scale = max(1.0, float(np.abs(ref).max()))
+    tol = (2e-3 if not out_f32 else 2e-5) * scale + 1e-4 * np.sqrt(K)
+    assert np.abs(got - ref).max() <= tol, (np.abs(got - ref).max(), tol)
+
+
+def test_gemm_every_tile_width_same_result():
+    M, N, K = 333, 256, 512
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(M, K, generator=g).half().cuda()
+    W = (torch.randn(N, K, generator=g) * 0.05).half().cuda()
+    outs = []
+    for bn in (32, 64, 128, 256):
+        out = torch.empty(M, N, dtype=torch.float32, device="cuda")
+        assert B.w2v_op_gemm(A, W, M, N, K, None, None, 0, out, 1, 0, _err(), bn=bn) == 0
+        outs.append(out)
+    torch.cuda.synchronize()
+    ref = A.double().cpu().numpy() @ W.double().cpu().numpy().T
+    for o in outs:
+        assert np.abs(o.double().cpu().numpy() - ref).max() < 1e-3
+
+
+@pytest.mark.parametrize("rows,cols,in_f32,act", [(1, 256, 0, 0), (37, 512, 0, 1), (800, 768, 1, 0),
+                                                  (799, 1024, 1, 2), (1000, 512, 0, 2), (64, 1024, 0, 0)])
+def test_layernorm_matches_oracle(rows, cols, in_f32, act):
+    g = torch.Generator().manual_seed(rows + cols)
+    x = torch.randn(rows, cols, generator=g) * 3 + 1.5
+    x = x.float() if in_f32 else x.half()
+    gamma = 1 + 0.1 * torch.randn(cols, generator=g)
+    beta = 0.1 * torch.randn(cols, generator=g)
+    y = torch.empty(rows, cols, dtype=torch.float16, device="cuda")
+    assert B.w2v_op_layernorm(x.cuda(), in_f32, y, rows, cols, gamma.float().cuda(), beta.float().cuda(), 1e-5,
+                              act) == 0
+    torch.cuda.synchronize()
+    ref = _act_ref(O.layer_norm(x.double().numpy(), gamma.double().numpy(), beta.double().numpy(), 1e-5), act)
+    got = y.double().cpu().numpy()
+    assert np.abs(got - ref).max() < 6e-3
+
+
+def _attn_ref(q, k, v, H):
+    Bt, T, d = q.shape
+    out = np.empty((Bt, T, d))
+    for b in range(Bt):
+        for h in range(H):
+            sl = slice(h * 64, (h + 1) * 64)
+            P = O.softmax_rows(q[b, :, sl] @ k[b, :, sl].T / 8.0)
+            out[b, :, sl] = P @ v[b, :, sl]
+    return out
+
+
+@pytest.mark.parametrize("batch,T,H", [(1, 1, 1), (1, 7, 2), (1, 128, 1), (2, 129, 2), (1, 799, 12),
+                                       (2, 499, 3), (1, 1000, 2), (1, 256, 16)])
+def test_attention_matches_oracle(batch, T, H):
+    g = torch.Generator().manual_seed(T * 31 + H)
+    d = 64 * H
+    q = torch.randn(batch, T, d, generator=g).half()
+    k = torch.randn(batch, T, d, generator=g).half()
+    v = torch.randn(batch, T, d, generator=g).half()
+    t_pad = (T + 7) // 8 * 8
+    vt = torch.zeros(batch, H, 64, t_pad, dtype=torch.float16)
+    vt[..., :T] = v.view(batch, T, H, 64).permute(0, 2, 3, 1)
+    out = torch.empty(batch, T, d, dtype=torch.float16, device="cuda")
+    err = _err()
+    assert B.w2v_op_attention(q.cuda(), k.cuda(), vt.cuda(), out, batch, T, H, t_pad, err) == 0
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = _attn_ref(q.double().numpy(), k.double().numpy(), v.double().numpy(), H)
+    got = out.double().cpu().numpy()
+    assert np.abs(got - ref).max() < 1e-2, np.abs(got - ref).max()
+
+
+def test_bounded_wait_reports_instead_of_hanging():
+    err = _err()
+    assert B.w2v_op_wait_probe(err, 20_000_000) == 0  # 20 ms
+    torch.cuda.synchronize()
+    assert int(err.item()) != 0
+    # The context is still usable afterwards.
+    A = torch.ones(128, 64, dtype=torch.float16, device="cuda")
+    out = torch.empty(128, 64, dtype=torch.float32, device="cuda")
+    err2 = _err()
+    assert B.w2v_op_gemm(A, A[:64], 128, 64, 64, None, None, 0, out, 1, 0, err2) == 0
+    torch.cuda.synchronize()
+    assert int(err2.item()) == 0 and float(out[0, 0]) == 64.0
