@@ -117,6 +117,34 @@ int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, fl
 int w2v_ctc_greedy(w2v_model* m, const float* logits_dev, int batch, int T, int t_valid, int32_t* tokens_dev,
                    int32_t* n_tokens_dev, void* stream);
 
+/* Greedy CTC decode that allocates no memory and needs no model handle.  The
+ * pages have no counterpart of this entry point: it exists for callers that
+ * cannot allocate device memory when they decode — code driven from a
+ * real-time audio callback (cudaMalloc may block on the whole device), programs
+ * whose GPU memory belongs to their own allocator, or plugins whose host
+ * forbids allocations after start-up.
+ *
+ * Same result as w2v_ctc_greedy: logits_dev float32 [batch][T][vocab], frames
+ * [0, t_valid) of each clip, argmax with the lowest index on ties, repeats
+ * merged, blank_id dropped; tokens_dev int32 [batch][t_valid] (clip b's
+ * tokens first), n_tokens_dev int32 [batch].  The caller owns logits and
+ * outputs; the per-frame argmax scratch is a fixed array of
+ * W2V_CTC_STATIC_MAX_ROWS int32 in the library's device memory, which every
+ * GPU that loads the library holds until the process exits.
+ *  - batch * T must not exceed W2V_CTC_STATIC_MAX_ROWS (1048576 frames, e.g.
+ *    16 clips of 30 s): larger requests return W2V_ESHAPE and launch nothing.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before any stream capture.
+ *  - All calls share the one array, so calls whose work overlaps on the GPU
+ *    (on different streams, or from different threads) race and may return
+ *    wrong tokens; serialise them.  Nothing in the array needs clearing: each
+ *    call writes every entry it reads.
+ *  - W2V_EINVAL for null or misaligned (not 16-byte) pointers or a bad
+ *    blank_id; W2V_ECUDA if the lookup or a launch fails. */
+#define W2V_CTC_STATIC_MAX_ROWS (1 << 20)
+int w2v_ctc_greedy_static(const float* logits_dev, int batch, int T, int vocab, int t_valid, int blank_id,
+                          int32_t* tokens_dev, int32_t* n_tokens_dev, void* stream);
+
 /* Waits for `stream`, then reports device-side errors latched since the last
  * call (W2V_ETIMEOUT) or a CUDA error; clears the latch. */
 int w2v_sync(w2v_model* m, void* stream);

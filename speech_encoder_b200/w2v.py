@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
         "w2v_last_error": (I, [VP, ctypes.c_char_p, SZ]),
         "w2v_destroy": (None, [VP]),
         "w2v_transcribe": (I, [VP, VP, I, I, I, VP, VP, VP]),
+        "w2v_ctc_greedy_static": (I, [VP, I, I, I, I, I, VP, VP, VP]),
         "w2v_last_launch_count": (I, [VP]),
         "w2v_kernel_class_name": (ctypes.c_char_p, [I]),
         "w2v_profile_forward": (I, [VP, VP, I, I, VP, VP, ctypes.POINTER(w2v_kernel_time), I, ctypes.POINTER(I)]),
@@ -161,6 +162,13 @@ def w2v_forward(model: int, pcm, n_samples: int, batch: int, logits, stream=None
 def w2v_ctc_greedy(model: int, logits, batch: int, T: int, t_valid: int, tokens, n_tokens, stream=None) -> None:
     _check(lib().w2v_ctc_greedy(model, _ptr(logits), int(batch), int(T), int(t_valid), _ptr(tokens), _ptr(n_tokens),
                                 _stream(stream)), model, "w2v_ctc_greedy")
+
+
+def w2v_ctc_greedy_static(logits, batch: int, T: int, vocab: int, t_valid: int, blank_id: int, tokens, n_tokens,
+                          stream=None) -> int:
+    """Allocation-free greedy CTC decode (no model handle); returns the status code."""
+    return lib().w2v_ctc_greedy_static(_ptr(logits), int(batch), int(T), int(vocab), int(t_valid), int(blank_id),
+                                       _ptr(tokens), _ptr(n_tokens), _stream(stream))
 
 
 def w2v_sync(model: int, stream=None) -> None:
