@@ -106,6 +106,10 @@ int w2v_create(const w2v_config* cfg, const float* host_weights, size_t n_floats
 /* Forward pass of `batch` clips of n_samples each, packed contiguously in
  * pcm_dev (float32 [batch][n_samples], already normalised).  Writes
  * logits_dev (float32 [batch][T][vocab], T = w2v_num_frames(n_samples)).
+ * The first call for a given (n_samples, batch) builds that shape's launch
+ * plan: it times the tile and split-K candidates of every GEMM on the device
+ * (a few milliseconds, synchronous; W2V_AUTOTUNE=0 in the environment uses a
+ * cost model instead), so make that first call outside any stream capture.
  * Errors: W2V_ESHAPE if n_samples < 400 or > max_samples or batch outside
  * [1, max_batch]; W2V_EINVAL for null/misaligned pointers. */
 int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, void* stream);
@@ -186,8 +190,9 @@ const char* w2v_kernel_class_name(int klass);
 
 /* Runs one forward (direct launches, no graph) plus the argmax/collapse over
  * all frames, with a CUDA event pair around every kernel launch, waits for the
- * stream and fills out[0 .. *n_out) in launch order.  Used for per-kernel
- * timing and roofline reporting. */
+ * stream and fills out[0 .. *n_out) in launch order.  The launches are queued
+ * behind a 20 ms device-side gate, so the events measure device time and not
+ * the host's launch rate.  Used for per-kernel timing and roofline reporting. */
 int w2v_profile_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, void* stream,
                         w2v_kernel_time* out, int max_out, int* n_out);
 

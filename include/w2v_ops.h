@@ -23,9 +23,11 @@ extern "C" {
  * 1 exact GELU, 2 tanh GELU.  This is the contraction of every projection in
  * the encoder blocks (README "Recipe" table: q/k/v/out projections,
  * intermediate_dense, output_dense) and of the CTC head.  bn = 0 picks the
- * tile width; 32/64/128/256 forces it. */
+ * tile width and split-K factor; otherwise bn (32/64/128/192/256) and splits
+ * (1..8, <= K/64: the K blocks are divided among a cluster of `splits` CTAs
+ * whose partial sums are reduced in distributed shared memory) are forced. */
 int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, const float* bias, const void* residual,
-                int res_f32, void* out, int out_f32, int act, int bn, int* err_dev, void* stream);
+                int res_f32, void* out, int out_f32, int act, int bn, int splits, int* err_dev, void* stream);
 
 /* O = softmax(Q K^T / 8) V per (clip, head) with no mask (plain SDPA, LiteRT
  * discussion fourth rewrite), head dim 64.  q, k: fp16 [batch][T][H*64];

@@ -10,6 +10,8 @@ namespace w2v {
 // fp32 compare on the stored logits, the same values the caller reads back.
 __global__ void __launch_bounds__(256)
 argmax_kernel(const float* __restrict__ logits, int rows, int V, int32_t* __restrict__ ids) {
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= rows) return;
@@ -37,8 +39,7 @@ argmax_kernel(const float* __restrict__ logits, int rows, int V, int32_t* __rest
 
 cudaError_t launch_argmax(const float* logits, int rows, int V, int32_t* ids, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  argmax_kernel<<<(rows + 7) / 8, 256, 0, st>>>(logits, rows, V, ids);
-  return cudaGetLastError();
+  return launch_pdl(argmax_kernel, dim3((rows + 7) / 8), dim3(256), 0, st, logits, rows, V, ids);
 }
 
 // One CTA of 1024 threads per clip; frames in chunks of 1024 with a block-wide
@@ -49,6 +50,8 @@ ctc_collapse_kernel(const int32_t* __restrict__ ids, int T, int t_valid, int bla
                     int32_t* __restrict__ n_tokens) {
   __shared__ int warp_sums[32];
   __shared__ int total_s;
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.x;
   const int32_t* a = ids + static_cast<int64_t>(b) * T;
   int32_t* out = tokens + static_cast<int64_t>(b) * t_valid;
@@ -88,8 +91,7 @@ ctc_collapse_kernel(const int32_t* __restrict__ ids, int T, int t_valid, int bla
 cudaError_t launch_ctc_collapse(const int32_t* ids, int batch, int T, int t_valid, int blank, int32_t* tokens,
                                 int32_t* n_tokens, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
-  ctc_collapse_kernel<<<batch, 1024, 0, st>>>(ids, T, t_valid, blank, tokens, n_tokens);
-  return cudaGetLastError();
+  return launch_pdl(ctc_collapse_kernel, dim3(batch), dim3(1024), 0, st, ids, T, t_valid, blank, tokens, n_tokens);
 }
 
 // -------------------------------------------------------- bounded-wait probe
@@ -104,6 +106,20 @@ __global__ void wait_timeout_probe_kernel(int* err, uint64_t limit_ns) {
     // Nothing arrives on this barrier: the wait must give up and report.
     if (!mbar_wait(&bar, 0, limit_ns)) atomicOr(err, kErrTest);
   }
+}
+
+// Holds the stream for `ns` nanoseconds (one thread sleeping in 1 us steps):
+// lets a host queue many launches before the device starts on them, so that
+// event timings between them measure device time only.
+__global__ void stream_gate_kernel(uint64_t ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) __nanosleep(1000);
+}
+
+cudaError_t launch_stream_gate(uint64_t ns, cudaStream_t st) {
+  if (ns > 100000000ull) ns = 100000000ull;  // at most 0.1 s
+  stream_gate_kernel<<<1, 1, 0, st>>>(ns);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_timeout_probe(int* err, uint64_t limit_ns, cudaStream_t st) {

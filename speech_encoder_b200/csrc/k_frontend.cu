@@ -22,9 +22,18 @@ constexpr int kK0 = 10;
 constexpr int kS0 = 5;
 constexpr int kMom = kK0 + kK0 * (kK0 + 1) / 2;  // 65
 
+// Moments of the conv-0 input windows of one clip: grid (nblocks, batch).
+// Every block writes its 65 partial sums; the last block of a clip to finish
+// (atomic ticket) adds the partials in block order (deterministic), turns them
+// into per-channel GroupNorm scale/shift (fp64) and re-arms the ticket.
 __global__ void __launch_bounds__(256)
-gn_moments_kernel(const float* __restrict__ pcm, int n, int t0, double* __restrict__ acc) {
-  const float* x = pcm + static_cast<int64_t>(blockIdx.y) * n;
+gn_moments_kernel(const float* __restrict__ pcm, int n, int t0, const float* __restrict__ w0,
+                  const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                  double* __restrict__ partial, unsigned* __restrict__ ticket, float2* __restrict__ scale_shift) {
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.y;
+  const float* x = pcm + static_cast<int64_t>(b) * n;
   float s[kMom];
 #pragma unroll
   for (int i = 0; i < kMom; ++i) s[i] = 0.f;
@@ -41,6 +50,8 @@ gn_moments_kernel(const float* __restrict__ pcm, int n, int t0, double* __restri
     }
   }
   __shared__ float red[8][kMom];
+  __shared__ double mom[kMom];
+  __shared__ unsigned last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int i = 0; i < kMom; ++i) {
@@ -50,66 +61,95 @@ gn_moments_kernel(const float* __restrict__ pcm, int n, int t0, double* __restri
     if (lane == 0) red[warp][i] = v;
   }
   __syncthreads();
+  double* mine = partial + (static_cast<int64_t>(b) * gridDim.x + blockIdx.x) * kMom;
   if (threadIdx.x < kMom) {
     double sum = 0.0;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w][threadIdx.x];
-    atomicAdd(acc + blockIdx.y * kMom + threadIdx.x, sum);
+    mine[threadIdx.x] = sum;
+    __threadfence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicAdd(ticket + b, 1u) == gridDim.x - 1) ? 1u : 0u;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (threadIdx.x < kMom) {
+    const volatile double* pb = partial + static_cast<int64_t>(b) * gridDim.x * kMom;
+    double sum = 0.0;
+    for (unsigned k = 0; k < gridDim.x; ++k) sum += pb[k * kMom + threadIdx.x];
+    mom[threadIdx.x] = sum;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ticket[b] = 0u;
+  const double inv = 1.0 / static_cast<double>(t0);
+  for (int c = threadIdx.x; c < kC; c += blockDim.x) {
+    double w[kK0], m[kK0];
+#pragma unroll
+    for (int j = 0; j < kK0; ++j) {
+      w[j] = w0[c * kK0 + j];
+      m[j] = mom[j] * inv;
+    }
+    double mean = 0.0, var = 0.0;
+    int idx = kK0;
+#pragma unroll
+    for (int j = 0; j < kK0; ++j) {
+      mean += w[j] * m[j];
+#pragma unroll
+      for (int jj = j; jj < kK0; ++jj) {
+        const double cov = mom[idx++] * inv - m[j] * m[jj];
+        var += (jj == j ? 1.0 : 2.0) * w[j] * w[jj] * cov;
+      }
+    }
+    if (var < 0.0) var = 0.0;
+    const double scale = static_cast<double>(gamma[c]) / sqrt(var + static_cast<double>(eps));
+    // a conv bias cancels inside the normalisation, so it never appears here
+    scale_shift[b * kC + c] = make_float2(static_cast<float>(scale),
+                                          static_cast<float>(static_cast<double>(beta[c]) - mean * scale));
   }
 }
 
-cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, double* acc, cudaStream_t st) {
+int gn_moment_blocks(int t0) {
   int nb = (t0 + 256 * 8 - 1) / (256 * 8);
   if (nb > 296) nb = 296;
   if (nb < 1) nb = 1;
-  gn_moments_kernel<<<dim3(nb, batch), 256, 0, st>>>(pcm, n, t0, acc);
-  return cudaGetLastError();
+  return nb;
+}
+
+cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, const float* w0, const float* gamma,
+                              const float* beta, float eps, double* partial, unsigned* ticket, float2* scale_shift,
+                              cudaStream_t st) {
+  return launch_pdl(gn_moments_kernel, dim3(gn_moment_blocks(t0), batch), dim3(256), 0, st, pcm, n, t0, w0, gamma,
+                    beta, eps, partial, ticket, scale_shift);
 }
 
 // One warp per output frame; lane l owns channel pairs (2l + 64i, 2l + 64i + 1),
 // i = 0..7, so each half2 store instruction of a warp writes 128 contiguous bytes.
-__global__ void __launch_bounds__(256)
+// group layout: y*scale + shift from the clip's GroupNorm statistics;
+// layer layout: bias, then LayerNorm over the 512 channels of the frame.
+__global__ void __launch_bounds__(256, 2)
 conv0_kernel(const float* __restrict__ pcm, int n, int t0, int clip_rows, const float* __restrict__ w0,
              const float* __restrict__ b0, const float* __restrict__ gamma, const float* __restrict__ beta,
-             const double* __restrict__ acc, int layer_norm, float eps, int act, __half* __restrict__ out) {
+             const float2* __restrict__ scale_shift, int layer_norm, float eps, int act, __half* __restrict__ out) {
   __shared__ __align__(16) float sw[kK0][kC];
   __shared__ __align__(16) float sa[kC];  // group: scale;  layer: gamma
   __shared__ __align__(16) float sb[kC];  // group: shift;  layer: beta
   __shared__ __align__(16) float sbias[kC];
+  if (threadIdx.x == 0) pdl_launch_dependents();
   const int b = blockIdx.y;
   for (int i = threadIdx.x; i < kC * kK0; i += blockDim.x) sw[i % kK0][i / kK0] = w0[i];
-  if (!layer_norm) {
-    // Per-channel GroupNorm statistics from the window moments of this clip.
-    const double* a = acc + b * kMom;
-    const double inv = 1.0 / static_cast<double>(t0);
-    double m[kK0];
-#pragma unroll
-    for (int j = 0; j < kK0; ++j) m[j] = a[j] * inv;
-    for (int c = threadIdx.x; c < kC; c += blockDim.x) {
-      double w[kK0];
-#pragma unroll
-      for (int j = 0; j < kK0; ++j) w[j] = w0[c * kK0 + j];
-      double mean = 0.0, var = 0.0;
-      int idx = kK0;
-#pragma unroll
-      for (int j = 0; j < kK0; ++j) {
-        mean += w[j] * m[j];
-#pragma unroll
-        for (int jj = j; jj < kK0; ++jj) {
-          const double cov = a[idx++] * inv - m[j] * m[jj];
-          var += (jj == j ? 1.0 : 2.0) * w[j] * w[jj] * cov;
-        }
-      }
-      if (var < 0.0) var = 0.0;
-      const double scale = static_cast<double>(gamma[c]) / sqrt(var + static_cast<double>(eps));
-      sa[c] = static_cast<float>(scale);
-      sb[c] = static_cast<float>(static_cast<double>(beta[c]) - mean * scale);
-      sbias[c] = 0.f;  // a conv bias cancels inside the normalisation
-    }
-  } else {
+  if (layer_norm) {
     for (int c = threadIdx.x; c < kC; c += blockDim.x) {
       sa[c] = gamma[c];
       sb[c] = beta[c];
       sbias[c] = b0 ? b0[c] : 0.f;
+    }
+  }
+  pdl_wait();
+  if (!layer_norm) {
+    for (int c = threadIdx.x; c < kC; c += blockDim.x) {
+      const float2 v = scale_shift[b * kC + c];
+      sa[c] = v.x;
+      sb[c] = v.y;
     }
   }
   __syncthreads();
@@ -136,14 +176,7 @@ conv0_kernel(const float* __restrict__ pcm, int n, int t0, int clip_rows, const 
       y[2 * i] = y0;
       y[2 * i + 1] = y1;
     }
-    if (!layer_norm) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = 2 * lane + 64 * i;
-        y[2 * i] = y[2 * i] * sa[c] + sb[c];
-        y[2 * i + 1] = y[2 * i + 1] * sa[c + 1] + sb[c + 1];
-      }
-    } else {
+    if (layer_norm) {
       float sum = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -165,30 +198,27 @@ conv0_kernel(const float* __restrict__ pcm, int n, int t0, int clip_rows, const 
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
       const float rstd = rsqrtf(sq * (1.0f / kC) + eps);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = 2 * lane + 64 * i;
-        y[2 * i] = (y[2 * i] - mean) * rstd * sa[c] + sb[c];
-        y[2 * i + 1] = (y[2 * i + 1] - mean) * rstd * sa[c + 1] + sb[c + 1];
-      }
+      for (int i = 0; i < 16; ++i) y[i] = (y[i] - mean) * rstd;
     }
     __half* orow = ob + static_cast<int64_t>(t) * kC;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int c = 2 * lane + 64 * i;
-      *reinterpret_cast<__half2*>(orow + c) =
-          __floats2half2_rn(apply_act(y[2 * i], act), apply_act(y[2 * i + 1], act));
+      const float a0 = fmaf(y[2 * i], sa[c], sb[c]);
+      const float a1 = fmaf(y[2 * i + 1], sa[c + 1], sb[c + 1]);
+      *reinterpret_cast<__half2*>(orow + c) = __floats2half2_rn(apply_act(a0, act), apply_act(a1, act));
     }
   }
 }
 
 cudaError_t launch_conv0(const float* pcm, int n, int batch, int t0, int clip_rows, const float* w0, const float* b0,
-                         const float* gamma, const float* beta, const double* acc, int layer_norm, float eps,
+                         const float* gamma, const float* beta, const float2* scale_shift, int layer_norm, float eps,
                          int act, __half* out, cudaStream_t st) {
-  int nbx = (t0 + 8 * 16 - 1) / (8 * 16);  // ~16 frames per warp
-  if (nbx > 148 * 8) nbx = 148 * 8;
+  int nbx = (t0 + 8 * 8 - 1) / (8 * 8);  // ~8 frames per warp
+  if (nbx > 148 * 4) nbx = 148 * 4;
   if (nbx < 1) nbx = 1;
-  conv0_kernel<<<dim3(nbx, batch), 256, 0, st>>>(pcm, n, t0, clip_rows, w0, b0, gamma, beta, acc, layer_norm, eps, act, out);
-  return cudaGetLastError();
+  return launch_pdl(conv0_kernel, dim3(nbx, batch), dim3(256), 0, st, pcm, n, t0, clip_rows, w0, b0, gamma, beta,
+                    scale_shift, layer_norm, eps, act, out);
 }
 
 // ------------------------------------------------------------------ LayerNorm
@@ -202,6 +232,8 @@ layernorm_kernel(const void* __restrict__ xin, __half* __restrict__ y, int rows,
   constexpr int VEC = F32IN ? 4 : 8;
   constexpr int NCH = COLS / (32 * VEC);
   constexpr int NPL = COLS / 32;
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= rows) return;
@@ -265,9 +297,9 @@ static void ln_dispatch(const void* x, int in_f32, __half* y, int rows, const fl
                         int act, cudaStream_t st) {
   const int blocks = (rows + 7) / 8;
   if (in_f32)
-    layernorm_kernel<COLS, true><<<blocks, 256, 0, st>>>(x, y, rows, g, b, eps, act);
+    launch_pdl(layernorm_kernel<COLS, true>, dim3(blocks), dim3(256), 0, st, x, y, rows, g, b, eps, act);
   else
-    layernorm_kernel<COLS, false><<<blocks, 256, 0, st>>>(x, y, rows, g, b, eps, act);
+    launch_pdl(layernorm_kernel<COLS, false>, dim3(blocks), dim3(256), 0, st, x, y, rows, g, b, eps, act);
 }
 
 cudaError_t launch_layernorm(const void* x, int in_f32, __half* y, int rows, int cols, const float* gamma,

@@ -2,16 +2,36 @@
 // pass (conv layers 1-6 as implicit GEMM, the feature projection, QKV, the
 // attention output projection, both FFN layers and the CTC head) runs here.
 //
-// One CTA computes a 128 x BN output tile.  Warp roles:
+// One CTA computes a 128 x BN output tile (or a K-range of it, see split-K),
+// 320 threads:
 //   warp 0      TMA producer: A and B K-blocks (64 fp16 = one 128-byte swizzle
-//               atom wide) into a STAGES-deep shared-memory ring
+//               atom wide) into a STAGES-deep shared-memory ring.  Weight (B)
+//               blocks of the first ring fill are issued before waiting on the
+//               previous kernel (programmatic dependent launch).
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16) into an fp32 accumulator in TMEM and frees ring slots
 //               with tcgen05.commit
-//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter of the
-//               accumulator, bias, GELU, residual add, fp16/fp32 stores (or
-//               the Q / K / V^T split of the fused QKV projection)
-#include <stdio.h>
+//   warps 2-9   epilogue.  Two warps per TMEM lane quarter (32 rows) split the
+//               columns.  Three forms:
+//     direct    (one CTA per tile, TMA-storable output): each thread takes its
+//               row's 32-column chunks from TMEM, adds bias and residual,
+//               applies GELU, writes the chunk in the output type into a
+//               swizzled staging box in the drained operand ring, and one lane
+//               per warp issues a TMA tensor store of the 32 x 32 box.
+//     split-K   (s.splits = S > 1): the S CTAs of a tile form a thread-block
+//               cluster, each reducing a contiguous range of K blocks.  After a
+//               cluster barrier (all rings drained) every thread pushes its fp32
+//               partial row chunks straight into the shared memory of the CTA
+//               that owns those rows (remote st.shared::cluster, fire and
+//               forget); after a second barrier each CTA sums the S received
+//               copies of its 128/S rows in rank order (deterministic) and
+//               stores coalesced rows.  Small-M projections thereby use wide,
+//               L2-friendly tiles, still fill the SMs, and split the epilogue.
+//     generic   (V part of the fused QKV projection, unaligned outputs): the
+//               fp32 tile is parked in shared memory and walked row by row
+//               (column by column for V, which is stored transposed per head)
+//               with coalesced stores.
+#include <cstring>
 
 #include "ptx.cuh"
 #include "w2v_internal.h"
@@ -25,88 +45,89 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
-  static constexpr int TMEM_COLS = BN;
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr int RING_MAX = 200 * 1024;
+  static constexpr int STAGES = (RING_MAX / STAGE) > 8 ? 8 : (RING_MAX / STAGE);
+  static constexpr int RING = STAGES * STAGE;
+  static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+  static constexpr int CHUNK = BN >= 64 ? 32 : 16;  // TMEM columns per load
+  static constexpr int ROW_CHUNKS = BN / 4;         // 16-byte fp32 chunks per row
+  static constexpr int BIAS_OFF = RING;
+  static constexpr int BAR_OFF = BIAS_OFF + BN * 4;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static_assert(BM * BN * 4 <= RING, "parked tile must fit in the operand ring");
+  static_assert(ROW_CHUNKS >= 8, "row swizzle needs >= 8 chunks");
 };
 
-__device__ __forceinline__ void store_chunk_f16(__half* dst, const float (&v)[32], int nvalid, bool vec) {
-  if (vec && nvalid >= 32) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-      uint4 u;
-      __half2 h0 = __floats2half2_rn(v[i + 0], v[i + 1]);
-      __half2 h1 = __floats2half2_rn(v[i + 2], v[i + 3]);
-      __half2 h2 = __floats2half2_rn(v[i + 4], v[i + 5]);
-      __half2 h3 = __floats2half2_rn(v[i + 6], v[i + 7]);
-      u.x = *reinterpret_cast<uint32_t*>(&h0);
-      u.y = *reinterpret_cast<uint32_t*>(&h1);
-      u.z = *reinterpret_cast<uint32_t*>(&h2);
-      u.w = *reinterpret_cast<uint32_t*>(&h3);
-      *reinterpret_cast<uint4*>(dst + i) = u;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (i < nvalid) dst[i] = __float2half_rn(v[i]);
-  }
+constexpr int kGemmThreads = 320;
+constexpr int kEpiThreads = 256;
+
+// fp32 tile rows of `row_chunks` 16-byte chunks; chunk j of row r lives at
+// chunk (j ^ (r & 7)) so that 8 consecutive rows hit 8 different bank groups.
+__device__ __forceinline__ uint32_t swz_off(int row_chunks, int r, int j) {
+  return static_cast<uint32_t>((r * row_chunks + (j ^ (r & 7))) * 16);
 }
 
-__device__ __forceinline__ void store_chunk_f32(float* dst, const float (&v)[32], int nvalid, bool vec) {
-  if (vec && nvalid >= 32) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (i < nvalid) dst[i] = v[i];
-  }
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void add_residual(float (&v)[32], const void* res, int res_f32, int nvalid, bool vec) {
-  if (res_f32) {
-    const float* r = static_cast<const float*>(res);
-    if (vec && nvalid >= 32) {
+// Final epilogue for 4 consecutive columns [col, col+4) of row grow: bias
+// (from shared memory), GELU, residual, store.  `vec` selects 16-/8-byte
+// accesses (row starts and pointers 16-byte aligned, full 4-vector in range).
+__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, int lcol, int grow, int col, int nv,
+                                        int bzb, const GemmEpilogue& e, void* outp, int ocol0, bool vec) {
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        float4 f = *reinterpret_cast<const float4*>(r + i);
-        v[i] += f.x; v[i + 1] += f.y; v[i + 2] += f.z; v[i + 3] += f.w;
+  for (int i = 0; i < 4; ++i) x[i] = apply_act(x[i] + bias_s[lcol + i], e.act);
+  if (e.residual) {
+    const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+    if (e.res_f32) {
+      const float* rp = static_cast<const float*>(e.residual) + roff;
+      if (vec && nv == 4) {
+        const float4 rv = *reinterpret_cast<const float4*>(rp);
+        x[0] += rv.x; x[1] += rv.y; x[2] += rv.z; x[3] += rv.w;
+      } else {
+        for (int i = 0; i < nv; ++i) x[i] += rp[i];
       }
     } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i < nvalid) v[i] += r[i];
-    }
-  } else {
-    const __half* r = static_cast<const __half*>(res);
-    if (vec && nvalid >= 32) {
-#pragma unroll
-      for (int i = 0; i < 32; i += 8) {
-        uint4 u = *reinterpret_cast<const uint4*>(r + i);
-        const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float2 f = __half22float2(h[j]);
-          v[i + 2 * j] += f.x;
-          v[i + 2 * j + 1] += f.y;
-        }
+      const __half* rp = static_cast<const __half*>(e.residual) + roff;
+      if (vec && nv == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(rp);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        x[0] += a.x; x[1] += a.y; x[2] += b.x; x[3] += b.y;
+      } else {
+        for (int i = 0; i < nv; ++i) x[i] += __half2float(rp[i]);
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i < nvalid) v[i] += __half2float(r[i]);
     }
+  }
+  const int64_t ooff = static_cast<int64_t>(bzb) * e.out_batch_stride + static_cast<int64_t>(grow) * e.ldo + (col - ocol0);
+  if (e.out_f32) {
+    float* op = static_cast<float*>(outp) + ooff;
+    if (vec && nv == 4)
+      *reinterpret_cast<float4*>(op) = make_float4(x[0], x[1], x[2], x[3]);
+    else
+      for (int i = 0; i < nv; ++i) op[i] = x[i];
+  } else {
+    __half* op = static_cast<__half*>(outp) + ooff;
+    if (vec && nv == 4)
+      *reinterpret_cast<uint2*>(op) = make_uint2(pack_h2(x[0], x[1]), pack_h2(x[2], x[3]));
+    else
+      for (int i = 0; i < nv; ++i) op[i] = __float2half_rn(x[i]);
   }
 }
 
+// mode: 0 generic, 1 direct (TMA store), 2 split-K
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmShape s,
-               GemmEpilogue e, int vec_ok, int* err) {
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2, GemmShape s,
+               GemmEpilogue e, int vec_ok, int mode, int* err) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
+  float* bias_s = reinterpret_cast<float*>(smem + C::BIAS_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
@@ -115,8 +136,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * C::BM;
   const int n0 = blockIdx.y * BN;
-  const int bz = blockIdx.z;
   const int nk = s.K / C::BK;
+  const int S = s.splits;
+  const int split = S > 1 ? static_cast<int>(blockIdx.z) : 0;
+  const int bzb = S > 1 ? 0 : static_cast<int>(blockIdx.z);  // batch index
+  const int kb0 = split * nk / S;
+  const int nkl = (split + 1) * nk / S - kb0;  // K blocks of this CTA (>= 1)
+  const int pre = nkl < C::STAGES ? nkl : C::STAGES;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
@@ -125,10 +151,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     mbar_init(accf, 1);
     fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
+    pdl_launch_dependents();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    // Weights do not depend on the previous kernel: start them right away.
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&full[i], C::STAGE);
+      tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, &full[i], (kb0 + i) * C::BK, n0);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -141,36 +171,41 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) {
+        const int k = (kb0 + i) * C::BK;
+        tma_load_3d(smem + i * C::STAGE, &tmA, &full[i], k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
+      }
+      int issued = pre;
       bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % C::STAGES;
-        const uint32_t ph = (kb / C::STAGES) & 1;
-        if (kb >= C::STAGES && !mbar_wait(&empty[st], ph ^ 1)) {
+      for (int i = pre; i < nkl; ++i) {
+        const int st = i % C::STAGES;
+        const uint32_t ph = (i / C::STAGES) & 1;
+        if (!mbar_wait(&empty[st], ph ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
           break;
         }
         uint8_t* sa = smem + st * C::STAGE;
         mbar_arrive_expect_tx(&full[st], C::STAGE);
-        const int k = kb * C::BK;
-        tma_load_3d(sa, &tmA, &full[st], k % s.a_kwrap, m0 + k / s.a_kwrap, bz);
+        const int k = (kb0 + i) * C::BK;
+        tma_load_3d(sa, &tmA, &full[st], k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
         tma_load_2d(sa + C::A_BYTES, &tmB, &full[st], k, n0);
-        issued = kb + 1;
+        issued = i + 1;
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA exits.
-        for (int kb = (issued > C::STAGES ? issued - C::STAGES : 0); kb < issued; ++kb)
-          mbar_wait(&full[kb % C::STAGES], (kb / C::STAGES) & 1);
+        for (int i = (issued > C::STAGES ? issued - C::STAGES : 0); i < issued; ++i)
+          mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, BN);
       bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % C::STAGES;
-        if (!mbar_wait(&full[st], (kb / C::STAGES) & 1)) {
+      for (int i = 0; i < nkl; ++i) {
+        const int st = i % C::STAGES;
+        if (!mbar_wait(&full[st], (i / C::STAGES) & 1)) {
           atomicOr(err, kErrWaitMma);
           ok = false;
           break;
@@ -180,86 +215,309 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16(tmem, desc_sw128(sa + kk * 32), desc_sw128(sb + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_f16(tmem, desc_sw128(sa + kk * 32), desc_sw128(sb + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
         umma_commit(&empty[st]);
       }
       if (ok) umma_commit(accf);
     }
-  } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;
-    bool ok = mbar_wait(accf, 0);
-    ok = __all_sync(0xffffffffu, ok);
+  }
+
+  const bool epi = warp >= 2;
+  const int et = threadIdx.x - 64;   // 0..255 for the epilogue warps
+  const int q = warp & 3;            // TMEM lane quarter this warp may access
+  const int half = (warp - 2) >> 2;  // which half of the columns
+  const int r = q * 32 + lane;       // tile row of this thread in pass 1
+  const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  const int region = e.qkv_d > 0 ? n0 / e.qkv_d : -1;
+  const bool vec = vec_ok != 0;
+  bool ok = true;
+  if (epi) {
+    for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (e.bias && n0 + i < s.N) ? e.bias[n0 + i] : 0.f;
+    ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
     if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
     tc_fence_after();
-    if (ok) {
-      const int row = m0 + r;
-      const bool row_ok = row < s.M;
-      const int64_t orow = static_cast<int64_t>(bz) * e.out_batch_stride + static_cast<int64_t>(row) * e.ldo;
+  }
+
+  if (mode == 1 && region == 2) mode = 0;  // V tiles: transposed, generic path
+  if (mode == 1) {
+    // ------------------------------------------------------------- direct
+    if (epi) {
+      named_barrier_sync(1, kEpiThreads);  // bias staged
+      const int grow = m0 + r;
+      void* outp = region == 1 ? e.out_k : e.out;
+      const int ocol0 = region > 0 ? region * e.qkv_d : 0;
+      const CUtensorMap* om = region == 1 ? &tmO2 : &tmO;
+      // Staging: this warp's boxes of 32 rows x 32 columns, 4 KB apart.
+      uint8_t* stage = smem + (warp - 2) * (BN / 2 / 32) * 4096;
+      int nbox = 0;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
         float v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, v);
-        const int nc = n0 + c;
-        if (nc >= s.N || !row_ok) continue;
-        const int nvalid = min(32, s.N - nc);
-        if (e.bias) {
+        if (ok) tmem_ld32(trow + c, v);
+        const int col = n0 + c;
+        if (e.residual && grow < s.M) {
+          const int64_t roff =
+              static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+          const int nv = min(32, s.N - col);
+          if (e.res_f32) {
+            const float* rp = static_cast<const float*>(e.residual) + roff;
+            if (nv == 32) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nvalid) v[i] += __ldg(e.bias + nc + i);
-        }
-        if (e.act) {
+              for (int i = 0; i < 32; i += 4) {
+                const float4 rv = *reinterpret_cast<const float4*>(rp + i);
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + rv.x;
+                v[i + 1] = apply_act(v[i + 1] + bias_s[c + i + 1], e.act) + rv.y;
+                v[i + 2] = apply_act(v[i + 2] + bias_s[c + i + 2], e.act) + rv.z;
+                v[i + 3] = apply_act(v[i + 3] + bias_s[c + i + 3], e.act) + rv.w;
+              }
+            } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i], e.act);
-        }
-        if (e.residual) {
-          const int64_t roff = static_cast<int64_t>(bz) * e.res_batch_stride + static_cast<int64_t>(row) * e.ldr + nc;
-          const void* rp = e.res_f32 ? static_cast<const void*>(static_cast<const float*>(e.residual) + roff)
-                                     : static_cast<const void*>(static_cast<const __half*>(e.residual) + roff);
-          add_residual(v, rp, e.res_f32, nvalid, vec_ok != 0);
-        }
-        if (e.qkv_d > 0) {
-          const int region = nc / e.qkv_d;
-          const int cc = nc - region * e.qkv_d;
-          if (region == 0) {
-            store_chunk_f16(static_cast<__half*>(e.out) + orow + cc, v, nvalid, vec_ok != 0);
-          } else if (region == 1) {
-            store_chunk_f16(static_cast<__half*>(e.out_k) + orow + cc, v, nvalid, vec_ok != 0);
+              for (int i = 0; i < 32; ++i)
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + (i < nv ? rp[i] : 0.f);
+            }
           } else {
-            // rows are clip-major: row = clip * t_len + t
-            const int clip = row / e.t_len;
-            const int t = row - clip * e.t_len;
-            const int h = cc >> 6;
-            const int dd0 = cc & 63;
-            __half* dst = static_cast<__half*>(e.vt) +
-                          (static_cast<int64_t>(clip * e.n_heads + h) * 64 + dd0) * e.t_pad + t;
+            const __half* rp = static_cast<const __half*>(e.residual) + roff;
+            if (nv == 32) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(v[i]);
+              for (int i = 0; i < 32; i += 8) {
+                const uint4 u = *reinterpret_cast<const uint4*>(rp + i);
+                const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float2 f = __half22float2(h[k]);
+                  v[i + 2 * k] = apply_act(v[i + 2 * k] + bias_s[c + i + 2 * k], e.act) + f.x;
+                  v[i + 2 * k + 1] = apply_act(v[i + 2 * k + 1] + bias_s[c + i + 2 * k + 1], e.act) + f.y;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + (i < nv ? __half2float(rp[i]) : 0.f);
+            }
           }
-        } else if (e.out_f32) {
-          store_chunk_f32(static_cast<float*>(e.out) + orow + nc, v, nvalid, vec_ok != 0);
         } else {
-          store_chunk_f16(static_cast<__half*>(e.out) + orow + nc, v, nvalid, vec_ok != 0);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i] + bias_s[c + i], e.act);
+        }
+        uint8_t* box = stage + nbox * 4096;
+        if (e.out_f32) {
+          // 128-byte rows, 128-byte swizzle: chunk k of row lane at k ^ (lane & 7)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(box + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        } else {
+          // 64-byte rows, 64-byte swizzle: chunk k of row lane at k ^ ((lane >> 1) & 3)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pack_h2(v[8 * k], v[8 * k + 1]), pack_h2(v[8 * k + 2], v[8 * k + 3]),
+                           pack_h2(v[8 * k + 4], v[8 * k + 5]), pack_h2(v[8 * k + 6], v[8 * k + 7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && ok && col < s.N) tma_store_3d(om, box, col - ocol0, m0 + q * 32, bzb);
+        ++nbox;
+      }
+      if (lane == 0) {
+        bulk_commit_group();
+        bulk_wait_all();
+      }
+      (void)outp;
+    }
+    tc_fence_before();
+    __syncthreads();
+  } else if (mode == 2) {
+    // ------------------------------------------------------------ split-K
+    const int rows_max = (C::BM + S - 1) / S;
+    const uint32_t slot_bytes = static_cast<uint32_t>(rows_max) * C::ROW_CHUNKS * 16;
+    const int rank = static_cast<int>(cluster_ctarank());
+    cluster_sync();  // every accumulator of the cluster is final: all rings are free
+    if (epi && ok) {
+      // Rows [o*128/S, (o+1)*128/S) belong to cluster CTA o.
+      const int owner = ((r + 1) * S + C::BM - 1) / C::BM - 1;
+      const int lrow = r - owner * C::BM / S;
+      const uint32_t dst0 = mapa_shared(smem_u32(smem) + rank * slot_bytes, owner);
+#pragma unroll 1
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += C::CHUNK) {
+        float v[32];
+        if (C::CHUNK == 32) {
+          tmem_ld32(trow + c, v);
+        } else {
+          float w[16];
+          tmem_ld16(trow + c, w);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = w[i];
+        }
+#pragma unroll
+        for (int i = 0; i < C::CHUNK; i += 4)
+          st_dsmem_f4(dst0 + swz_off(C::ROW_CHUNKS, lrow, (c + i) >> 2), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+      }
+    }
+    tc_fence_before();
+    cluster_sync();  // every partial has landed in its owner's shared memory
+    if (epi && ok) {
+      const int r0 = rank * C::BM / S;
+      const int nrows = (rank + 1) * C::BM / S - r0;
+      auto fetch = [&](int lr, int j) -> float4 {
+        float4 a = *reinterpret_cast<const float4*>(smem + swz_off(C::ROW_CHUNKS, lr, j));
+        for (int p = 1; p < S; ++p) {
+          const float4 b = *reinterpret_cast<const float4*>(smem + p * slot_bytes + swz_off(C::ROW_CHUNKS, lr, j));
+          a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        return a;
+      };
+      if (region == 2) {
+        const int total = nrows * C::ROW_CHUNKS;
+#pragma unroll 1
+        for (int idx = et; idx < total; idx += kEpiThreads) {
+          const int j = idx / nrows;
+          const int lr = idx - j * nrows;
+          const int grow = m0 + r0 + lr;
+          const int col = n0 + 4 * j;
+          if (grow >= s.M || col >= s.N) continue;
+          const float4 v = fetch(lr, j);
+          const float x[4] = {v.x, v.y, v.z, v.w};
+          const int cc = col - 2 * e.qkv_d;
+          const int clip = grow / e.t_len;
+          const int t = grow - clip * e.t_len;
+          __half* dst = static_cast<__half*>(e.vt) +
+                        (static_cast<int64_t>(clip * e.n_heads + (cc >> 6)) * 64 + (cc & 63)) * e.t_pad + t;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(apply_act(x[i] + bias_s[4 * j + i], e.act));
+        }
+      } else {
+        void* outp = region == 1 ? e.out_k : e.out;
+        const int ocol0 = region > 0 ? region * e.qkv_d : 0;
+        const int total = nrows * C::ROW_CHUNKS;
+#pragma unroll 2
+        for (int idx = et; idx < total; idx += kEpiThreads) {
+          const int lr = idx / C::ROW_CHUNKS;
+          const int j = idx - lr * C::ROW_CHUNKS;
+          const int grow = m0 + r0 + lr;
+          const int col = n0 + 4 * j;
+          if (grow >= s.M || col >= s.N) continue;
+          const float4 v = fetch(lr, j);
+          float x[4] = {v.x, v.y, v.z, v.w};
+          finish4(x, bias_s, 4 * j, grow, col, min(4, s.N - col), bzb, e, outp, ocol0, vec);
         }
       }
     }
+    tc_fence_before();
+    __syncthreads();
+  } else {
+    // ------------------------------------------------------------ generic
+    uint8_t* park = smem;
+    if (epi && ok) {
+#pragma unroll 1
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += C::CHUNK) {
+        float v[32];
+        if (C::CHUNK == 32) {
+          tmem_ld32(trow + c, v);
+        } else {
+          float w[16];
+          tmem_ld16(trow + c, w);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = w[i];
+        }
+#pragma unroll
+        for (int i = 0; i < C::CHUNK; i += 4)
+          *reinterpret_cast<float4*>(park + swz_off(C::ROW_CHUNKS, r, (c + i) >> 2)) =
+              make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (epi && ok) {
+      const int total = C::BM * C::ROW_CHUNKS;
+      if (region == 2) {
+#pragma unroll 1
+        for (int idx = et; idx < total; idx += kEpiThreads) {
+          const int j = idx / C::BM;
+          const int rr = idx - j * C::BM;
+          const int grow = m0 + rr;
+          const int col = n0 + 4 * j;
+          if (grow >= s.M || col >= s.N) continue;
+          const float4 v = *reinterpret_cast<const float4*>(park + swz_off(C::ROW_CHUNKS, rr, j));
+          const float x[4] = {v.x, v.y, v.z, v.w};
+          const int cc = col - 2 * e.qkv_d;
+          const int clip = grow / e.t_len;
+          const int t = grow - clip * e.t_len;
+          __half* dst = static_cast<__half*>(e.vt) +
+                        (static_cast<int64_t>(clip * e.n_heads + (cc >> 6)) * 64 + (cc & 63)) * e.t_pad + t;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(apply_act(x[i] + bias_s[4 * j + i], e.act));
+        }
+      } else {
+        void* outp = region == 1 ? e.out_k : e.out;
+        const int ocol0 = region > 0 ? region * e.qkv_d : 0;
+#pragma unroll 2
+        for (int idx = et; idx < total; idx += kEpiThreads) {
+          const int rr = idx / C::ROW_CHUNKS;
+          const int j = idx - rr * C::ROW_CHUNKS;
+          const int grow = m0 + rr;
+          const int col = n0 + 4 * j;
+          if (grow >= s.M || col >= s.N) continue;
+          const float4 v = *reinterpret_cast<const float4*>(park + swz_off(C::ROW_CHUNKS, rr, j));
+          float x[4] = {v.x, v.y, v.z, v.w};
+          finish4(x, bias_s, 4 * j, grow, col, min(4, s.N - col), bzb, e, outp, ocol0, vec);
+        }
+      }
+    }
+    __syncthreads();
   }
 
-  tc_fence_before();
-  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-int gemm_pick_bn(const GemmShape& s) {
-  if (s.N <= 32) return 32;
-  if (s.N <= 64) return 64;
-  const long mt = static_cast<long>((s.M + 127) / 128) * s.batch;
-  if (mt * ((s.N + 255) / 256) >= 148) return 256;
-  if (mt * ((s.N + 127) / 128) >= 100) return 128;
-  return 64;
+// Tile width and split-K factor: the candidate whose launch should finish
+// first under a simple model of this kernel on B200 (148 SMs):
+//  * MMA time per CTA: per 64-deep K block the larger of the MMA time
+//    (2*BN cycles for M=128) and the shared-memory operand reads
+//    ((16 KB + BN*128 B) at 128 B/cycle), times waves of CTAs;
+//  * operand delivery: every CTA streams its A and B blocks from L2; the
+//    measured aggregate L2->SM throughput of these kernels is ~4.6 KB/cycle
+//    (~8.8 TB/s) and one SM takes in at most ~110 B/cycle, so both the total
+//    and the per-CTA operand bytes give floors;
+//  * fixed costs: set-up, the epilogue (split S ways), the cluster reduction.
+int gemm_pick(GemmShape* s, int bn_divides) {
+  const int cands[] = {32, 64, 128, 192, 256};
+  const int splits[] = {1, 2, 3, 4, 6, 8};
+  const long mt = static_cast<long>((s->M + 127) / 128) * s->batch;
+  const long nk = s->K / 64;
+  int best_bn = 64, best_s = 1;
+  double best_t = 1e30;
+  for (int bn : cands) {
+    if (bn > 32 && s->N <= bn / 2) continue;  // much wider than N: wasted MMA columns
+    if (bn_divides > 0 && bn_divides % bn != 0) continue;
+    const long tiles = mt * ((s->N + bn - 1) / bn);
+    for (int sp : splits) {
+      if (sp > 1 && (s->batch != 1 || sp > nk)) continue;
+      const long ctas = tiles * sp;
+      const long waves = (ctas + 147) / 148;
+      const long nkl = (nk + sp - 1) / sp;
+      const double per_k = (2.0 * bn > 128.0 + bn) ? 2.0 * bn : 128.0 + bn;
+      const double t_mma = waves * nkl * per_k;
+      const double t_l2 = static_cast<double>(ctas) * nkl * (128.0 + bn) * 128.0 / 4600.0;
+      const double t_sm = waves * nkl * (128.0 + bn) * 128.0 / 110.0;
+      double t_max = t_mma > t_l2 ? t_mma : t_l2;
+      if (t_sm > t_max) t_max = t_sm;
+      const double t = t_max + 2000.0 + waves * (600.0 + 6.0 * bn / sp) +
+                       (sp > 1 ? 800.0 + 150.0 * sp : 0.0);
+      if (t < best_t - 1e-9) {
+        best_t = t;
+        best_bn = bn;
+        best_s = sp;
+      }
+    }
+  }
+  s->splits = best_s;
+  return best_bn;
 }
 
 template <int BN>
@@ -268,40 +526,83 @@ static cudaError_t prepare_bn() {
 }
 
 cudaError_t gemm_prepare() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaSuccess) return done;
   cudaError_t r;
   if ((r = prepare_bn<32>()) != cudaSuccess) return r;
   if ((r = prepare_bn<64>()) != cudaSuccess) return r;
   if ((r = prepare_bn<128>()) != cudaSuccess) return r;
-  return prepare_bn<256>();
+  if ((r = prepare_bn<192>()) != cudaSuccess) return r;
+  done = prepare_bn<256>();
+  return done;
 }
 
 template <int BN>
-static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s,
-                             const GemmEpilogue& e, int vec_ok, int* err, cudaStream_t st) {
+static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmO,
+                             const CUtensorMap& tmO2, const GemmShape& s, const GemmEpilogue& e, int vec_ok, int mode,
+                             int* err, cudaStream_t st) {
   using C = GemmCfg<BN>;
-  dim3 grid((s.M + 127) / 128, (s.N + BN - 1) / BN, s.batch);
-  gemm_tc_kernel<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmB, s, e, vec_ok, err);
-  return cudaGetLastError();
+  const int S = s.splits;
+  dim3 grid((s.M + 127) / 128, (s.N + BN - 1) / BN, S > 1 ? S : s.batch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = S > 1 ? S : 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, tmA, tmB, tmO, tmO2, s, e, vec_ok, mode, err);
 }
 
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
                         const GemmEpilogue& e, int* err, cudaStream_t st) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0) return cudaSuccess;
   if (s.K <= 0 || s.K % 64 != 0 || s.a_kwrap <= 0 || s.a_kwrap % 64 != 0) return cudaErrorInvalidValue;
-  // Vector loads/stores need 16-byte aligned rows and column offsets.
+  if (s.splits < 1 || s.splits > 8 || s.splits > s.K / 64 || (s.splits > 1 && s.batch != 1))
+    return cudaErrorInvalidValue;
+  if (e.qkv_d > 0 && (e.qkv_d % bn != 0 || s.N != 3 * e.qkv_d || e.t_len <= 0)) return cudaErrorInvalidValue;
+  // Vector loads/stores need 16-byte aligned bases and 4-element-aligned rows.
   const int esz_out = e.out_f32 ? 4 : 2;
   const int esz_res = e.res_f32 ? 4 : 2;
-  bool vec = (reinterpret_cast<uintptr_t>(e.out) % 16 == 0) && ((e.ldo * esz_out) % 16 == 0) &&
+  bool vec = (reinterpret_cast<uintptr_t>(e.out) % 16 == 0) && (e.ldo % 4 == 0) &&
              ((e.out_batch_stride * esz_out) % 16 == 0);
   if (e.residual)
-    vec = vec && (reinterpret_cast<uintptr_t>(e.residual) % 16 == 0) && ((e.ldr * esz_res) % 16 == 0) &&
+    vec = vec && (reinterpret_cast<uintptr_t>(e.residual) % 16 == 0) && (e.ldr % 4 == 0) &&
           ((e.res_batch_stride * esz_res) % 16 == 0);
   if (e.qkv_d > 0) vec = vec && (reinterpret_cast<uintptr_t>(e.out_k) % 16 == 0);
+  // Direct (TMA-store) epilogue: rows must be 16-byte multiples and any
+  // residual vector-loadable; tiles at least 64 wide.
+  CUtensorMap tmO, tmO2;
+  std::memset(&tmO, 0, sizeof tmO);
+  std::memset(&tmO2, 0, sizeof tmO2);
+  int mode = s.splits > 1 ? 2 : 0;
+  const bool tma_ok = s.splits == 1 && bn >= 64 && vec && (e.ldo * esz_out) % 16 == 0 &&
+                      (e.residual == nullptr || (e.ldr * esz_res) % 16 == 0);
+  if (tma_ok) {
+    const uint64_t cols = e.qkv_d > 0 ? static_cast<uint64_t>(e.qkv_d) : static_cast<uint64_t>(s.N);
+    const uint64_t dims[3] = {cols, static_cast<uint64_t>(s.M), static_cast<uint64_t>(s.batch)};
+    const uint64_t bstride = s.batch > 1 ? static_cast<uint64_t>(e.out_batch_stride) * esz_out
+                                         : static_cast<uint64_t>(s.M) * e.ldo * esz_out;
+    const uint64_t str[2] = {static_cast<uint64_t>(e.ldo) * esz_out, bstride};
+    const uint32_t box[3] = {32, 32, 1};
+    const int swz = e.out_f32 ? 128 : 64;
+    bool built = make_tmap(&tmO, e.out, 3, dims, str, box, esz_out, swz) == cudaSuccess;
+    if (built && e.qkv_d > 0) built = make_tmap(&tmO2, e.out_k, 3, dims, str, box, esz_out, swz) == cudaSuccess;
+    if (built) mode = 1;
+  }
   switch (bn) {
-    case 32: return launch_bn<32>(tmA, tmB, s, e, vec, err, st);
-    case 64: return launch_bn<64>(tmA, tmB, s, e, vec, err, st);
-    case 128: return launch_bn<128>(tmA, tmB, s, e, vec, err, st);
-    case 256: return launch_bn<256>(tmA, tmB, s, e, vec, err, st);
+    case 32: return launch_bn<32>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
+    case 64: return launch_bn<64>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
+    case 128: return launch_bn<128>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
+    case 192: return launch_bn<192>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
+    case 256: return launch_bn<256>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
     default: return cudaErrorInvalidValue;
   }
 }

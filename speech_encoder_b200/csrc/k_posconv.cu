@@ -63,6 +63,7 @@ posconv_kernel(const __grid_constant__ CUtensorMap tmX, const __half* __restrict
     mbar_init(a_full, 1);
     mbar_init(accf, 1);
     fence_mbar_init();
+    pdl_launch_dependents();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmX);
   if (warp == 1) {
@@ -76,15 +77,22 @@ posconv_kernel(const __grid_constant__ CUtensorMap tmX, const __half* __restrict
 
   if (warp == 0) {
     if (lane == 0) {
+      const uint8_t* wg = reinterpret_cast<const uint8_t*>(wpack) + static_cast<int64_t>(g) * kPosK * C::TAP_BYTES;
+      // Weights first (independent of the previous kernel), then the window.
+      const int pre = C::ITERS < C::STAGES ? C::ITERS : C::STAGES;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&full[it], C::STAGE);
+        bulk_load(sB + it * C::STAGE, wg + static_cast<int64_t>(it) * C::STAGE, C::STAGE, &full[it]);
+      }
+      pdl_wait();
       mbar_arrive_expect_tx(a_full, C::A_BYTES);
 #pragma unroll
       for (int c = 0; c < C::KCH; ++c) tma_load_3d(sA + c * kWin * 16, &tmX, a_full, g * MG + 8 * c, t0 - 64, b);
-      const uint8_t* wg = reinterpret_cast<const uint8_t*>(wpack) + static_cast<int64_t>(g) * kPosK * C::TAP_BYTES;
-      int issued = 0;
+      int issued = pre;
       bool ok = true;
-      for (int it = 0; it < C::ITERS; ++it) {
+      for (int it = pre; it < C::ITERS; ++it) {
         const int st = it % C::STAGES;
-        if (it >= C::STAGES && !mbar_wait(&empty[st], ((it / C::STAGES) & 1) ^ 1)) {
+        if (!mbar_wait(&empty[st], ((it / C::STAGES) & 1) ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
           break;
@@ -187,8 +195,7 @@ static cudaError_t launch_mg(const CUtensorMap& tmX, const __half* x, const __ha
                              int batch, int d, int act, float* h, int* err, cudaStream_t st) {
   using C = PosCfg<MG>;
   dim3 grid((T + 127) / 128, 16, batch);
-  posconv_kernel<MG><<<grid, 192, C::SMEM, st>>>(tmX, x, wpack, bias, T, d, act, h, err);
-  return cudaGetLastError();
+  return launch_pdl(posconv_kernel<MG>, grid, dim3(192), C::SMEM, st, tmX, x, wpack, bias, T, d, act, h, err);
 }
 
 cudaError_t launch_posconv(const CUtensorMap& tmX, const __half* x, const __half* wpack, const float* bias, int T,

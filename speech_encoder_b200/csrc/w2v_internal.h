@@ -8,12 +8,35 @@
 
 namespace w2v {
 
+// Launches a kernel with programmatic dependent launch enabled: it may begin
+// (set-up, weight prefetch) while the previous kernel on the stream drains,
+// and waits in-kernel (griddepcontrol.wait) before reading that kernel's
+// outputs.  Recorded as programmatic edges when captured into a CUDA graph.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- tensor maps
 // Encodes a tiled TMA descriptor for a row-major fp16 tensor with up to 3
 // dimensions (dims[0] innermost).  strides_bytes[i] is the stride of dims[i+1].
 // Returns cudaSuccess or an error (bad alignment, driver entry point missing).
 cudaError_t make_tmap_f16(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
                           const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+// Same for fp16 (elem_bytes 2) or fp32 (4) with a 0/32/64/128-byte swizzle.
+cudaError_t make_tmap(CUtensorMap* out, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                      const uint32_t* box, int elem_bytes, int swizzle_bytes);
 
 // ----------------------------------------------------------------------- GEMM
 // D = A * B^T over fp16 operands with fp32 accumulation on tcgen05 and a fused
@@ -49,11 +72,16 @@ struct GemmShape {
   int K = 0;        // multiple of 64
   int a_kwrap = 0;  // see above
   int batch = 1;
+  int splits = 1;   // split-K factor (batch must be 1 when > 1): the splits of
+                    // one output tile form a thread-block cluster and reduce
+                    // their fp32 partials through distributed shared memory
 };
 
-// Chooses the N tile and launches.  tmA: {cols, rows, batch}, box {64,128,1};
-// tmB: {K, N}, box {64, bn} where bn = gemm_pick_bn(...).
-int gemm_pick_bn(const GemmShape& s);
+// Chooses the N tile width (returned) and the split-K factor (s->splits) for
+// this shape.  bn_divides > 0 restricts the width to divisors of it (the fused
+// QKV projection needs tiles that do not straddle Q/K/V).
+// tmA: {cols, rows, batch}, box {64,128,1}; tmB: {K, N}, box {64, bn}.
+int gemm_pick(GemmShape* s, int bn_divides);
 // Raise the dynamic shared-memory limits of the tcgen05 kernels (idempotent;
 // called before any launch or stream capture).
 cudaError_t gemm_prepare();
@@ -63,14 +91,20 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
                         const GemmEpilogue& e, int* err, cudaStream_t st);
 
 // ------------------------------------------------------------------ frontend
-// Group layout: per-clip first and second moments of the conv-0 input windows
-// (10 taps, hop 5) accumulated into acc[b][65] (fp64; must be zero on entry).
-cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, double* acc, cudaStream_t st);
+// Group layout: GroupNorm statistics of conv layer 0 from the moments of its
+// 10-sample input windows.  Writes scale_shift[b][512] = (gamma/sigma,
+// beta - mean*gamma/sigma).  partial: [batch][gn_moment_blocks(t0)][65] fp64
+// scratch; ticket: [batch] counters that must be zero before the first call
+// (the kernel leaves them zero).
+int gn_moment_blocks(int t0);
+cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, const float* w0, const float* gamma,
+                              const float* beta, float eps, double* partial, unsigned* ticket, float2* scale_shift,
+                              cudaStream_t st);
 // conv0 + norm + GELU -> fp16 [batch][clip_rows][512] (rows >= t0 untouched).
-//   group layout: per-channel GroupNorm from acc (over all t0 frames),
+//   group layout: per-channel scale/shift from launch_gn_moments,
 //   layer layout: conv bias, per-frame LayerNorm over the 512 channels.
 cudaError_t launch_conv0(const float* pcm, int n, int batch, int t0, int clip_rows, const float* w0, const float* b0,
-                         const float* gamma, const float* beta, const double* acc, int layer_norm, float eps,
+                         const float* gamma, const float* beta, const float2* scale_shift, int layer_norm, float eps,
                          int act, __half* out, cudaStream_t st);
 // Row LayerNorm over `cols` channels (512, 768 or 1024), fp16 or fp32 input,
 // fp16 output, optional GELU after the affine.
@@ -96,6 +130,9 @@ cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, con
 cudaError_t launch_argmax(const float* logits, int rows, int V, int32_t* ids, cudaStream_t st);
 cudaError_t launch_ctc_collapse(const int32_t* ids, int batch, int T, int t_valid, int blank, int32_t* tokens,
                                 int32_t* n_tokens, cudaStream_t st);
+
+// Holds the stream for `ns` nanoseconds (<= 0.1 s).
+cudaError_t launch_stream_gate(uint64_t ns, cudaStream_t st);
 
 // A kernel whose bounded wait runs out on purpose (nothing ever arrives on its
 // barrier); it records kErrTest in *err and returns.

@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
         "w2v_last_launch_count": (I, [VP]),
         "w2v_kernel_class_name": (ctypes.c_char_p, [I]),
         "w2v_profile_forward": (I, [VP, VP, I, I, VP, VP, ctypes.POINTER(w2v_kernel_time), I, ctypes.POINTER(I)]),
-        "w2v_op_gemm": (I, [VP, VP, I, I, I, VP, VP, I, VP, I, I, I, VP, VP]),
+        "w2v_op_gemm": (I, [VP, VP, I, I, I, VP, VP, I, VP, I, I, I, I, VP, VP]),
         "w2v_op_attention": (I, [VP, VP, VP, VP, I, I, I, I, VP, VP]),
         "w2v_op_layernorm": (I, [VP, I, VP, I, I, VP, VP, ctypes.c_float, I, VP]),
         "w2v_op_wait_probe": (I, [VP, ctypes.c_uint64, VP]),
@@ -214,9 +214,9 @@ def w2v_destroy(model: int) -> None:
         lib().w2v_destroy(model)
 
 
-def w2v_op_gemm(A, B, M, N, K, bias, residual, res_f32, out, out_f32, act, err, bn=0, stream=None) -> int:
+def w2v_op_gemm(A, B, M, N, K, bias, residual, res_f32, out, out_f32, act, err, bn=0, splits=1, stream=None) -> int:
     return lib().w2v_op_gemm(_ptr(A), _ptr(B), M, N, K, _ptr(bias), _ptr(residual), res_f32, _ptr(out), out_f32,
-                             act, bn, _ptr(err), _stream(stream))
+                             act, bn, splits, _ptr(err), _stream(stream))
 
 
 def w2v_op_attention(q, k, vt, out, batch, T, H, t_pad, err, stream=None) -> int:

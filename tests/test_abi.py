@@ -85,7 +85,7 @@ def test_blob_size_mismatch_and_null_args():
     assert L.w2v_sync(None, None) == B.W2V_EINVAL
     L.w2v_destroy(None)
     err = np.zeros(1, np.int32)
-    assert L.w2v_op_gemm(None, None, 1, 1, 64, None, None, 0, None, 0, 0, 0, None, None) == B.W2V_EINVAL
+    assert L.w2v_op_gemm(None, None, 1, 1, 64, None, None, 0, None, 0, 0, 0, 1, None, None) == B.W2V_EINVAL
     assert L.w2v_op_wait_probe(None, 1000, None) == B.W2V_EINVAL
     assert L.w2v_op_layernorm(None, 0, None, 1, 512, None, None, 1e-5, 0, None) == B.W2V_EINVAL
 

@@ -21,7 +21,7 @@ def _act_ref(x, act):
 
 
 GEMM_CASES = [
-    # M, N, K, bn, act, residual, out_f32
+    # M, N, K, bn, act, residual, out_f32  (bn may be (bn, splits))
     (128, 64, 64, 64, 0, None, 0),
     (1, 32, 64, 32, 0, None, 0),
     (130, 96, 128, 64, 1, None, 0),
@@ -34,11 +34,19 @@ GEMM_CASES = [
     (7984, 768, 768, 256, 0, "f16", 1),
     (49, 32, 768, 32, 0, None, 1),
     (200, 200, 192, 128, 1, "f32", 0),
+    (799, 768, 3072, (256, 3), 0, "f16", 1),
+    (799, 768, 3072, (256, 6), 0, "f32", 1),
+    (799, 2304, 768, (256, 2), 1, None, 0),
+    (799, 768, 768, (128, 4), 0, "f32", 1),
+    (130, 96, 512, (64, 8), 2, None, 0),
+    (1, 2341, 1024, (256, 5), 0, None, 1),
+    (799, 512, 1024, (192, 3), 1, "f16", 0),
 ]
 
 
 @pytest.mark.parametrize("M,N,K,bn,act,res,out_f32", GEMM_CASES)
 def test_gemm_matches_fp64(M, N, K, bn, act, res, out_f32):
+    bn, splits = bn if isinstance(bn, tuple) else (bn, 1)
     g = torch.Generator().manual_seed(M * 7 + N * 13 + K)
     A = (torch.rand(M, K, generator=g) * 2 - 1).half()
     W = ((torch.rand(N, K, generator=g) * 2 - 1) / np.sqrt(K) * 2).half()
@@ -53,7 +61,7 @@ def test_gemm_matches_fp64(M, N, K, bn, act, res, out_f32):
     out = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.float16, device="cuda")
     err = _err()
     rc = B.w2v_op_gemm(A.cuda(), W.cuda(), M, N, K, bias.cuda(), None if resid is None else resid.cuda(),
-                       1 if res == "f32" else 0, out, out_f32, act, err, bn=bn)
+                       1 if res == "f32" else 0, out, out_f32, act, err, bn=bn, splits=splits)
     assert rc == 0
     torch.cuda.synchronize()
     assert int(err.item()) == 0
@@ -69,9 +77,9 @@ def test_gemm_every_tile_width_same_result():
     A = torch.randn(M, K, generator=g).half().cuda()
     W = (torch.randn(N, K, generator=g) * 0.05).half().cuda()
     outs = []
-    for bn in (32, 64, 128, 256):
+    for bn, sp in ((32, 1), (64, 1), (128, 1), (192, 1), (256, 1), (256, 2), (128, 8), (64, 3)):
         out = torch.empty(M, N, dtype=torch.float32, device="cuda")
-        assert B.w2v_op_gemm(A, W, M, N, K, None, None, 0, out, 1, 0, _err(), bn=bn) == 0
+        assert B.w2v_op_gemm(A, W, M, N, K, None, None, 0, out, 1, 0, _err(), bn=bn, splits=sp) == 0
         outs.append(out)
     torch.cuda.synchronize()
     ref = A.double().cpu().numpy() @ W.double().cpu().numpy().T
