@@ -196,6 +196,16 @@ const char* w2v_kernel_class_name(int klass);
 int w2v_profile_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, void* stream,
                         w2v_kernel_time* out, int max_out, int* n_out);
 
+/* Per-launch device time of one kernel class: records `reps` passes of only
+ * that class's launches of a forward of this shape (inputs as the buffers
+ * hold them) as one CUDA graph, replays it once to warm up, times one replay
+ * with CUDA events on `stream` and divides by the number of launches.  Also
+ * returns the launches per forward and the algorithmic FLOPs and bytes per
+ * launch.  Synchronises the stream. */
+int w2v_time_class(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, int klass,
+                   int reps, float* us_per_launch, int* launches, double* flops_per_launch, double* bytes_per_launch,
+                   void* stream);
+
 /* Copies the last error message into buf (NUL-terminated). */
 int w2v_last_error(w2v_model* m, char* buf, size_t len);
 

@@ -2,7 +2,7 @@
 // window, as the LiteRT wav2vec2 discussion's fourth GPU rewrite leaves it),
 // head dim 64, scale 1/8, fused flash-style on tcgen05.
 //
-// One CTA per (128-query tile, head, clip), 320 threads:
+// One CTA per (128-query tile, head, clip), 576 threads:
 //   warp 0      TMA: the Q tile once, then K and V^T tiles of 128 keys into a
 //               2-deep ring
 //   warp 1      TMEM owner; one thread issues S_j = Q K_j^T (M=128, N=128,
@@ -10,10 +10,10 @@
 //               shared memory, O_j = P_j V_j (M=128, N=64, K=128).  S_{j+1} is
 //               issued before waiting for P_j, so the next scores are computed
 //               while the softmax of the current tile runs.
-//   warps 2-9   softmax: two warps per TMEM lane quarter, each owning half of
-//               the 128 key columns (and half of the 64 output columns) of its
+//   warps 2-17  softmax: four warps per TMEM lane quarter, each owning 32 of
+//               the 128 key columns (and 16 of the 64 output columns) of its
 //               32 query rows.  Row maxima and sums are combined through shared
-//               memory with a 64-thread named barrier per pair.  fp32 online
+//               memory with a 128-thread named barrier per quarter.  fp32 online
 //               softmax with exp2 (1/8 scale folded in), P rounded to fp16
 //               into the 128-byte-swizzled K-major layout the MMA reads, O
 //               accumulated in registers with the running rescale.
@@ -30,15 +30,19 @@ struct AttnSmem {
   static constexpr int K0 = 16384;
   static constexpr int V0 = K0 + 2 * 16384;
   static constexpr int P = V0 + 2 * 16384;
-  static constexpr int RED = P + 32768;       // float red_max[2][2][128], red_sum[2][128]
-  static constexpr int BAR = RED + 4096;
+  static constexpr int RED = P + 32768;       // float red_max[2][4][128], red_sum[4][128]
+  static constexpr int BAR = RED + 6144;
   static constexpr int TOTAL = BAR + 256 + 1024;
 };
 
-constexpr int kAttnThreads = 320;
+constexpr int kSoftWarps = 16;
+constexpr int kAttnThreads = 64 + 32 * kSoftWarps;
+constexpr int kSubs = kSoftWarps / 4;    // warps per TMEM lane quarter
+constexpr int kSCols = 128 / kSubs;      // score columns per warp
+constexpr int kOCols = 64 / kSubs;       // output columns per warp
 
-__device__ __forceinline__ void pair_barrier(int q) {
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+__device__ __forceinline__ void quarter_barrier(int q) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kSubs) : "memory");
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -46,8 +50,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmVt, int T, int H, __half* __restrict__ out, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* red_max = reinterpret_cast<float*>(smem + AttnSmem::RED);  // [slot][half][row]
-  float* red_sum = red_max + 2 * 2 * 128;                           // [half][row]
+  float* red_max = reinterpret_cast<float*>(smem + AttnSmem::RED);  // [slot][sub][row]
+  float* red_sum = red_max + 2 * kSubs * 128;                       // [sub][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [2]
@@ -69,7 +73,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     mbar_init(&kv_empty[1], 1);
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 256);
+    mbar_init(p_full, 32 * kSoftWarps);
     mbar_init(o_full, 1);
     fence_mbar_init();
     pdl_launch_dependents();
@@ -161,48 +165,44 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else {
     const int q = warp & 3;
-    const int hf = (warp - 2) >> 2;  // column half: S columns [64 hf, 64 hf + 64), O columns [32 hf, 32 hf + 32)
+    const int sub = (warp - 2) >> 2;  // score columns [32 sub, 32 sub + 32), output columns [16 sub, 16 sub + 16)
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float c = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
-    float o[32];
+    float o[kOCols];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) o[i] = 0.f;
+    for (int i = 0; i < kOCols; ++i) o[i] = 0.f;
     float m = -INFINITY, l = 0.f;
-    uint8_t* prow = smem + AttnSmem::P + hf * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+    // This warp's 32 keys are half of the 64-key swizzle atom (sub >> 1).
+    uint8_t* prow = smem + AttnSmem::P + (sub >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+    const int ch0 = (sub & 1) * 4;
     bool ok = true;
-    // Every iteration runs the pair barrier and the p_full arrival even after a
-    // failed wait (the work is skipped), so no thread is left waiting on a
-    // barrier that its partner will never reach.
+    // Every iteration runs the quarter barrier and the p_full arrival even
+    // after a failed wait (the work is skipped), so no thread is left waiting
+    // on a barrier that another warp of its quarter will never reach.
     for (int j = 0; j < nkv; ++j) {
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1));
-      float s[64];
-      const int nvalid = min(128, T - j * 128) - hf * 64;  // valid columns of this half
+      float s[kSCols];
+      const int nvalid = min(128, T - j * 128) - sub * kSCols;  // valid columns of this warp
       float mx = -INFINITY;
       if (ok) {
         tc_fence_after();
-        const uint32_t tS = tmem + (j & 1) * 128 + hf * 64;
-        float v[32];
-        tmem_ld32(tS + lane_base, v);
+        tmem_ld32(tmem + (j & 1) * 128 + sub * kSCols + lane_base, s);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = v[i];
-        tmem_ld32(tS + lane_base + 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 + i] = v[i];
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < kSCols; ++i)
           if (i < nvalid) mx = fmaxf(mx, s[i]);
       }
-      float* slot = red_max + (j & 1) * 256;
-      slot[hf * 128 + r] = mx;
-      pair_barrier(q);
-      mx = fmaxf(slot[r], slot[128 + r]);
+      float* slot = red_max + (j & 1) * (kSubs * 128);
+      slot[sub * 128 + r] = mx;
+      quarter_barrier(q);
+#pragma unroll
+      for (int k = 0; k < kSubs; ++k) mx = fmaxf(mx, slot[k * 128 + r]);
       const float m_new = fmaxf(m, mx * c);
       const float alpha = ex2_approx(m - m_new);
       float rs = 0.f;
-      uint32_t pk[32];
+      uint32_t pk[kSCols / 2];
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
+      for (int i = 0; i < kSCols; i += 2) {
         const float p0 = (i < nvalid) ? ex2_approx(fmaf(s[i], c, -m_new)) : 0.f;
         const float p1 = (i + 1 < nvalid) ? ex2_approx(fmaf(s[i + 1], c, -m_new)) : 0.f;
         __half2 hp = __floats2half2_rn(p0, p1);
@@ -214,18 +214,17 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         ok = __all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1));
         if (ok) {
           tc_fence_after();
-          float v[32];
-          tmem_ld32(tO + lane_base + hf * 32, v);
+          float v[16];
+          tmem_ld16(tO + lane_base + sub * kOCols, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = (o[i] + v[i]) * alpha;
+          for (int i = 0; i < kOCols; ++i) o[i] = (o[i] + v[i]) * alpha;
         }
       }
       l = l * alpha + rs;
       m = m_new;
-      // P half-row -> this half's 128-byte swizzle atom (keys 64 hf .. 64 hf + 63).
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
+      for (int ch = 0; ch < 4; ++ch)
+        *reinterpret_cast<uint4*>(prow + (((ch0 + ch) ^ (r & 7)) << 4)) =
             make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
@@ -234,32 +233,31 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, (nkv - 1) & 1));
     if (ok) {
       tc_fence_after();
-      float v[32];
-      tmem_ld32(tO + lane_base + hf * 32, v);
+      float v[16];
+      tmem_ld16(tO + lane_base + sub * kOCols, v);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] += v[i];
+      for (int i = 0; i < kOCols; ++i) o[i] += v[i];
     } else if (lane == 0) {
       atomicOr(err, kErrWaitSoftmax);
     }
-    red_sum[hf * 128 + r] = l;
-    pair_barrier(q);
-    const float ltot = red_sum[r] + red_sum[128 + r];
+    red_sum[sub * 128 + r] = l;
+    quarter_barrier(q);
+    float ltot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kSubs; ++k) ltot += red_sum[k * 128 + r];
     const int t = qt * 128 + r;
     if (ok && t < T) {
       const float inv = 1.0f / ltot;
-      __half* dst = out + (static_cast<int64_t>(b) * T + t) * (H * 64) + h * 64 + hf * 32;
+      __half* dst = out + (static_cast<int64_t>(b) * T + t) * (H * 64) + h * 64 + sub * kOCols;
 #pragma unroll
-      for (int i = 0; i < 32; i += 8) {
+      for (int i = 0; i < kOCols; i += 8) {
         __half2 h0 = __floats2half2_rn(o[i] * inv, o[i + 1] * inv);
         __half2 h1 = __floats2half2_rn(o[i + 2] * inv, o[i + 3] * inv);
         __half2 h2 = __floats2half2_rn(o[i + 4] * inv, o[i + 5] * inv);
         __half2 h3 = __floats2half2_rn(o[i + 6] * inv, o[i + 7] * inv);
-        uint4 u;
-        u.x = *reinterpret_cast<uint32_t*>(&h0);
-        u.y = *reinterpret_cast<uint32_t*>(&h1);
-        u.z = *reinterpret_cast<uint32_t*>(&h2);
-        u.w = *reinterpret_cast<uint32_t*>(&h3);
-        *reinterpret_cast<uint4*>(dst + i) = u;
+        *reinterpret_cast<uint4*>(dst + i) =
+            make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                       *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
       }
     }
   }

@@ -9,7 +9,8 @@ namespace w2v {
 // One warp per frame.  Ties resolve to the lowest index; the comparison is an
 // fp32 compare on the stored logits, the same values the caller reads back.
 __global__ void __launch_bounds__(256)
-argmax_kernel(const float* __restrict__ logits, int rows, int V, int32_t* __restrict__ ids) {
+argmax_kernel(const float* logits, int rows, int V, int32_t* __restrict__ ids) {
+  // logits come from the previous kernel: plain loads after pdl_wait().
   if (threadIdx.x == 0) pdl_launch_dependents();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -19,7 +20,7 @@ argmax_kernel(const float* __restrict__ logits, int rows, int V, int32_t* __rest
   float best = -INFINITY;
   int bi = 0x7fffffff;
   for (int v = lane; v < V; v += 32) {
-    const float x = __ldg(z + v);
+    const float x = z[v];
     if (x > best) {  // strictly greater: keeps the first (lowest) index per lane
       best = x;
       bi = v;
@@ -46,7 +47,7 @@ cudaError_t launch_argmax(const float* logits, int rows, int V, int32_t* ids, cu
 // exclusive scan of the keep flags (keep a_t iff a_t != blank and
 // (t == 0 or a_t != a_{t-1})).
 __global__ void __launch_bounds__(1024)
-ctc_collapse_kernel(const int32_t* __restrict__ ids, int T, int t_valid, int blank, int32_t* __restrict__ tokens,
+ctc_collapse_kernel(const int32_t* ids, int T, int t_valid, int blank, int32_t* __restrict__ tokens,
                     int32_t* __restrict__ n_tokens) {
   __shared__ int warp_sums[32];
   __shared__ int total_s;

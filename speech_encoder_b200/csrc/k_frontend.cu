@@ -27,7 +27,7 @@ constexpr int kMom = kK0 + kK0 * (kK0 + 1) / 2;  // 65
 // (atomic ticket) adds the partials in block order (deterministic), turns them
 // into per-channel GroupNorm scale/shift (fp64) and re-arms the ticket.
 __global__ void __launch_bounds__(256)
-gn_moments_kernel(const float* __restrict__ pcm, int n, int t0, const float* __restrict__ w0,
+gn_moments_kernel(const float* pcm, int n, int t0, const float* __restrict__ w0,
                   const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                   double* __restrict__ partial, unsigned* __restrict__ ticket, float2* __restrict__ scale_shift) {
   if (threadIdx.x == 0) pdl_launch_dependents();
@@ -40,7 +40,7 @@ gn_moments_kernel(const float* __restrict__ pcm, int n, int t0, const float* __r
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < t0; t += gridDim.x * blockDim.x) {
     float w[kK0];
 #pragma unroll
-    for (int j = 0; j < kK0; ++j) w[j] = __ldg(x + kS0 * t + j);
+    for (int j = 0; j < kK0; ++j) w[j] = x[kS0 * t + j];
     int idx = kK0;
 #pragma unroll
     for (int j = 0; j < kK0; ++j) {
@@ -122,120 +122,147 @@ cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, const 
                     beta, eps, partial, ticket, scale_shift);
 }
 
-// One warp per output frame; lane l owns channel pairs (2l + 64i, 2l + 64i + 1),
-// i = 0..7, so each half2 store instruction of a warp writes 128 contiguous bytes.
+// Conv layer 0 + norm + GELU.  Two warps per output frame, four frames per
+// 256-thread CTA iteration; lane l of half h owns channel pairs
+// (256 h + 2 l + 64 i, +1), i = 0..3, so each half2 store instruction of a warp
+// writes 128 contiguous bytes.  The 8 channels' 10 taps stay in registers for
+// the whole kernel (no shared-memory traffic per output).
 // group layout: y*scale + shift from the clip's GroupNorm statistics;
-// layer layout: bias, then LayerNorm over the 512 channels of the frame.
+// layer layout: bias, then LayerNorm over the 512 channels of the frame (the
+// two halves' partial sums meet in shared memory).
 __global__ void __launch_bounds__(256, 2)
-conv0_kernel(const float* __restrict__ pcm, int n, int t0, int clip_rows, const float* __restrict__ w0,
+conv0_kernel(const float* pcm, int n, int t0, int clip_rows, const float* __restrict__ w0,
              const float* __restrict__ b0, const float* __restrict__ gamma, const float* __restrict__ beta,
-             const float2* __restrict__ scale_shift, int layer_norm, float eps, int act, __half* __restrict__ out) {
-  __shared__ __align__(16) float sw[kK0][kC];
-  __shared__ __align__(16) float sa[kC];  // group: scale;  layer: gamma
-  __shared__ __align__(16) float sb[kC];  // group: shift;  layer: beta
-  __shared__ __align__(16) float sbias[kC];
+             const float2* scale_shift, int layer_norm, float eps, int act, __half* __restrict__ out) {
+  // scale_shift is written by the previous kernel (programmatic dependent
+  // launch): it is read with plain coherent loads after pdl_wait(), never
+  // through a restrict/read-only path that could be hoisted above the wait.
+  __shared__ float red[2][4][2];
   if (threadIdx.x == 0) pdl_launch_dependents();
   const int b = blockIdx.y;
-  for (int i = threadIdx.x; i < kC * kK0; i += blockDim.x) sw[i % kK0][i / kK0] = w0[i];
-  if (layer_norm) {
-    for (int c = threadIdx.x; c < kC; c += blockDim.x) {
-      sa[c] = gamma[c];
-      sb[c] = beta[c];
-      sbias[c] = b0 ? b0[c] : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = warp >> 1;   // frame slot of this CTA iteration
+  const int hh = warp & 1;   // channel half
+  float w[8][kK0], sa[8], sb[8], bias[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = hh * 256 + 2 * lane + 64 * (k >> 1) + (k & 1);
+#pragma unroll
+    for (int j = 0; j < kK0; ++j) w[k][j] = __ldg(w0 + c * kK0 + j);
+    if (layer_norm) {
+      sa[k] = __ldg(gamma + c);
+      sb[k] = __ldg(beta + c);
+      bias[k] = b0 ? __ldg(b0 + c) : 0.f;
     }
   }
   pdl_wait();
   if (!layer_norm) {
-    for (int c = threadIdx.x; c < kC; c += blockDim.x) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = hh * 256 + 2 * lane + 64 * (k >> 1) + (k & 1);
       const float2 v = scale_shift[b * kC + c];
-      sa[c] = v.x;
-      sb[c] = v.y;
+      sa[k] = v.x;
+      sb[k] = v.y;
+      bias[k] = 0.f;
     }
   }
-  __syncthreads();
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
   const float* x = pcm + static_cast<int64_t>(b) * n;
   __half* ob = out + static_cast<int64_t>(b) * clip_rows * kC;
-  for (int t = blockIdx.x * wpb + warp; t < t0; t += gridDim.x * wpb) {
-    float xw[kK0];
+  // The frame loop bound is uniform across the CTA (barriers inside).
+  for (int base = blockIdx.x * 4; base < t0; base += gridDim.x * 4) {
+    const int t = base + f;
+    const bool live = t < t0;
+    float y[8];
+    if (live) {
+      float xw[kK0];
 #pragma unroll
-    for (int j = 0; j < kK0; ++j) xw[j] = __ldg(x + kS0 * t + j);
-    float y[16];
+      for (int j = 0; j < kK0; ++j) xw[j] = x[kS0 * t + j];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 2 * lane + 64 * i;
-      float y0 = 0.f, y1 = 0.f;
+      for (int k = 0; k < 8; ++k) {
+        float a = bias[k];
 #pragma unroll
-      for (int j = 0; j < kK0; ++j) {
-        const float2 w = *reinterpret_cast<const float2*>(&sw[j][c]);
-        y0 = fmaf(w.x, xw[j], y0);
-        y1 = fmaf(w.y, xw[j], y1);
+        for (int j = 0; j < kK0; ++j) a = fmaf(w[k][j], xw[j], a);
+        y[k] = a;
       }
-      y[2 * i] = y0;
-      y[2 * i + 1] = y1;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[k] = 0.f;
     }
     if (layer_norm) {
-      float sum = 0.f;
+      float s1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = 2 * lane + 64 * i;
-        y[2 * i] += sbias[c];
-        y[2 * i + 1] += sbias[c + 1];
-        sum += y[2 * i] + y[2 * i + 1];
+      for (int k = 0; k < 8; ++k) s1 += y[k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      if (lane == 0) red[0][f][hh] = s1;
+      __syncthreads();
+      const float mean = (red[0][f][0] + red[0][f][1]) * (1.0f / kC);
+      float s2 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float d = y[k] - mean;
+        s2 += d * d;
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      const float mean = sum * (1.0f / kC);
-      float sq = 0.f;
+      for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      if (lane == 0) red[1][f][hh] = s2;
+      __syncthreads();
+      const float rstd = rsqrtf((red[1][f][0] + red[1][f][1]) * (1.0f / kC) + eps);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float dlt = y[i] - mean;
-        sq += dlt * dlt;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      const float rstd = rsqrtf(sq * (1.0f / kC) + eps);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) y[i] = (y[i] - mean) * rstd;
+      for (int k = 0; k < 8; ++k) y[k] = (y[k] - mean) * rstd;
     }
-    __half* orow = ob + static_cast<int64_t>(t) * kC;
+    if (live) {
+      __half* orow = ob + static_cast<int64_t>(t) * kC + hh * 256 + 2 * lane;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 2 * lane + 64 * i;
-      const float a0 = fmaf(y[2 * i], sa[c], sb[c]);
-      const float a1 = fmaf(y[2 * i + 1], sa[c + 1], sb[c + 1]);
-      *reinterpret_cast<__half2*>(orow + c) = __floats2half2_rn(apply_act(a0, act), apply_act(a1, act));
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<__half2*>(orow + 64 * i) =
+            __floats2half2_rn(apply_act(fmaf(y[2 * i], sa[2 * i], sb[2 * i]), act),
+                              apply_act(fmaf(y[2 * i + 1], sa[2 * i + 1], sb[2 * i + 1]), act));
     }
+    if (layer_norm) __syncthreads();  // red[] is rewritten next iteration
   }
 }
 
 cudaError_t launch_conv0(const float* pcm, int n, int batch, int t0, int clip_rows, const float* w0, const float* b0,
                          const float* gamma, const float* beta, const float2* scale_shift, int layer_norm, float eps,
                          int act, __half* out, cudaStream_t st) {
-  int nbx = (t0 + 8 * 8 - 1) / (8 * 8);  // ~8 frames per warp
-  if (nbx > 148 * 4) nbx = 148 * 4;
+  int nbx = (t0 + 4 * 16 - 1) / (4 * 16);  // ~16 frames per warp pair
+  if (nbx > 148 * 2 * 4) nbx = 148 * 2 * 4;
   if (nbx < 1) nbx = 1;
   return launch_pdl(conv0_kernel, dim3(nbx, batch), dim3(256), 0, st, pcm, n, t0, clip_rows, w0, b0, gamma, beta,
                     scale_shift, layer_norm, eps, act, out);
 }
 
 // ------------------------------------------------------------------ LayerNorm
-// One warp per row.  fp16 input: lane owns 8-element chunks (lane + 32 i);
-// fp32 input: 4-element chunks.  Two passes over registers (mean, then the
-// centred sum of squares), fp32 throughout, fp16 output.
+// One warp per row, two rows per 64-thread CTA (many small CTAs spread a
+// ~800-row activation over every SM).  fp16 input: lane owns 8-element chunks
+// (lane + 32 i); fp32 input: 4-element chunks.  The row, gamma and beta are
+// all requested before any arithmetic (one memory round trip); two passes over
+// registers (mean, then the centred sum of squares), fp32 throughout, fp16 out.
 template <int COLS, bool F32IN>
-__global__ void __launch_bounds__(256)
-layernorm_kernel(const void* __restrict__ xin, __half* __restrict__ y, int rows, const float* __restrict__ gamma,
+__global__ void __launch_bounds__(64)
+layernorm_kernel(const void* xin, __half* __restrict__ y, int rows, const float* __restrict__ gamma,
                  const float* __restrict__ beta, float eps, int act) {
+  // xin is the previous kernel's output: plain loads after pdl_wait().
   constexpr int VEC = F32IN ? 4 : 8;
   constexpr int NCH = COLS / (32 * VEC);
   constexpr int NPL = COLS / 32;
   if (threadIdx.x == 0) pdl_launch_dependents();
-  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int row = blockIdx.x * 2 + warp;
+  float g[NPL], bt[NPL];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const int c0 = (lane + 32 * i) * VEC;
+#pragma unroll
+    for (int k = 0; k < VEC; k += 4) {
+      const float4 gv = __ldg(reinterpret_cast<const float4*>(gamma + c0 + k));
+      const float4 bv = __ldg(reinterpret_cast<const float4*>(beta + c0 + k));
+      g[VEC * i + k] = gv.x; g[VEC * i + k + 1] = gv.y; g[VEC * i + k + 2] = gv.z; g[VEC * i + k + 3] = gv.w;
+      bt[VEC * i + k] = bv.x; bt[VEC * i + k + 1] = bv.y; bt[VEC * i + k + 2] = bv.z; bt[VEC * i + k + 3] = bv.w;
+    }
+  }
+  pdl_wait();
   if (row >= rows) return;
   float v[NPL];
   if (F32IN) {
@@ -278,28 +305,29 @@ layernorm_kernel(const void* __restrict__ xin, __half* __restrict__ y, int rows,
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c0 = (lane + 32 * i) * VEC;
-    __align__(16) __half2 hv[VEC / 2];
+    uint32_t hv[VEC / 2];
 #pragma unroll
     for (int j = 0; j < VEC; j += 2) {
-      const float a0 = (v[VEC * i + j] - mean) * rstd * __ldg(gamma + c0 + j) + __ldg(beta + c0 + j);
-      const float a1 = (v[VEC * i + j + 1] - mean) * rstd * __ldg(gamma + c0 + j + 1) + __ldg(beta + c0 + j + 1);
-      hv[j / 2] = __floats2half2_rn(apply_act(a0, act), apply_act(a1, act));
+      const float a0 = fmaf((v[VEC * i + j] - mean) * rstd, g[VEC * i + j], bt[VEC * i + j]);
+      const float a1 = fmaf((v[VEC * i + j + 1] - mean) * rstd, g[VEC * i + j + 1], bt[VEC * i + j + 1]);
+      __half2 h2 = __floats2half2_rn(apply_act(a0, act), apply_act(a1, act));
+      hv[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
     }
     if (VEC == 8)
-      *reinterpret_cast<uint4*>(yr + c0) = *reinterpret_cast<const uint4*>(hv);
+      *reinterpret_cast<uint4*>(yr + c0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
     else
-      *reinterpret_cast<uint2*>(yr + c0) = *reinterpret_cast<const uint2*>(hv);
+      *reinterpret_cast<uint2*>(yr + c0) = make_uint2(hv[0], hv[1]);
   }
 }
 
 template <int COLS>
 static void ln_dispatch(const void* x, int in_f32, __half* y, int rows, const float* g, const float* b, float eps,
                         int act, cudaStream_t st) {
-  const int blocks = (rows + 7) / 8;
+  const int blocks = (rows + 1) / 2;
   if (in_f32)
-    launch_pdl(layernorm_kernel<COLS, true>, dim3(blocks), dim3(256), 0, st, x, y, rows, g, b, eps, act);
+    launch_pdl(layernorm_kernel<COLS, true>, dim3(blocks), dim3(64), 0, st, x, y, rows, g, b, eps, act);
   else
-    launch_pdl(layernorm_kernel<COLS, false>, dim3(blocks), dim3(256), 0, st, x, y, rows, g, b, eps, act);
+    launch_pdl(layernorm_kernel<COLS, false>, dim3(blocks), dim3(64), 0, st, x, y, rows, g, b, eps, act);
 }
 
 cudaError_t launch_layernorm(const void* x, int in_f32, __half* y, int rows, int cols, const float* gamma,

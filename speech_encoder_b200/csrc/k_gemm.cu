@@ -121,8 +121,8 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, int 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2, GemmShape s,
-               GemmEpilogue e, int vec_ok, int mode, int* err) {
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+               const __grid_constant__ CUtensorMap tmV, GemmShape s, GemmEpilogue e, int vec_ok, int mode, int* err) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -238,8 +238,57 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_after();
   }
 
-  if (mode == 1 && region == 2) mode = 0;  // V tiles: transposed, generic path
-  if (mode == 1) {
+  if (mode == 1 && region == 2) {
+    // ------------------------------------------- direct, V^T of fused QKV
+    // Each warp stages its 32 time steps x 32 dims boxes transposed
+    // ([dim][time], 64-byte rows, 64-byte swizzle) and stores them with a TMA
+    // tensor store on V^T when its rows lie in one clip at an 8-aligned time
+    // offset (always at batch 1); otherwise it scatters from registers, each
+    // store instruction covering 32 consecutive time steps of one dim.
+    if (epi) {
+      named_barrier_sync(1, kEpiThreads);  // bias staged
+      const int grow = m0 + r;
+      const int rfirst = m0 + q * 32;
+      const int clip0 = rfirst / e.t_len;
+      const int t_first = rfirst - clip0 * e.t_len;
+      const int rlast = min(rfirst + 31, s.M - 1);
+      const bool boxed = (rlast / e.t_len == clip0) && (t_first % 8 == 0);
+      const int clip = grow / e.t_len;
+      const int t = grow - clip * e.t_len;
+      uint8_t* stage = smem + (warp - 2) * (BN / 2 / 32) * 4096;
+      int nbox = 0;
+#pragma unroll 1
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+        float v[32];
+        if (ok) tmem_ld32(trow + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i] + bias_s[c + i], e.act);
+        const int cc = n0 + c - 2 * e.qkv_d;  // column within V: head * 64 + dim
+        if (boxed) {
+          uint8_t* box = stage + nbox * 4096;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<__half*>(box + i * 64 + ((((lane >> 3) ^ ((i >> 1) & 3))) << 4) + (lane & 7) * 2) =
+                __float2half_rn(v[i]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && ok) tma_store_2d(&tmV, box, t_first, (clip0 * e.n_heads + (cc >> 6)) * 64 + (cc & 63));
+          ++nbox;
+        } else if (ok && grow < s.M) {
+          __half* dst = static_cast<__half*>(e.vt) +
+                        (static_cast<int64_t>(clip * e.n_heads + (cc >> 6)) * 64 + (cc & 63)) * e.t_pad + t;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(v[i]);
+        }
+      }
+      if (lane == 0) {
+        bulk_commit_group();
+        bulk_wait_all();
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  } else if (mode == 1) {
     // ------------------------------------------------------------- direct
     if (epi) {
       named_barrier_sync(1, kEpiThreads);  // bias staged
@@ -539,8 +588,8 @@ cudaError_t gemm_prepare() {
 
 template <int BN>
 static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmO,
-                             const CUtensorMap& tmO2, const GemmShape& s, const GemmEpilogue& e, int vec_ok, int mode,
-                             int* err, cudaStream_t st) {
+                             const CUtensorMap& tmO2, const CUtensorMap& tmV, const GemmShape& s,
+                             const GemmEpilogue& e, int vec_ok, int mode, int* err, cudaStream_t st) {
   using C = GemmCfg<BN>;
   const int S = s.splits;
   dim3 grid((s.M + 127) / 128, (s.N + BN - 1) / BN, S > 1 ? S : s.batch);
@@ -558,7 +607,7 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
   attr[1].val.clusterDim.z = S > 1 ? S : 1;
   cfg.attrs = attr;
   cfg.numAttrs = S > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, tmA, tmB, tmO, tmO2, s, e, vec_ok, mode, err);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, tmA, tmB, tmO, tmO2, tmV, s, e, vec_ok, mode, err);
 }
 
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
@@ -579,9 +628,10 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   if (e.qkv_d > 0) vec = vec && (reinterpret_cast<uintptr_t>(e.out_k) % 16 == 0);
   // Direct (TMA-store) epilogue: rows must be 16-byte multiples and any
   // residual vector-loadable; tiles at least 64 wide.
-  CUtensorMap tmO, tmO2;
+  CUtensorMap tmO, tmO2, tmV;
   std::memset(&tmO, 0, sizeof tmO);
   std::memset(&tmO2, 0, sizeof tmO2);
+  std::memset(&tmV, 0, sizeof tmV);
   int mode = s.splits > 1 ? 2 : 0;
   const bool tma_ok = s.splits == 1 && bn >= 64 && vec && (e.ldo * esz_out) % 16 == 0 &&
                       (e.residual == nullptr || (e.ldr * esz_res) % 16 == 0);
@@ -594,15 +644,24 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
     const uint32_t box[3] = {32, 32, 1};
     const int swz = e.out_f32 ? 128 : 64;
     bool built = make_tmap(&tmO, e.out, 3, dims, str, box, esz_out, swz) == cudaSuccess;
-    if (built && e.qkv_d > 0) built = make_tmap(&tmO2, e.out_k, 3, dims, str, box, esz_out, swz) == cudaSuccess;
+    if (built && e.qkv_d > 0) {
+      built = make_tmap(&tmO2, e.out_k, 3, dims, str, box, esz_out, swz) == cudaSuccess;
+      // V^T [clip][head][64][t_pad]: time innermost, one row per (clip, head, dim)
+      const uint64_t vd[2] = {static_cast<uint64_t>(e.t_len),
+                              static_cast<uint64_t>(s.M / e.t_len) * e.n_heads * 64};
+      const uint64_t vs[1] = {static_cast<uint64_t>(e.t_pad) * 2};
+      const uint32_t vb[2] = {32, 32};
+      built = built && !e.out_f32 && e.t_pad % 8 == 0 &&
+              make_tmap(&tmV, e.vt, 2, vd, vs, vb, 2, 64) == cudaSuccess;
+    }
     if (built) mode = 1;
   }
   switch (bn) {
-    case 32: return launch_bn<32>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
-    case 64: return launch_bn<64>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
-    case 128: return launch_bn<128>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
-    case 192: return launch_bn<192>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
-    case 256: return launch_bn<256>(tmA, tmB, tmO, tmO2, s, e, vec, mode, err, st);
+    case 32: return launch_bn<32>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
+    case 64: return launch_bn<64>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
+    case 128: return launch_bn<128>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
+    case 192: return launch_bn<192>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
+    case 256: return launch_bn<256>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
     default: return cudaErrorInvalidValue;
   }
 }

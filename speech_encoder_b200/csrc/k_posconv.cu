@@ -37,7 +37,7 @@ struct PosCfg {
 
 template <int MG>
 __global__ void __launch_bounds__(192, 1)
-posconv_kernel(const __grid_constant__ CUtensorMap tmX, const __half* __restrict__ x, const __half* __restrict__ wpack,
+posconv_kernel(const __grid_constant__ CUtensorMap tmX, const __half* x, const __half* __restrict__ wpack,
                const float* __restrict__ bias, int T, int d, int act, float* __restrict__ h, int* err) {
   using C = PosCfg<MG>;
   extern __shared__ uint8_t smem_raw[];

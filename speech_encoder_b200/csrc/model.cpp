@@ -482,6 +482,7 @@ int get_plan(w2v_model* m, int n, int batch, const Plan** out) {
 // cost (FLOPs and the bytes it must move at minimum).
 struct Prof {
   bool timing = false;
+  int only_class = -1;  // >= 0: launch only the kernels of this class (timing replays)
   int launches = 0;
   std::vector<cudaEvent_t> pool;
   size_t used = 0;
@@ -506,6 +507,10 @@ struct Prof {
 
 #define LAUNCH(KL, FL, BY, EXPR)                                             \
   do {                                                                       \
+    if (prof && prof->only_class >= 0 && prof->only_class != (KL)) break;    \
+    if (prof && prof->only_class >= 0) {                                     \
+      prof->recs.push_back({(KL), double(FL), double(BY), nullptr, nullptr}); \
+    }                                                                        \
     cudaEvent_t e0_ = nullptr;                                               \
     if (prof && prof->timing) {                                              \
       e0_ = prof->next();                                                    \
@@ -1029,6 +1034,74 @@ extern "C" int w2v_profile_forward(w2v_model* m, const float* pcm_dev, int n_sam
   }
   *n_out = n;
   m->last_launches = prof.launches;
+  return W2V_OK;
+}
+
+extern "C" int w2v_time_class(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev,
+                              int klass, int reps, float* us_per_launch, int* launches, double* flops_per_launch,
+                              double* bytes_per_launch, void* stream) {
+  if (!m || !us_per_launch || !launches || !flops_per_launch || !bytes_per_launch) return W2V_EINVAL;
+  if (!pcm_dev || !logits_dev || !aligned16(pcm_dev) || !aligned16(logits_dev)) return fail(m, W2V_EINVAL, "bad pointer");
+  if (klass < 0 || klass >= W2V_K_NUM_CLASSES || reps < 1 || reps > 1000) return fail(m, W2V_EINVAL, "bad class/reps");
+  if (n_samples < 400 || n_samples > m->cfg.max_samples) return fail(m, W2V_ESHAPE, "n_samples=%d out of range", n_samples);
+  if (batch < 1 || batch > m->cfg.max_batch) return fail(m, W2V_ESHAPE, "batch=%d out of range", batch);
+  CUDA_OR(m, cudaSetDevice(m->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Plan* p = nullptr;
+  int rc = get_plan(m, n_samples, batch, &p);
+  if (rc != W2V_OK) return rc;
+  // Record `reps` passes of only this class's launches as one graph.
+  Prof filt;
+  filt.only_class = klass;
+  cudaGraph_t g = nullptr;
+  CUDA_OR(m, cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+  for (int r = 0; r < reps && rc == W2V_OK; ++r) {
+    rc = enqueue_forward(m, *p, pcm_dev, logits_dev, m->cap_stream, &filt);
+    if (rc == W2V_OK && klass >= W2V_K_ARGMAX)
+      rc = enqueue_ctc(m, logits_dev, batch, p->Tf, p->Tf, m->ids + static_cast<size_t>(batch) * p->Tf,
+                       m->ids + static_cast<size_t>(2) * batch * p->Tf, m->cap_stream, &filt);
+  }
+  cudaError_t e = cudaStreamEndCapture(m->cap_stream, &g);
+  if (rc != W2V_OK) {
+    if (g) cudaGraphDestroy(g);
+    return rc;
+  }
+  if (e != cudaSuccess) return fail(m, W2V_ECUDA, "capture: %s", cudaGetErrorString(e));
+  const int n = filt.launches;
+  if (n == 0) {
+    cudaGraphDestroy(g);
+    *launches = 0;
+    *us_per_launch = 0.f;
+    *flops_per_launch = *bytes_per_launch = 0.0;
+    return W2V_OK;
+  }
+  cudaGraphExec_t ex = nullptr;
+  e = cudaGraphInstantiate(&ex, g, 0);
+  cudaGraphDestroy(g);
+  if (e != cudaSuccess) return fail(m, W2V_ECUDA, "instantiate: %s", cudaGetErrorString(e));
+  cudaEvent_t e0, e1;
+  cudaEventCreate(&e0);
+  cudaEventCreate(&e1);
+  cudaGraphLaunch(ex, st);  // warm
+  cudaEventRecord(e0, st);
+  cudaGraphLaunch(ex, st);
+  cudaEventRecord(e1, st);
+  e = cudaEventSynchronize(e1);
+  float ms = 0.f;
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  cudaGraphExecDestroy(ex);
+  if (e != cudaSuccess) return fail(m, W2V_ECUDA, "timing: %s", cudaGetErrorString(e));
+  double fl = 0.0, by = 0.0;
+  for (auto& r : filt.recs) {
+    fl += r.flops;
+    by += r.bytes;
+  }
+  *launches = n / reps;
+  *us_per_launch = 1000.f * ms / n;
+  *flops_per_launch = fl / n;
+  *bytes_per_launch = by / n;
   return W2V_OK;
 }
 

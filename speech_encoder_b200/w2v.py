@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         "w2v_last_launch_count": (I, [VP]),
         "w2v_kernel_class_name": (ctypes.c_char_p, [I]),
         "w2v_profile_forward": (I, [VP, VP, I, I, VP, VP, ctypes.POINTER(w2v_kernel_time), I, ctypes.POINTER(I)]),
+        "w2v_time_class": (I, [VP, VP, I, I, VP, I, I, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(I),
+                               ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), VP]),
         "w2v_op_gemm": (I, [VP, VP, I, I, I, VP, VP, I, VP, I, I, I, I, VP, VP]),
         "w2v_op_attention": (I, [VP, VP, VP, VP, I, I, I, I, VP, VP]),
         "w2v_op_layernorm": (I, [VP, I, VP, I, I, VP, VP, ctypes.c_float, I, VP]),
@@ -207,6 +209,24 @@ def w2v_profile_forward(model: int, pcm, n_samples: int, batch: int, logits, str
                                      max_out, ctypes.byref(n)), model, "w2v_profile_forward")
     return [(w2v_kernel_class_name(buf[i].klass), float(buf[i].ms), float(buf[i].flops), float(buf[i].bytes))
             for i in range(n.value)]
+
+
+KERNEL_CLASSES = ["gn_moments", "conv0_norm_gelu", "conv_gemm", "conv_layernorm", "fp_layernorm", "proj_gemm",
+                  "posconv", "enc_layernorm", "qkv_gemm", "attention", "out_gemm", "ffn1_gemm", "ffn2_gemm",
+                  "lm_head_gemm", "argmax", "ctc_collapse"]
+
+
+def w2v_time_class(model: int, pcm, n_samples: int, batch: int, logits, klass, reps: int = 10, stream=None):
+    """(us_per_launch, launches_per_forward, flops_per_launch, bytes_per_launch) of one kernel class."""
+    k = KERNEL_CLASSES.index(klass) if isinstance(klass, str) else int(klass)
+    us = ctypes.c_float()
+    n = ctypes.c_int()
+    fl = ctypes.c_double()
+    by = ctypes.c_double()
+    _check(lib().w2v_time_class(model, _ptr(pcm), int(n_samples), int(batch), _ptr(logits), k, int(reps),
+                                ctypes.byref(us), ctypes.byref(n), ctypes.byref(fl), ctypes.byref(by),
+                                _stream(stream)), model, "w2v_time_class")
+    return float(us.value), int(n.value), float(fl.value), float(by.value)
 
 
 def w2v_destroy(model: int) -> None:
