@@ -206,8 +206,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const float p0 = (i < nvalid) ? ex2_approx(fmaf(s[i], c, -m_new)) : 0.f;
         const float p1 = (i + 1 < nvalid) ? ex2_approx(fmaf(s[i + 1], c, -m_new)) : 0.f;
         __half2 hp = __floats2half2_rn(p0, p1);
-        const float2 back = __half22float2(hp);
-        rs += back.x + back.y;
+        rs += p0 + p1;  // fp32 row sum (the conversion unit is the scarce pipe here)
         pk[i / 2] = *reinterpret_cast<uint32_t*>(&hp);
       }
       if (j > 0 && ok) {

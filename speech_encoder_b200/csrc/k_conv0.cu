@@ -1,0 +1,225 @@
+// Conv layer 0 of the feature encoder on the tensor core: Conv1d(1 -> 512,
+// kernel 10, stride 5) is a GEMM with K = 10 taps (zero-padded to the MMA's
+// K = 16): A[t, j] = pcm[5 t + j], B[c, j] = w0[c, j].  One CTA per 128 output
+// frames of one clip computes all 512 channels with two tcgen05 MMAs
+// (M = 128, N = 256, K = 16) into 512 TMEM columns; the epilogue applies the
+// norm and GELU and stores through TMA:
+//   group layout: GroupNorm with per-channel statistics over every frame of
+//     the clip (the TensorRT wav2vec2 README's "group norm over every time
+//     step"), precomputed as scale/shift by the moments kernel;
+//   layer layout: conv bias, then LayerNorm over the 512 channels of each
+//     frame (the four warps that share a row combine their partial sums).
+// 576 threads: warp 0 stages the operands and issues the MMAs, warp 1 owns
+// TMEM, warps 2-17 run the epilogue (four warps per TMEM lane quarter, one per
+// 128-channel slice).  The PCM is rounded to fp16 for the MMA, the same
+// rounding every inter-layer activation of this path gets.
+#include "ptx.cuh"
+#include "w2v_internal.h"
+
+namespace w2v {
+
+namespace {
+constexpr int kC0 = 512;
+constexpr int kTaps = 10;
+constexpr int kHop = 5;
+constexpr int A_OFF = 0;                   // [2 k-chunks][128 rows][8] fp16, 4 KB
+constexpr int B_OFF = 4096;                // [2 k-chunks][512 rows][8] fp16, 16 KB
+constexpr int P_OFF = B_OFF + 16384;       // float2 params[512]: (scale, shift) or (gamma, beta)
+constexpr int BIAS_OFF = P_OFF + 4096;     // float bias[512]
+constexpr int kEpiWarps = 16;              // 4 per TMEM lane quarter, 128 channels each
+constexpr int kCols = 512 / (kEpiWarps / 4);
+constexpr int RED_OFF = BIAS_OFF + 2048;   // float red[4 slices][128 rows]
+constexpr int STG_OFF = RED_OFF + 2048;    // staging: 16 warps x 4 boxes x 2 KB
+constexpr int BAR_OFF = STG_OFF + kEpiWarps * (kCols / 32) * 2048;
+constexpr int SMEM = BAR_OFF + 64 + 1024;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int n, int t0,
+                const __half* __restrict__ wpack, const float* __restrict__ b0, const float* __restrict__ gamma,
+                const float* __restrict__ beta, const float2* scale_shift, int layer_norm, float eps, int act,
+                int* err) {
+  // pcm and scale_shift may be written by the previous kernel (programmatic
+  // dependent launch): plain coherent loads after pdl_wait() only.
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float2* par = reinterpret_cast<float2*>(smem + P_OFF);
+  float* bias = reinterpret_cast<float*>(smem + BIAS_OFF);
+  float* red = reinterpret_cast<float*>(smem + RED_OFF);
+  uint64_t* w_full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* accf = w_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f0 = blockIdx.x * 128;
+  const int b = blockIdx.z;
+
+  if (threadIdx.x == 0) {
+    mbar_init(w_full, 1);
+    mbar_init(accf, 1);
+    fence_mbar_init();
+    pdl_launch_dependents();
+    // The packed weights do not depend on the previous kernel.
+    mbar_arrive_expect_tx(w_full, 16384);
+    bulk_load(smem + B_OFF, wpack, 16384, w_full);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (layer_norm) {
+    for (int c = threadIdx.x; c < kC0; c += kThreads) {
+      par[c] = make_float2(gamma[c], beta[c]);
+      bias[c] = b0 ? b0[c] : 0.f;
+    }
+  }
+  pdl_wait();
+  if (!layer_norm)
+    for (int c = threadIdx.x; c < kC0; c += kThreads) par[c] = scale_shift[b * kC0 + c];
+  // A tile: row t holds pcm[5 (f0 + t) + j], j < 10, then zeros; 16-byte
+  // chunk (row, k-chunk) at k-chunk * 2048 + row * 16 (no-swizzle core matrices).
+  if (threadIdx.x < 256) {
+    const int row = threadIdx.x >> 1, kc = threadIdx.x & 1;
+    const int t = f0 + row;
+    const float* x = pcm + static_cast<int64_t>(b) * n + static_cast<int64_t>(kHop) * t;
+    uint32_t hv[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const int j = kc * 8 + e;
+      const float v0 = (t < t0 && j < kTaps) ? x[j] : 0.f;
+      const float v1 = (t < t0 && j + 1 < kTaps) ? x[j + 1] : 0.f;
+      __half2 h = __floats2half2_rn(v0, v1);
+      hv[e / 2] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(smem + A_OFF + kc * 2048 + row * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      if (mbar_wait(w_full, 0)) {
+        tc_fence_after();
+        constexpr uint32_t idesc = idesc_f16_f32(128, 256);
+        const uint32_t sa = smem_u32(smem + A_OFF);
+        const uint32_t sb = smem_u32(smem + B_OFF);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          umma_f16(tmem + h * 256, smem_desc(sa, 2048, 128, kSwizzleNone), smem_desc(sb + h * 256 * 16, 8192, 128,
+                   kSwizzleNone), idesc, 0u);
+        umma_commit(accf);
+      } else {
+        atomicOr(err, kErrWaitMma);
+      }
+    }
+  } else if (warp >= 2) {
+    const int q = warp & 3;              // TMEM lane quarter
+    const int sl = (warp - 2) >> 2;      // channel slice [kCols sl, kCols sl + kCols)
+    const int r = q * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16) + sl * kCols;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
+    if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+    tc_fence_after();
+    float mean = 0.f, rstd = 1.f;
+    if (layer_norm) {
+      // Per-frame LayerNorm statistics over all 512 channels (two passes; the
+      // four slices of a row meet in shared memory).
+      float s1 = 0.f;
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < kCols; c += 32) {
+          float v[32];
+          tmem_ld32(trow + c, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s1 += v[i] + bias[sl * kCols + c + i];
+        }
+      }
+      red[sl * 128 + r] = s1;
+      named_barrier_sync(1, 32 * kEpiWarps);
+      mean = ((red[r] + red[128 + r]) + (red[256 + r] + red[384 + r])) * (1.0f / kC0);
+      named_barrier_sync(1, 32 * kEpiWarps);
+      float s2 = 0.f;
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < kCols; c += 32) {
+          float v[32];
+          tmem_ld32(trow + c, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float d = v[i] + bias[sl * kCols + c + i] - mean;
+            s2 += d * d;
+          }
+        }
+      }
+      red[sl * 128 + r] = s2;
+      named_barrier_sync(1, 32 * kEpiWarps);
+      rstd = rsqrtf(((red[r] + red[128 + r]) + (red[256 + r] + red[384 + r])) * (1.0f / kC0) + eps);
+    }
+    uint8_t* stage = smem + STG_OFF + (warp - 2) * (kCols / 32) * 2048;
+#pragma unroll 1
+    for (int cb = 0; cb < kCols / 32; ++cb) {
+      const int c = cb * 32;
+      const int ch = sl * kCols + c;
+      float v[32];
+      if (ok) tmem_ld32(trow + c, v);
+      uint32_t hv[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float a0, a1;
+        if (layer_norm) {
+          a0 = fmaf((v[i] + bias[ch + i] - mean) * rstd, par[ch + i].x, par[ch + i].y);
+          a1 = fmaf((v[i + 1] + bias[ch + i + 1] - mean) * rstd, par[ch + i + 1].x, par[ch + i + 1].y);
+        } else {
+          a0 = fmaf(v[i], par[ch + i].x, par[ch + i].y);
+          a1 = fmaf(v[i + 1], par[ch + i + 1].x, par[ch + i + 1].y);
+        }
+        __half2 h2 = __floats2half2_rn(apply_act(a0, act), apply_act(a1, act));
+        hv[i / 2] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      // 32 rows x 32 channels box, 64-byte rows, 64-byte swizzle.
+      uint8_t* box = stage + cb * 2048;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) tma_store_3d(&tmOut, box, ch, f0 + q * 32, b);
+    }
+    if (lane == 0) {
+      bulk_commit_group();
+      bulk_wait_all();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t conv0_prepare() {
+  return cudaFuncSetAttribute(conv0_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+}
+
+cudaError_t launch_conv0_tc(const float* pcm, int n, int batch, int t0, int clip_rows, const __half* wpack,
+                            const float* b0, const float* gamma, const float* beta, const float2* scale_shift,
+                            int layer_norm, float eps, int act, __half* out, int* err, cudaStream_t st) {
+  if (t0 <= 0 || batch <= 0) return cudaSuccess;
+  CUtensorMap tm;
+  const uint64_t dims[3] = {static_cast<uint64_t>(kC0), static_cast<uint64_t>(t0), static_cast<uint64_t>(batch)};
+  const uint64_t str[2] = {static_cast<uint64_t>(kC0) * 2, static_cast<uint64_t>(clip_rows) * kC0 * 2};
+  const uint32_t box[3] = {32, 32, 1};
+  cudaError_t r = make_tmap(&tm, out, 3, dims, str, box, 2, 64);
+  if (r != cudaSuccess) return r;
+  dim3 grid((t0 + 127) / 128, 1, batch);
+  return launch_pdl(conv0_tc_kernel, grid, dim3(kThreads), SMEM, st, tm, pcm, n, t0, wpack, b0, gamma, beta,
+                    scale_shift, layer_norm, eps, act, err);
+}
+
+}  // namespace w2v

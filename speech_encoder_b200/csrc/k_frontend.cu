@@ -73,11 +73,26 @@ gn_moments_kernel(const float* pcm, int n, int t0, const float* __restrict__ w0,
   __syncthreads();
   if (!last) return;
   __threadfence();
-  if (threadIdx.x < kMom) {
-    const volatile double* pb = partial + static_cast<int64_t>(b) * gridDim.x * kMom;
-    double sum = 0.0;
-    for (unsigned k = 0; k < gridDim.x; ++k) sum += pb[k * kMom + threadIdx.x];
-    mom[threadIdx.x] = sum;
+  {
+    // All 256 threads add the per-block partials (L2-coherent loads, which
+    // pipeline) in four fixed groups, then the groups combine in order.
+    __shared__ double part[4][kMom];
+    const double* pb = partial + static_cast<int64_t>(b) * gridDim.x * kMom;
+    const int mi = threadIdx.x % kMom, grp = threadIdx.x / kMom;  // 260 slots > 256 threads: grp 3 has 61
+    if (grp < 4) {
+      double sum = 0.0;
+      for (unsigned k = grp; k < gridDim.x; k += 4) sum += __ldcg(pb + k * kMom + mi);
+      part[grp][mi] = sum;
+    }
+    __syncthreads();
+    if (threadIdx.x < kMom) {
+      // threads 195..255 cover moments 0..60 of group 3; moments 61..64 of
+      // group 3 were not visited: add their blocks here.
+      double s3 = threadIdx.x < 256 - 3 * kMom ? part[3][threadIdx.x] : 0.0;
+      if (threadIdx.x >= 256 - 3 * kMom)
+        for (unsigned k = 3; k < gridDim.x; k += 4) s3 += __ldcg(pb + k * kMom + threadIdx.x);
+      mom[threadIdx.x] = ((part[0][threadIdx.x] + part[1][threadIdx.x]) + part[2][threadIdx.x]) + s3;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) ticket[b] = 0u;
@@ -109,7 +124,7 @@ gn_moments_kernel(const float* pcm, int n, int t0, const float* __restrict__ w0,
 }
 
 int gn_moment_blocks(int t0) {
-  int nb = (t0 + 256 * 8 - 1) / (256 * 8);
+  int nb = (t0 + 256 * 2 - 1) / (256 * 2);
   if (nb > 296) nb = 296;
   if (nb < 1) nb = 1;
   return nb;
@@ -120,117 +135,6 @@ cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, const 
                               cudaStream_t st) {
   return launch_pdl(gn_moments_kernel, dim3(gn_moment_blocks(t0), batch), dim3(256), 0, st, pcm, n, t0, w0, gamma,
                     beta, eps, partial, ticket, scale_shift);
-}
-
-// Conv layer 0 + norm + GELU.  Two warps per output frame, four frames per
-// 256-thread CTA iteration; lane l of half h owns channel pairs
-// (256 h + 2 l + 64 i, +1), i = 0..3, so each half2 store instruction of a warp
-// writes 128 contiguous bytes.  The 8 channels' 10 taps stay in registers for
-// the whole kernel (no shared-memory traffic per output).
-// group layout: y*scale + shift from the clip's GroupNorm statistics;
-// layer layout: bias, then LayerNorm over the 512 channels of the frame (the
-// two halves' partial sums meet in shared memory).
-__global__ void __launch_bounds__(256, 2)
-conv0_kernel(const float* pcm, int n, int t0, int clip_rows, const float* __restrict__ w0,
-             const float* __restrict__ b0, const float* __restrict__ gamma, const float* __restrict__ beta,
-             const float2* scale_shift, int layer_norm, float eps, int act, __half* __restrict__ out) {
-  // scale_shift is written by the previous kernel (programmatic dependent
-  // launch): it is read with plain coherent loads after pdl_wait(), never
-  // through a restrict/read-only path that could be hoisted above the wait.
-  __shared__ float red[2][4][2];
-  if (threadIdx.x == 0) pdl_launch_dependents();
-  const int b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f = warp >> 1;   // frame slot of this CTA iteration
-  const int hh = warp & 1;   // channel half
-  float w[8][kK0], sa[8], sb[8], bias[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int c = hh * 256 + 2 * lane + 64 * (k >> 1) + (k & 1);
-#pragma unroll
-    for (int j = 0; j < kK0; ++j) w[k][j] = __ldg(w0 + c * kK0 + j);
-    if (layer_norm) {
-      sa[k] = __ldg(gamma + c);
-      sb[k] = __ldg(beta + c);
-      bias[k] = b0 ? __ldg(b0 + c) : 0.f;
-    }
-  }
-  pdl_wait();
-  if (!layer_norm) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int c = hh * 256 + 2 * lane + 64 * (k >> 1) + (k & 1);
-      const float2 v = scale_shift[b * kC + c];
-      sa[k] = v.x;
-      sb[k] = v.y;
-      bias[k] = 0.f;
-    }
-  }
-  const float* x = pcm + static_cast<int64_t>(b) * n;
-  __half* ob = out + static_cast<int64_t>(b) * clip_rows * kC;
-  // The frame loop bound is uniform across the CTA (barriers inside).
-  for (int base = blockIdx.x * 4; base < t0; base += gridDim.x * 4) {
-    const int t = base + f;
-    const bool live = t < t0;
-    float y[8];
-    if (live) {
-      float xw[kK0];
-#pragma unroll
-      for (int j = 0; j < kK0; ++j) xw[j] = x[kS0 * t + j];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float a = bias[k];
-#pragma unroll
-        for (int j = 0; j < kK0; ++j) a = fmaf(w[k][j], xw[j], a);
-        y[k] = a;
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) y[k] = 0.f;
-    }
-    if (layer_norm) {
-      float s1 = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) s1 += y[k];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      if (lane == 0) red[0][f][hh] = s1;
-      __syncthreads();
-      const float mean = (red[0][f][0] + red[0][f][1]) * (1.0f / kC);
-      float s2 = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float d = y[k] - mean;
-        s2 += d * d;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-      if (lane == 0) red[1][f][hh] = s2;
-      __syncthreads();
-      const float rstd = rsqrtf((red[1][f][0] + red[1][f][1]) * (1.0f / kC) + eps);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) y[k] = (y[k] - mean) * rstd;
-    }
-    if (live) {
-      __half* orow = ob + static_cast<int64_t>(t) * kC + hh * 256 + 2 * lane;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<__half2*>(orow + 64 * i) =
-            __floats2half2_rn(apply_act(fmaf(y[2 * i], sa[2 * i], sb[2 * i]), act),
-                              apply_act(fmaf(y[2 * i + 1], sa[2 * i + 1], sb[2 * i + 1]), act));
-    }
-    if (layer_norm) __syncthreads();  // red[] is rewritten next iteration
-  }
-}
-
-cudaError_t launch_conv0(const float* pcm, int n, int batch, int t0, int clip_rows, const float* w0, const float* b0,
-                         const float* gamma, const float* beta, const float2* scale_shift, int layer_norm, float eps,
-                         int act, __half* out, cudaStream_t st) {
-  int nbx = (t0 + 4 * 16 - 1) / (4 * 16);  // ~16 frames per warp pair
-  if (nbx > 148 * 2 * 4) nbx = 148 * 2 * 4;
-  if (nbx < 1) nbx = 1;
-  return launch_pdl(conv0_kernel, dim3(nbx, batch), dim3(256), 0, st, pcm, n, t0, clip_rows, w0, b0, gamma, beta,
-                    scale_shift, layer_norm, eps, act, out);
 }
 
 // ------------------------------------------------------------------ LayerNorm

@@ -164,6 +164,7 @@ struct w2v_model {
   void* ws = nullptr;
   // weights
   float *c0w = nullptr, *c0b = nullptr, *c0g = nullptr, *c0beta = nullptr;
+  __half* c0wp = nullptr;  // conv-0 taps for the tensor core, [2][512][8] fp16
   __half* cw[7] = {};
   float* cb[7] = {};
   float* cg[7] = {};
@@ -543,8 +544,8 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
                              m->gn_ss, st));
   }
   LAUNCH(W2V_K_CONV0, 2.0 * 10 * kC * p.T[0] * B, 4.0 * p.n * B + 2.0 * kC * p.T[0] * B,
-         launch_conv0(pcm, p.n, B, p.T[0], p.Tpad[0], m->c0w, m->c0b, m->c0g, m->c0beta, m->gn_ss, c.conv_norm,
-                      eps, act, m->act_a, st));
+         launch_conv0_tc(pcm, p.n, B, p.T[0], p.Tpad[0], m->c0wp, m->c0b, m->c0g, m->c0beta, m->gn_ss, c.conv_norm,
+                         eps, act, m->act_a, m->err_word, st));
   for (int i = 1; i < 7; ++i) {
     const GemmEpilogue e = epi_conv(m, p, i);
     const double K = p.convS[i].K;
@@ -684,7 +685,8 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     return W2V_EDEVICE;
   }
 
-  if (gemm_prepare() != cudaSuccess || posconv_prepare() != cudaSuccess || attention_prepare() != cudaSuccess) {
+  if (gemm_prepare() != cudaSuccess || posconv_prepare() != cudaSuccess || attention_prepare() != cudaSuccess ||
+      conv0_prepare() != cudaSuccess) {
     std::fprintf(stderr, "w2v_create: cannot configure kernels: %s\n", cudaGetErrorString(cudaGetLastError()));
     return W2V_ECUDA;
   }
@@ -725,6 +727,13 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   };
 
   put_f32(reinterpret_cast<void**>(&m->c0w), src("conv0.weight"), kC * 10);
+  {
+    const float* w = src("conv0.weight");  // [512][1][10]
+    put_f16(reinterpret_cast<void**>(&m->c0wp), 2 * kC * 8, [&](size_t i) {
+      const size_t kc = i / (kC * 8), rem = i % (kC * 8), ch = rem / 8, j = kc * 8 + rem % 8;
+      return j < 10 ? w[ch * 10 + j] : 0.f;
+    });
+  }
   if (c.conv_bias)
     put_f32(reinterpret_cast<void**>(&m->c0b), src("conv0.bias"), kC);
   put_f32(reinterpret_cast<void**>(&m->c0g), src("conv0.norm.weight"), kC);

@@ -100,12 +100,15 @@ int gn_moment_blocks(int t0);
 cudaError_t launch_gn_moments(const float* pcm, int n, int batch, int t0, const float* w0, const float* gamma,
                               const float* beta, float eps, double* partial, unsigned* ticket, float2* scale_shift,
                               cudaStream_t st);
-// conv0 + norm + GELU -> fp16 [batch][clip_rows][512] (rows >= t0 untouched).
+// conv0 + norm + GELU on the tensor core -> fp16 [batch][clip_rows][512]
+// (rows >= t0 untouched).  wpack: fp16 taps [2][512][8] (tap j of channel c
+// at [j/8][c][j%8], taps 10..15 zero).
 //   group layout: per-channel scale/shift from launch_gn_moments,
 //   layer layout: conv bias, per-frame LayerNorm over the 512 channels.
-cudaError_t launch_conv0(const float* pcm, int n, int batch, int t0, int clip_rows, const float* w0, const float* b0,
-                         const float* gamma, const float* beta, const float2* scale_shift, int layer_norm, float eps,
-                         int act, __half* out, cudaStream_t st);
+cudaError_t conv0_prepare();
+cudaError_t launch_conv0_tc(const float* pcm, int n, int batch, int t0, int clip_rows, const __half* wpack,
+                            const float* b0, const float* gamma, const float* beta, const float2* scale_shift,
+                            int layer_norm, float eps, int act, __half* out, int* err, cudaStream_t st);
 // Row LayerNorm over `cols` channels (512, 768 or 1024), fp16 or fp32 input,
 // fp16 output, optional GELU after the affine.
 cudaError_t launch_layernorm(const void* x, int in_f32, __half* y, int rows, int cols, const float* gamma,
