@@ -7,19 +7,26 @@
 //               2-deep ring
 //   warp 1      TMEM owner; one thread issues S_j = Q K_j^T (M=128, N=128,
 //               K=64) into one of two TMEM score buffers and, once P_j is in
-//               shared memory, O_j = P_j V_j (M=128, N=64, K=128).  S_{j+1} is
-//               issued before waiting for P_j, so the next scores are computed
-//               while the softmax of the current tile runs.
+//               shared memory, O += P_j [V_j | 1] (M=128, N=80, K=128) into a
+//               TMEM accumulator that lives across all key tiles.  S_{j+1} is
+//               issued before waiting for P_j.
 //   warps 2-17  softmax: four warps per TMEM lane quarter, each owning 32 of
 //               the 128 key columns (and 16 of the 64 output columns) of its
-//               32 query rows.  Row maxima and sums are combined through shared
-//               memory with a 128-thread named barrier per quarter.  fp32 online
-//               softmax with exp2 (1/8 scale folded in), P rounded to fp16
-//               into the 128-byte-swizzled K-major layout the MMA reads, O
-//               accumulated in registers with the running rescale.
+//               32 query rows; the tile's row maximum is combined through
+//               shared memory with a 128-thread named barrier per quarter.
+// Online softmax with a lazily moved reference: a row's reference maximum m
+// (log2 units, 1/8 scale folded in) moves only when the tile's maximum exceeds
+// it by more than 8, so P = 2^(s/8 log2 e - m) stays <= 256 and the rescale of
+// the TMEM accumulator (wait for the previous P V, load, scale, store) is rare;
+// otherwise no softmax step waits for the tensor core.  P is formed as packed
+// fp16 pairs (packed fp32 FMA, rounding, fp16x2 exponent) and written in the
+// 128-byte-swizzled K-major layout the MMA reads, double-buffered.  The row sum
+// is not accumulated by the threads: V^T carries a 65th row of ones, so column
+// 64 of the accumulator is sum_k P[r][k] computed from the same fp16 P that
+// multiplies V.
 // V arrives transposed ([clip][head][64][T], written by the QKV projection's
 // epilogue) so both MMAs read K-major operands.  Keys past T are zero-filled by
-// TMA and masked before the exponent.
+// TMA and masked to -inf before the exponent.
 #include "ptx.cuh"
 #include "w2v_internal.h"
 
@@ -27,11 +34,12 @@ namespace w2v {
 
 struct AttnSmem {
   static constexpr int Q = 0;
-  static constexpr int K0 = 16384;
-  static constexpr int V0 = K0 + 2 * 16384;
-  static constexpr int P = V0 + 2 * 16384;
-  static constexpr int RED = P + 32768;       // float red_max[2][4][128], red_sum[4][128]
-  static constexpr int BAR = RED + 6144;
+  static constexpr int K0 = 16384;                 // [2 stages] 128 keys x 64 dims, SW128
+  static constexpr int kVHalf = 10240;             // 80 rows (64 dims + ones + zeros) x 64 keys
+  static constexpr int V0 = K0 + 2 * 16384;        // [2 stages][2 key halves] kVHalf
+  static constexpr int P = V0 + 4 * kVHalf;        // [2 buffers] 128 rows x 128 keys fp16, SW128
+  static constexpr int RED = P + 2 * 32768;        // float red_max[2][4][128]
+  static constexpr int BAR = RED + 4096;
   static constexpr int TOTAL = BAR + 256 + 1024;
 };
 
@@ -40,6 +48,7 @@ constexpr int kAttnThreads = 64 + 32 * kSoftWarps;
 constexpr int kSubs = kSoftWarps / 4;    // warps per TMEM lane quarter
 constexpr int kSCols = 128 / kSubs;      // score columns per warp
 constexpr int kOCols = 64 / kSubs;       // output columns per warp
+constexpr float kLazyLimit = 8.0f;       // log2 of the largest P value allowed (256)
 
 __device__ __forceinline__ void quarter_barrier(int q) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kSubs) : "memory");
@@ -51,15 +60,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red_max = reinterpret_cast<float*>(smem + AttnSmem::RED);  // [slot][sub][row]
-  float* red_sum = red_max + 2 * kSubs * 128;                       // [sub][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* p_full = bars + 7;
-  uint64_t* o_full = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* p_full = bars + 7;    // [2]
+  uint64_t* pv_done = bars + 9;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -67,14 +75,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(&kv_full[0], 1);
-    mbar_init(&kv_full[1], 1);
-    mbar_init(&kv_empty[0], 1);
-    mbar_init(&kv_empty[1], 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 32 * kSoftWarps);
-    mbar_init(o_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 32 * kSoftWarps);
+      mbar_init(&pv_done[i], 1);
+    }
     fence_mbar_init();
     pdl_launch_dependents();
   }
@@ -87,11 +94,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  // Rows 64..79 of every V^T half-tile: row 64 all ones (fp16 1.0), the rest
+  // zero.  They sit in the last two 1 KB swizzle atoms of each half-tile; a row
+  // of identical 16-byte chunks is unchanged by the swizzle.
+  for (int i = threadIdx.x; i < 4 * 2048 / 16; i += kAttnThreads) {
+    const int half = i / 128, off = (i % 128) * 16;
+    const uint32_t v = off < 128 ? 0x3C003C00u : 0u;
+    *reinterpret_cast<uint4*>(smem + AttnSmem::V0 + half * AttnSmem::kVHalf + 8192 + off) = make_uint4(v, v, v, v);
+  }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 256;
+  const uint32_t tO = tmem + 256;   // 80 columns: O (64) | row sum | zeros
 
   if (warp == 0) {
     if (lane == 0) {
@@ -109,9 +125,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           break;
         }
         mbar_arrive_expect_tx(&kv_full[st], 32768);
+        uint8_t* vs = smem + AttnSmem::V0 + st * 2 * AttnSmem::kVHalf;
         tma_load_3d(smem + AttnSmem::K0 + st * 16384, &tmK, &kv_full[st], h * 64, j * 128, b);
-        tma_load_2d(smem + AttnSmem::V0 + st * 16384, &tmVt, &kv_full[st], j * 128, vrow);
-        tma_load_2d(smem + AttnSmem::V0 + st * 16384 + 8192, &tmVt, &kv_full[st], j * 128 + 64, vrow);
+        tma_load_2d(vs, &tmVt, &kv_full[st], j * 128, vrow);
+        tma_load_2d(vs + AttnSmem::kVHalf, &tmVt, &kv_full[st], j * 128 + 64, vrow);
         issued = j + 1;
       }
       if (!ok) {
@@ -122,9 +139,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16_f32(128, 128);
-      constexpr uint32_t idO = idesc_f16_f32(128, 64);
+      constexpr uint32_t idO = idesc_f16_f32(128, 80);
       const uint32_t sQ = smem_u32(smem + AttnSmem::Q);
-      const uint32_t sP = smem_u32(smem + AttnSmem::P);
       auto issue_s = [&](int j) {
         const uint32_t sK = smem_u32(smem + AttnSmem::K0 + (j & 1) * 16384);
         const uint32_t tS = tmem + (j & 1) * 128;
@@ -138,6 +154,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         issue_s(0);
       }
       for (int j = 0; ok && j < nkv; ++j) {
+        // S_{j+1} reuses the score buffer of S_{j-1}, whose softmax finished
+        // reading it before P_{j-1} was published.
         if (j + 1 < nkv) {
           if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) {
             ok = false;
@@ -146,19 +164,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tc_fence_after();
           issue_s(j + 1);
         }
-        if (!mbar_wait(p_full, j & 1)) {
+        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + AttnSmem::V0 + (j & 1) * 16384);
+        const uint32_t sP = smem_u32(smem + AttnSmem::P + (j & 1) * 32768);
+        const uint32_t sV = smem_u32(smem + AttnSmem::V0 + (j & 1) * 2 * AttnSmem::kVHalf);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t a = sP + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t bv = sV + (kk >> 2) * 8192 + (kk & 3) * 32;
-          umma_f16(tO, desc_sw128(a), desc_sw128(bv), idO, kk);
+          const uint32_t bv = sV + (kk >> 2) * AttnSmem::kVHalf + (kk & 3) * 32;
+          umma_f16(tO, desc_sw128(a), desc_sw128(bv), idO, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(o_full);
+        umma_commit(&pv_done[j & 1]);
         umma_commit(&kv_empty[j & 1]);
       }
       if (!ok) atomicOr(err, kErrWaitMma);
@@ -169,12 +188,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float c = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
-    float o[kOCols];
-#pragma unroll
-    for (int i = 0; i < kOCols; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f;
-    // This warp's 32 keys are half of the 64-key swizzle atom (sub >> 1).
-    uint8_t* prow = smem + AttnSmem::P + (sub >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+    float m_ref = -INFINITY;                        // reference maximum, log2 units
+    // This warp's 32 keys are half of a 64-key swizzle atom (sub >> 1).
+    const int prow_off = AttnSmem::P + (sub >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     const int ch0 = (sub & 1) * 4;
     bool ok = true;
     // Every iteration runs the quarter barrier and the p_full arrival even
@@ -188,76 +204,91 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (ok) {
         tc_fence_after();
         tmem_ld32(tmem + (j & 1) * 128 + sub * kSCols + lane_base, s);
+        if (nvalid < kSCols) {
 #pragma unroll
-        for (int i = 0; i < kSCols; ++i)
-          if (i < nvalid) mx = fmaxf(mx, s[i]);
+          for (int i = 0; i < kSCols; ++i)
+            if (i >= nvalid) s[i] = -INFINITY;
+        }
+        float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+#pragma unroll
+        for (int i = 6; i + 3 < kSCols; i += 4) {
+          m0 = fmax3(m0, s[i], s[i + 1]);
+          m1 = fmax3(m1, s[i + 2], s[i + 3]);
+        }
+        mx = fmax3(m0, m1, s[kSCols - 2]);
+        mx = fmaxf(mx, s[kSCols - 1]);
       }
       float* slot = red_max + (j & 1) * (kSubs * 128);
       slot[sub * 128 + r] = mx;
       quarter_barrier(q);
+      mx = fmaxf(fmaxf(slot[r], slot[128 + r]), fmaxf(slot[256 + r], slot[384 + r]));
+      const float mt = mx * c;  // finite: every key tile has a valid column
+      // Move the reference when the tile's maximum is more than 2^8 above it.
+      // The four warps of a row see the same mt and m_ref and decide alike.
+      const bool move = mt > m_ref + kLazyLimit;
+      if (__any_sync(0xffffffffu, move)) {
+        const float m_new = move ? mt : m_ref;
+        if (j > 0 && ok) {
+          // Rescale this warp's accumulator columns (and, for sub 0, the row
+          // sum column) once the previous P V has landed.
+          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
+          if (ok) {
+            tc_fence_after();
+            const float alpha = ex2_approx(m_ref - m_new);
+            float v[16];
+            tmem_ld16(tO + lane_base + sub * kOCols, v);
 #pragma unroll
-      for (int k = 0; k < kSubs; ++k) mx = fmaxf(mx, slot[k * 128 + r]);
-      const float m_new = fmaxf(m, mx * c);
-      const float alpha = ex2_approx(m - m_new);
-      float rs = 0.f;
-      uint32_t pk[kSCols / 2];
+            for (int i = 0; i < 16; ++i) v[i] *= alpha;
+            tmem_st16(tO + lane_base + sub * kOCols, v);
+            if (sub == 0) {
+              tmem_ld16(tO + lane_base + 64, v);
 #pragma unroll
-      for (int i = 0; i < kSCols; i += 2) {
-        const float p0 = (i < nvalid) ? ex2_approx(fmaf(s[i], c, -m_new)) : 0.f;
-        const float p1 = (i + 1 < nvalid) ? ex2_approx(fmaf(s[i + 1], c, -m_new)) : 0.f;
-        __half2 hp = __floats2half2_rn(p0, p1);
-        rs += p0 + p1;  // fp32 row sum (the conversion unit is the scarce pipe here)
-        pk[i / 2] = *reinterpret_cast<uint32_t*>(&hp);
-      }
-      if (j > 0 && ok) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1));
-        if (ok) {
-          tc_fence_after();
-          float v[16];
-          tmem_ld16(tO + lane_base + sub * kOCols, v);
-#pragma unroll
-          for (int i = 0; i < kOCols; ++i) o[i] = (o[i] + v[i]) * alpha;
+              for (int i = 0; i < 16; ++i) v[i] *= alpha;
+              tmem_st16(tO + lane_base + 64, v);
+            }
+          }
         }
+        m_ref = m_new;
       }
-      l = l * alpha + rs;
-      m = m_new;
+      uint32_t pk[kSCols / 2];
+      const float nb = -m_ref;
+#pragma unroll
+      for (int i = 0; i < kSCols; i += 2) pk[i / 2] = exp2_affine_f16x2(s[i], s[i + 1], c, nb);
+      // P buffer j & 1 was last read by P_{j-2} V_{j-2}.
+      if (j >= 2 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1));
+      uint8_t* prow = smem + prow_off + (j & 1) * 32768;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch)
         *reinterpret_cast<uint4*>(prow + (((ch0 + ch) ^ (r & 7)) << 4)) =
             make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, (nkv - 1) & 1));
+    const int last = nkv - 1;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[last & 1], (last >> 1) & 1));
+    const int t = qt * 128 + r;
     if (ok) {
       tc_fence_after();
-      float v[16];
-      tmem_ld16(tO + lane_base + sub * kOCols, v);
+      float o[16];
+      tmem_ld16(tO + lane_base + sub * kOCols, o);
+      const float l = tmem_ld1(tO + lane_base + 64);
+      if (t < T) {
+        const float inv = 1.0f / l;
+        __half* dst = out + (static_cast<int64_t>(b) * T + t) * (H * 64) + h * 64 + sub * kOCols;
 #pragma unroll
-      for (int i = 0; i < kOCols; ++i) o[i] += v[i];
+        for (int i = 0; i < kOCols; i += 8) {
+          __half2 h0 = __floats2half2_rn(o[i] * inv, o[i + 1] * inv);
+          __half2 h1 = __floats2half2_rn(o[i + 2] * inv, o[i + 3] * inv);
+          __half2 h2 = __floats2half2_rn(o[i + 4] * inv, o[i + 5] * inv);
+          __half2 h3 = __floats2half2_rn(o[i + 6] * inv, o[i + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + i) =
+              make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                         *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+        }
+      }
     } else if (lane == 0) {
       atomicOr(err, kErrWaitSoftmax);
-    }
-    red_sum[sub * 128 + r] = l;
-    quarter_barrier(q);
-    float ltot = 0.f;
-#pragma unroll
-    for (int k = 0; k < kSubs; ++k) ltot += red_sum[k * 128 + r];
-    const int t = qt * 128 + r;
-    if (ok && t < T) {
-      const float inv = 1.0f / ltot;
-      __half* dst = out + (static_cast<int64_t>(b) * T + t) * (H * 64) + h * 64 + sub * kOCols;
-#pragma unroll
-      for (int i = 0; i < kOCols; i += 8) {
-        __half2 h0 = __floats2half2_rn(o[i] * inv, o[i + 1] * inv);
-        __half2 h1 = __floats2half2_rn(o[i + 2] * inv, o[i + 3] * inv);
-        __half2 h2 = __floats2half2_rn(o[i + 4] * inv, o[i + 5] * inv);
-        __half2 h3 = __floats2half2_rn(o[i + 6] * inv, o[i + 7] * inv);
-        *reinterpret_cast<uint4*>(dst + i) =
-            make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                       *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
-      }
     }
   }
 

@@ -210,6 +210,33 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// One column variant.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r)
+      : "r"(taddr)
+      : "memory");
+  return __uint_as_float(r);
+}
+
+// Stores 16 consecutive 32-bit TMEM columns of this warp's 32 lanes and waits
+// for the store to complete.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05 form): start address, leading and
 // stride byte offsets (all >> 4), descriptor version 1 at bit 46, layout
 // (swizzle) type at bits 61..63.
@@ -292,6 +319,26 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^(s0 c + b), 2^(s1 c + b) as a packed fp16 pair (s0 in the low half): one
+// packed fp32 FMA, one rounding to fp16x2 and one fp16x2 exponent.
+__device__ __forceinline__ uint32_t exp2_affine_f16x2(float s0, float s1, float c, float b) {
+  uint32_t out;
+  asm("{\n\t.reg .b64 sv, cv, bv, xv;\n\t.reg .f32 x0, x1;\n\t.reg .b32 h;\n\t"
+      "mov.b64 sv, {%1, %2};\n\tmov.b64 cv, {%3, %3};\n\tmov.b64 bv, {%4, %4};\n\t"
+      "fma.rn.f32x2 xv, sv, cv, bv;\n\tmov.b64 {x0, x1}, xv;\n\t"
+      "cvt.rn.f16x2.f32 h, x1, x0;\n\tex2.approx.f16x2 %0, h;\n\t}"
+      : "=r"(out)
+      : "f"(s0), "f"(s1), "f"(c), "f"(b));
+  return out;
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ float tanh_approx(float x) {

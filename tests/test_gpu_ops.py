@@ -115,14 +115,25 @@ def _attn_ref(q, k, v, H):
     return out
 
 
-@pytest.mark.parametrize("batch,T,H", [(1, 1, 1), (1, 7, 2), (1, 128, 1), (2, 129, 2), (1, 799, 12),
-                                       (2, 499, 3), (1, 1000, 2), (1, 256, 16)])
-def test_attention_matches_oracle(batch, T, H):
-    g = torch.Generator().manual_seed(T * 31 + H)
+@pytest.mark.parametrize("batch,T,H,growth", [(1, 1, 1, 0), (1, 7, 2, 0), (1, 128, 1, 0), (2, 129, 2, 0),
+                                              (1, 799, 12, 0), (2, 499, 3, 0), (1, 1000, 2, 0), (1, 256, 16, 0),
+                                              (1, 799, 2, 1), (2, 640, 2, 2)])
+def test_attention_matches_oracle(batch, T, H, growth):
+    """growth > 0 makes later key tiles score much higher than the first ones
+    (growth 1: key t scaled by 1 + 4 t / T and the queries by 2; growth 2: every
+    128-key block scaled by twice the previous one), so a row's running maximum
+    rises by more than 2^8 across tiles and the accumulator rescale runs."""
+    g = torch.Generator().manual_seed(T * 31 + H + 7 * growth)
     d = 64 * H
-    q = torch.randn(batch, T, d, generator=g).half()
-    k = torch.randn(batch, T, d, generator=g).half()
+    q = torch.randn(batch, T, d, generator=g)
+    k = torch.randn(batch, T, d, generator=g)
     v = torch.randn(batch, T, d, generator=g).half()
+    if growth == 1:
+        q = q * 2.0
+        k = k * (1.0 + 4.0 * torch.arange(T, dtype=torch.float32) / T)[None, :, None]
+    elif growth == 2:
+        k = k * (2.0 ** (torch.arange(T) // 128).float())[None, :, None] * 0.5
+    q, k = q.half(), k.half()
     t_pad = (T + 7) // 8 * 8
     vt = torch.zeros(batch, H, 64, t_pad, dtype=torch.float16)
     vt[..., :T] = v.view(batch, T, H, 64).permute(0, 2, 3, 1)
