@@ -24,8 +24,9 @@ constexpr int kTaps = 10;
 constexpr int kHop = 5;
 constexpr int A_OFF = 0;                   // [2 k-chunks][128 rows][8] fp16, 4 KB
 constexpr int B_OFF = 4096;                // [2 k-chunks][512 rows][8] fp16, 16 KB
-constexpr int P_OFF = B_OFF + 16384;       // float2 params[512]: (scale, shift) or (gamma, beta)
-constexpr int BIAS_OFF = P_OFF + 4096;     // float bias[512]
+constexpr int PA_OFF = B_OFF + 16384;      // float[512]: GroupNorm scale, or LayerNorm gamma
+constexpr int PB_OFF = PA_OFF + 2048;      // float[512]: GroupNorm shift, or LayerNorm beta
+constexpr int BIAS_OFF = PB_OFF + 2048;    // float bias[512]
 constexpr int kEpiWarps = 16;              // 4 per TMEM lane quarter, 128 channels each
 constexpr int kCols = 512 / (kEpiWarps / 4);
 constexpr int RED_OFF = BIAS_OFF + 2048;   // float red[4 slices][128 rows]
@@ -35,16 +36,17 @@ constexpr int SMEM = BAR_OFF + 64 + 1024;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 }  // namespace
 
+template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
 conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int n, int t0,
                 const __half* __restrict__ wpack, const float* __restrict__ b0, const float* __restrict__ gamma,
-                const float* __restrict__ beta, const float2* scale_shift, int layer_norm, float eps, int act,
-                int* err) {
+                const float* __restrict__ beta, const float2* scale_shift, int layer_norm, float eps, int* err) {
   // pcm and scale_shift may be written by the previous kernel (programmatic
   // dependent launch): plain coherent loads after pdl_wait() only.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float2* par = reinterpret_cast<float2*>(smem + P_OFF);
+  float* pa = reinterpret_cast<float*>(smem + PA_OFF);
+  float* pb = reinterpret_cast<float*>(smem + PB_OFF);
   float* bias = reinterpret_cast<float*>(smem + BIAS_OFF);
   float* red = reinterpret_cast<float*>(smem + RED_OFF);
   uint64_t* w_full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
@@ -70,13 +72,18 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
   }
   if (layer_norm) {
     for (int c = threadIdx.x; c < kC0; c += kThreads) {
-      par[c] = make_float2(gamma[c], beta[c]);
+      pa[c] = gamma[c];
+      pb[c] = beta[c];
       bias[c] = b0 ? b0[c] : 0.f;
     }
   }
   pdl_wait();
   if (!layer_norm)
-    for (int c = threadIdx.x; c < kC0; c += kThreads) par[c] = scale_shift[b * kC0 + c];
+    for (int c = threadIdx.x; c < kC0; c += kThreads) {
+      const float2 ss = scale_shift[b * kC0 + c];
+      pa[c] = ss.x;
+      pb[c] = ss.y;
+    }
   // A tile: row t holds pcm[5 (f0 + t) + j], j < 10, then zeros; 16-byte
   // chunk (row, k-chunk) at k-chunk * 2048 + row * 16 (no-swizzle core matrices).
   if (threadIdx.x < 256) {
@@ -124,6 +131,9 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
     bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
     if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
     tc_fence_after();
+    // Per element: pre-activation a = v * A + B with per-channel (A, B) pairs:
+    // GroupNorm (scale, shift), or for LayerNorm A = rstd gamma and
+    // B = (bias - mean) rstd gamma + beta, folded per 4-channel group below.
     float mean = 0.f, rstd = 1.f;
     if (layer_norm) {
       // Per-frame LayerNorm statistics over all 512 channels (two passes; the
@@ -164,21 +174,41 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
     for (int cb = 0; cb < kCols / 32; ++cb) {
       const int c = cb * 32;
       const int ch = sl * kCols + c;
-      float v[32];
-      if (ok) tmem_ld32(trow + c, v);
       uint32_t hv[16];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float a0, a1;
-        if (layer_norm) {
-          a0 = fmaf((v[i] + bias[ch + i] - mean) * rstd, par[ch + i].x, par[ch + i].y);
-          a1 = fmaf((v[i + 1] + bias[ch + i + 1] - mean) * rstd, par[ch + i + 1].x, par[ch + i + 1].y);
-        } else {
-          a0 = fmaf(v[i], par[ch + i].x, par[ch + i].y);
-          a1 = fmaf(v[i + 1], par[ch + i + 1].x, par[ch + i + 1].y);
+      for (int hh = 0; hh < 2; ++hh) {
+        float v[16];
+        if (ok) tmem_ld16(trow + c + hh * 16, v);
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const int cc = ch + hh * 16 + i;
+          // Warp-uniform addresses: broadcast loads of 4 channels' parameters.
+          const float4 A4 = *reinterpret_cast<const float4*>(pa + cc);
+          const float4 B4 = *reinterpret_cast<const float4*>(pb + cc);
+          float2 a01, a23;
+          if (layer_norm) {
+            const float4 c4 = *reinterpret_cast<const float4*>(bias + cc);
+            // ((v + bias) - mean) * rstd * gamma + beta
+            const float2 m2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
+            a01 = fmul2(fadd2(fadd2(make_float2(v[i], v[i + 1]), make_float2(c4.x, c4.y)), m2), r2);
+            a23 = fmul2(fadd2(fadd2(make_float2(v[i + 2], v[i + 3]), make_float2(c4.z, c4.w)), m2), r2);
+            a01 = ffma2(a01, make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
+            a23 = ffma2(a23, make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
+          } else {
+            a01 = ffma2(make_float2(v[i], v[i + 1]), make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
+            a23 = ffma2(make_float2(v[i + 2], v[i + 3]), make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
+          }
+          if (ACT == 2) {
+            a01 = gelu_tanh2(a01);
+            a23 = gelu_tanh2(a23);
+          } else if (ACT == 1) {
+            a01 = make_float2(gelu_erf(a01.x), gelu_erf(a01.y));
+            a23 = make_float2(gelu_erf(a23.x), gelu_erf(a23.y));
+          }
+          __half2 h01 = __floats2half2_rn(a01.x, a01.y), h23 = __floats2half2_rn(a23.x, a23.y);
+          hv[hh * 8 + i / 2] = *reinterpret_cast<uint32_t*>(&h01);
+          hv[hh * 8 + i / 2 + 1] = *reinterpret_cast<uint32_t*>(&h23);
         }
-        __half2 h2 = __floats2half2_rn(apply_act(a0, act), apply_act(a1, act));
-        hv[i / 2] = *reinterpret_cast<uint32_t*>(&h2);
       }
       // 32 rows x 32 channels box, 64-byte rows, 64-byte swizzle.
       uint8_t* box = stage + cb * 2048;
@@ -204,7 +234,10 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
 }
 
 cudaError_t conv0_prepare() {
-  return cudaFuncSetAttribute(conv0_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t r = cudaFuncSetAttribute(conv0_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (r == cudaSuccess) r = cudaFuncSetAttribute(conv0_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (r == cudaSuccess) r = cudaFuncSetAttribute(conv0_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  return r;
 }
 
 cudaError_t launch_conv0_tc(const float* pcm, int n, int batch, int t0, int clip_rows, const __half* wpack,
@@ -218,8 +251,9 @@ cudaError_t launch_conv0_tc(const float* pcm, int n, int batch, int t0, int clip
   cudaError_t r = make_tmap(&tm, out, 3, dims, str, box, 2, 64);
   if (r != cudaSuccess) return r;
   dim3 grid((t0 + 127) / 128, 1, batch);
-  return launch_pdl(conv0_tc_kernel, grid, dim3(kThreads), SMEM, st, tm, pcm, n, t0, wpack, b0, gamma, beta,
-                    scale_shift, layer_norm, eps, act, err);
+  auto k = act == 2 ? conv0_tc_kernel<2> : (act == 1 ? conv0_tc_kernel<1> : conv0_tc_kernel<0>);
+  return launch_pdl(k, grid, dim3(kThreads), SMEM, st, tm, pcm, n, t0, wpack, b0, gamma, beta, scale_shift,
+                    layer_norm, eps, err);
 }
 
 }  // namespace w2v

@@ -367,6 +367,53 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return x * rcp_approx(1.0f + e);
 }
 
+// Packed fp32 pair arithmetic (one f32x2 instruction for two lanes of data).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 av, bv, cv, dv;\n\tmov.b64 av, {%2, %3};\n\tmov.b64 bv, {%4, %5};\n\t"
+      "mov.b64 cv, {%6, %7};\n\tfma.rn.f32x2 dv, av, bv, cv;\n\tmov.b64 {%0, %1}, dv;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 av, bv, dv;\n\tmov.b64 av, {%2, %3};\n\tmov.b64 bv, {%4, %5};\n\t"
+      "mul.rn.f32x2 dv, av, bv;\n\tmov.b64 {%0, %1}, dv;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 av, bv, dv;\n\tmov.b64 av, {%2, %3};\n\tmov.b64 bv, {%4, %5};\n\t"
+      "add.rn.f32x2 dv, av, bv;\n\tmov.b64 {%0, %1}, dv;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// tanh-form GELU of a pair in the same sigmoid form as gelu_tanh, with the
+// exponent taken as fp16x2: the argument w = -2 sqrt(2/pi) log2(e) u is
+// rounded to fp16 (relative error of 2^w below 2^-11 |w| ln 2) and 1 / (1 + e)
+// passes that error on scaled by e / (1 + e) <= 1, so the result stays within
+// about one fp16 ulp of the fp32 form.
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) {
+  const float k2 = -2.0f * 0.7978845608028654f * 1.4426950408889634f;
+  const float2 x2 = fmul2(x, x);
+  const float2 in = ffma2(x2, make_float2(k2 * 0.044715f, k2 * 0.044715f), make_float2(k2, k2));
+  const float2 w = fmul2(x, in);
+  uint32_t eh;
+  asm("{\n\t.reg .b32 h;\n\tcvt.rn.f16x2.f32 h, %2, %1;\n\tex2.approx.f16x2 %0, h;\n\t}"
+      : "=r"(eh)
+      : "f"(w.x), "f"(w.y));
+  const float2 e = __half22float2(*reinterpret_cast<const __half2*>(&eh));
+  const float2 d = fadd2(e, make_float2(1.0f, 1.0f));
+  return fmul2(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 __device__ __forceinline__ float apply_act(float x, int act) {
   if (act == 1) return gelu_erf(x);
   if (act == 2) return gelu_tanh(x);
