@@ -107,9 +107,11 @@ int w2v_create(const w2v_config* cfg, const float* host_weights, size_t n_floats
  * pcm_dev (float32 [batch][n_samples], already normalised).  Writes
  * logits_dev (float32 [batch][T][vocab], T = w2v_num_frames(n_samples)).
  * The first call for a given (n_samples, batch) builds that shape's launch
- * plan: it times the tile and split-K candidates of every GEMM on the device
- * (a few milliseconds, synchronous; W2V_AUTOTUNE=0 in the environment uses a
- * cost model instead), so make that first call outside any stream capture.
+ * plan: it times the tile and split-K candidates of every GEMM on the device,
+ * then re-chooses the per-layer GEMMs by timing the whole forward with each
+ * candidate (a few hundred milliseconds, synchronous; W2V_AUTOTUNE=0 in the
+ * environment uses a cost model instead, W2V_TUNE_LOG=1 prints the choices),
+ * so make that first call outside any stream capture.
  * Errors: W2V_ESHAPE if n_samples < 400 or > max_samples or batch outside
  * [1, max_batch]; W2V_EINVAL for null/misaligned pointers. */
 int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, void* stream);

@@ -4,12 +4,16 @@
 //
 // One CTA per (128-query tile, head, clip), 576 threads:
 //   warp 0      TMA: the Q tile once, then K and V^T tiles of 128 keys into a
-//               2-deep ring
+//               3-deep ring
 //   warp 1      TMEM owner; one thread issues S_j = Q K_j^T (M=128, N=128,
-//               K=64) into one of two TMEM score buffers and, once P_j is in
+//               K=64) into one of three TMEM score buffers and, once P_j is in
 //               shared memory, O += P_j [V_j | 1] (M=128, N=80, K=128) into a
-//               TMEM accumulator that lives across all key tiles.  S_{j+1} is
-//               issued before waiting for P_j.
+//               TMEM accumulator that lives across all key tiles.  The scores
+//               run two tiles ahead (S_{j+2} is issued before waiting for
+//               P_j), so the softmax never waits behind a P V product: every
+//               tcgen05.mma of M=128, K=16 occupies the tensor pipe about the
+//               same ~100-140 cycles whatever its N up to 192, which makes the
+//               eight P V instructions per tile the longer of the two chains.
 //   warps 2-17  softmax: four warps per TMEM lane quarter, each owning 32 of
 //               the 128 key columns (and 16 of the 64 output columns) of its
 //               32 query rows; the tile's row maximum is combined through
@@ -19,7 +23,8 @@
 // it by more than 8, so P = 2^(s/8 log2 e - m) stays <= 256 and the rescale of
 // the TMEM accumulator (wait for the previous P V, load, scale, store) is rare;
 // otherwise no softmax step waits for the tensor core.  P is formed as packed
-// fp16 pairs (packed fp32 FMA, rounding, fp16x2 exponent) and written in the
+// fp16 pairs (packed fp32 FMA, rounding, then the fp16x2 exponent instruction
+// or, for a share of the pairs, a cubic on the FMA pipe) and written in the
 // 128-byte-swizzled K-major layout the MMA reads, double-buffered.  The row sum
 // is not accumulated by the threads: V^T carries a 65th row of ones, so column
 // 64 of the accumulator is sum_k P[r][k] computed from the same fp16 P that
@@ -32,12 +37,14 @@
 
 namespace w2v {
 
+constexpr int kKvStages = 3;
+
 struct AttnSmem {
   static constexpr int Q = 0;
-  static constexpr int K0 = 16384;                 // [2 stages] 128 keys x 64 dims, SW128
-  static constexpr int kVHalf = 10240;             // 80 rows (64 dims + ones + zeros) x 64 keys
-  static constexpr int V0 = K0 + 2 * 16384;        // [2 stages][2 key halves] kVHalf
-  static constexpr int P = V0 + 4 * kVHalf;        // [2 buffers] 128 rows x 128 keys fp16, SW128
+  static constexpr int K0 = 16384;                        // [stages] 128 keys x 64 dims, SW128
+  static constexpr int kVHalf = 10240;                    // 80 rows (64 dims + ones + zeros) x 64 keys
+  static constexpr int V0 = K0 + kKvStages * 16384;       // [stages][2 key halves] kVHalf
+  static constexpr int P = V0 + kKvStages * 2 * kVHalf;   // [2 buffers] 128 rows x 128 keys fp16, SW128
   static constexpr int RED = P + 2 * 32768;        // float red_max[2][4][128]
   static constexpr int BAR = RED + 4096;
   static constexpr int TOTAL = BAR + 256 + 1024;
@@ -49,6 +56,7 @@ constexpr int kSubs = kSoftWarps / 4;    // warps per TMEM lane quarter
 constexpr int kSCols = 128 / kSubs;      // score columns per warp
 constexpr int kOCols = 64 / kSubs;       // output columns per warp
 constexpr float kLazyLimit = 8.0f;       // log2 of the largest P value allowed (256)
+constexpr int kPolyPairs = 6;            // exponential pairs per warp and tile computed by polynomial
 
 __device__ __forceinline__ void quarter_barrier(int q) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kSubs) : "memory");
@@ -62,12 +70,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* red_max = reinterpret_cast<float*>(smem + AttnSmem::RED);  // [slot][sub][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* p_full = bars + 7;    // [2]
-  uint64_t* pv_done = bars + 9;   // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* kv_full = bars + 1;   // [3]
+  uint64_t* kv_empty = bars + 4;  // [3]
+  uint64_t* s_full = bars + 7;    // [3]
+  uint64_t* p_full = bars + 10;   // [2]
+  uint64_t* pv_done = bars + 12;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -75,10 +83,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKvStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], 32 * kSoftWarps);
       mbar_init(&pv_done[i], 1);
     }
@@ -97,7 +107,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   // Rows 64..79 of every V^T half-tile: row 64 all ones (fp16 1.0), the rest
   // zero.  They sit in the last two 1 KB swizzle atoms of each half-tile; a row
   // of identical 16-byte chunks is unchanged by the swizzle.
-  for (int i = threadIdx.x; i < 4 * 2048 / 16; i += kAttnThreads) {
+  for (int i = threadIdx.x; i < kKvStages * 2 * 2048 / 16; i += kAttnThreads) {
     const int half = i / 128, off = (i % 128) * 16;
     const uint32_t v = off < 128 ? 0x3C003C00u : 0u;
     *reinterpret_cast<uint4*>(smem + AttnSmem::V0 + half * AttnSmem::kVHalf + 8192 + off) = make_uint4(v, v, v, v);
@@ -107,7 +117,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 256;   // 80 columns: O (64) | row sum | zeros
+  const uint32_t tO = tmem + 384;   // 80 columns: O (64) | row sum | zeros; scores at 0, 128, 256
 
   if (warp == 0) {
     if (lane == 0) {
@@ -118,8 +128,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1)) {
+        const int st = j % kKvStages;
+        if (j >= kKvStages && !mbar_wait(&kv_empty[st], ((j / kKvStages) & 1) ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
           break;
@@ -133,7 +143,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       if (!ok) {
         mbar_wait(q_full, 0);
-        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) mbar_wait(&kv_full[j & 1], (j >> 1) & 1);
+        for (int j = (issued > kKvStages ? issued - kKvStages : 0); j < issued; ++j)
+          mbar_wait(&kv_full[j % kKvStages], (j / kKvStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -142,27 +153,35 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       constexpr uint32_t idO = idesc_f16_f32(128, 80);
       const uint32_t sQ = smem_u32(smem + AttnSmem::Q);
       auto issue_s = [&](int j) {
-        const uint32_t sK = smem_u32(smem + AttnSmem::K0 + (j & 1) * 16384);
-        const uint32_t tS = tmem + (j & 1) * 128;
+        const int b = j % kKvStages;
+        const uint32_t sK = smem_u32(smem + AttnSmem::K0 + b * 16384);
+        const uint32_t tS = tmem + b * 128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) umma_f16(tS, desc_sw128(sQ + kk * 32), desc_sw128(sK + kk * 32), idS, kk);
-        umma_commit(&s_full[j & 1]);
+        umma_commit(&s_full[b]);
       };
       bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
+        if (nkv > 1) {
+          ok = mbar_wait(&kv_full[1], 0);
+          if (ok) {
+            tc_fence_after();
+            issue_s(1);
+          }
+        }
       }
       for (int j = 0; ok && j < nkv; ++j) {
-        // S_{j+1} reuses the score buffer of S_{j-1}, whose softmax finished
+        // S_{j+2} reuses the score buffer of S_{j-1}, whose softmax finished
         // reading it before P_{j-1} was published.
-        if (j + 1 < nkv) {
-          if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) {
+        if (j + 2 < nkv) {
+          if (!mbar_wait(&kv_full[(j + 2) % kKvStages], ((j + 2) / kKvStages) & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_s(j + 1);
+          issue_s(j + 2);
         }
         if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) {
           ok = false;
@@ -170,7 +189,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         tc_fence_after();
         const uint32_t sP = smem_u32(smem + AttnSmem::P + (j & 1) * 32768);
-        const uint32_t sV = smem_u32(smem + AttnSmem::V0 + (j & 1) * 2 * AttnSmem::kVHalf);
+        const uint32_t sV = smem_u32(smem + AttnSmem::V0 + (j % kKvStages) * 2 * AttnSmem::kVHalf);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t a = sP + (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -178,7 +197,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           umma_f16(tO, desc_sw128(a), desc_sw128(bv), idO, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[j & 1]);
-        umma_commit(&kv_empty[j & 1]);
+        umma_commit(&kv_empty[j % kKvStages]);
       }
       if (!ok) atomicOr(err, kErrWaitMma);
     }
@@ -197,13 +216,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // after a failed wait (the work is skipped), so no thread is left waiting
     // on a barrier that another warp of its quarter will never reach.
     for (int j = 0; j < nkv; ++j) {
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j % kKvStages], (j / kKvStages) & 1));
       float s[kSCols];
       const int nvalid = min(128, T - j * 128) - sub * kSCols;  // valid columns of this warp
       float mx = -INFINITY;
       if (ok) {
         tc_fence_after();
-        tmem_ld32(tmem + (j & 1) * 128 + sub * kSCols + lane_base, s);
+        tmem_ld32(tmem + (j % kKvStages) * 128 + sub * kSCols + lane_base, s);
         if (nvalid < kSCols) {
 #pragma unroll
           for (int i = 0; i < kSCols; ++i)
@@ -252,8 +271,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       uint32_t pk[kSCols / 2];
       const float nb = -m_ref;
+      // The first kPolyPairs pairs on the FMA/ALU pipes, the rest on the
+      // exponent unit (16 results per clock per SM), so both pipes share the load.
 #pragma unroll
-      for (int i = 0; i < kSCols; i += 2) pk[i / 2] = exp2_affine_f16x2(s[i], s[i + 1], c, nb);
+      for (int i = 0; i < kSCols; i += 2)
+        pk[i / 2] = (i / 2 < kPolyPairs) ? exp2_affine_poly_f16x2(s[i], s[i + 1], c, nb)
+                                         : exp2_affine_f16x2(s[i], s[i + 1], c, nb);
       // P buffer j & 1 was last read by P_{j-2} V_{j-2}.
       if (j >= 2 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1));
       uint8_t* prow = smem + prow_off + (j & 1) * 32768;

@@ -1,18 +1,22 @@
 // Conv layer 0 of the feature encoder on the tensor core: Conv1d(1 -> 512,
 // kernel 10, stride 5) is a GEMM with K = 10 taps (zero-padded to the MMA's
-// K = 16): A[t, j] = pcm[5 t + j], B[c, j] = w0[c, j].  One CTA per 128 output
-// frames of one clip computes all 512 channels with two tcgen05 MMAs
-// (M = 128, N = 256, K = 16) into 512 TMEM columns; the epilogue applies the
-// norm and GELU and stores through TMA:
+// K = 16): A[t, j] = pcm[5 t + j], B[c, j] = w0[c, j].  A tile is 128 output
+// frames of one clip x all 512 channels: two tcgen05 MMAs (M = 128, N = 256,
+// K = 16) into 512 TMEM columns; the epilogue applies the norm and GELU and
+// stores through TMA:
 //   group layout: GroupNorm with per-channel statistics over every frame of
 //     the clip (the TensorRT wav2vec2 README's "group norm over every time
 //     step"), precomputed as scale/shift by the moments kernel;
 //   layer layout: conv bias, then LayerNorm over the 512 channels of each
 //     frame (the four warps that share a row combine their partial sums).
-// 576 threads: warp 0 stages the operands and issues the MMAs, warp 1 owns
-// TMEM, warps 2-17 run the epilogue (four warps per TMEM lane quarter, one per
-// 128-channel slice).  The PCM is rounded to fp16 for the MMA, the same
-// rounding every inter-layer activation of this path gets.
+// Persistent: one CTA per SM walks the tiles (stride gridDim.x), so the
+// weights, TMEM and barriers are set up once; warp 0 builds the next tile's
+// window matrix while the epilogue of the current one runs (two A buffers),
+// and issues its MMAs as soon as the epilogue has read the accumulator.
+// 576 threads: warp 0 stages A and issues the MMAs, warp 1 owns TMEM, warps
+// 2-17 run the epilogue (four warps per TMEM lane quarter, one per 128-channel
+// slice).  The PCM is rounded to fp16 for the MMA, the same rounding every
+// inter-layer activation of this path gets.
 #include "ptx.cuh"
 #include "w2v_internal.h"
 
@@ -22,8 +26,8 @@ namespace {
 constexpr int kC0 = 512;
 constexpr int kTaps = 10;
 constexpr int kHop = 5;
-constexpr int A_OFF = 0;                   // [2 k-chunks][128 rows][8] fp16, 4 KB
-constexpr int B_OFF = 4096;                // [2 k-chunks][512 rows][8] fp16, 16 KB
+constexpr int A_OFF = 0;                   // [2 buffers][2 k-chunks][128 rows][8] fp16, 2 x 4 KB
+constexpr int B_OFF = 8192;                // [2 k-chunks][512 rows][8] fp16, 16 KB
 constexpr int PA_OFF = B_OFF + 16384;      // float[512]: GroupNorm scale, or LayerNorm gamma
 constexpr int PB_OFF = PA_OFF + 2048;      // float[512]: GroupNorm shift, or LayerNorm beta
 constexpr int BIAS_OFF = PB_OFF + 2048;    // float bias[512]
@@ -34,13 +38,15 @@ constexpr int STG_OFF = RED_OFF + 2048;    // staging: 16 warps x 4 boxes x 2 KB
 constexpr int BAR_OFF = STG_OFF + kEpiWarps * (kCols / 32) * 2048;
 constexpr int SMEM = BAR_OFF + 64 + 1024;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
 }  // namespace
 
 template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
-conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int n, int t0,
-                const __half* __restrict__ wpack, const float* __restrict__ b0, const float* __restrict__ gamma,
-                const float* __restrict__ beta, const float2* scale_shift, int layer_norm, float eps, int* err) {
+conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int n, int t0, int tiles_per_clip,
+                int ntiles, const __half* __restrict__ wpack, const float* __restrict__ b0,
+                const float* __restrict__ gamma, const float* __restrict__ beta, const float2* scale_shift,
+                int layer_norm, float eps, int* err) {
   // pcm and scale_shift may be written by the previous kernel (programmatic
   // dependent launch): plain coherent loads after pdl_wait() only.
   extern __shared__ uint8_t smem_raw[];
@@ -50,16 +56,19 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
   float* bias = reinterpret_cast<float*>(smem + BIAS_OFF);
   float* red = reinterpret_cast<float*>(smem + RED_OFF);
   uint64_t* w_full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* accf = w_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* accf = w_full + 1;         // MMA of a tile done (one completion per tile)
+  uint64_t* tmem_empty = w_full + 2;   // epilogue has read the accumulator (16 warp arrivals)
+  uint64_t* a_free = w_full + 3;       // [2] MMA done reading A buffer b
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(w_full + 5);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f0 = blockIdx.x * 128;
-  const int b = blockIdx.z;
 
   if (threadIdx.x == 0) {
     mbar_init(w_full, 1);
     mbar_init(accf, 1);
+    mbar_init(tmem_empty, kEpiWarps);
+    mbar_init(&a_free[0], 1);
+    mbar_init(&a_free[1], 1);
     fence_mbar_init();
     pdl_launch_dependents();
     // The packed weights do not depend on the previous kernel.
@@ -77,153 +86,192 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
       bias[c] = b0 ? b0[c] : 0.f;
     }
   }
-  pdl_wait();
-  if (!layer_norm)
-    for (int c = threadIdx.x; c < kC0; c += kThreads) {
-      const float2 ss = scale_shift[b * kC0 + c];
-      pa[c] = ss.x;
-      pb[c] = ss.y;
-    }
-  // A tile: row t holds pcm[5 (f0 + t) + j], j < 10, then zeros; 16-byte
-  // chunk (row, k-chunk) at k-chunk * 2048 + row * 16 (no-swizzle core matrices).
-  if (threadIdx.x < 256) {
-    const int row = threadIdx.x >> 1, kc = threadIdx.x & 1;
-    const int t = f0 + row;
-    const float* x = pcm + static_cast<int64_t>(b) * n + static_cast<int64_t>(kHop) * t;
-    uint32_t hv[4];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const int j = kc * 8 + e;
-      const float v0 = (t < t0 && j < kTaps) ? x[j] : 0.f;
-      const float v1 = (t < t0 && j + 1 < kTaps) ? x[j + 1] : 0.f;
-      __half2 h = __floats2half2_rn(v0, v1);
-      hv[e / 2] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    *reinterpret_cast<uint4*>(smem + A_OFF + kc * 2048 + row * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
 
   if (warp == 0) {
-    if (lane == 0) {
-      if (mbar_wait(w_full, 0)) {
-        tc_fence_after();
-        constexpr uint32_t idesc = idesc_f16_f32(128, 256);
-        const uint32_t sa = smem_u32(smem + A_OFF);
-        const uint32_t sb = smem_u32(smem + B_OFF);
+    // ------------------------------------------------ A builder + MMA issuer
+    bool ok = true;
+    int i = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int b = tile / tiles_per_clip;
+      const int f0 = (tile - b * tiles_per_clip) * 128;
+      // A buffer i & 1 was last read by the MMA of tile i - 2.
+      if (i >= 2 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&a_free[i & 1], ((i >> 1) - 1) & 1));
+      // row t of A holds pcm[5 (f0 + t) + j], j < 10, then zeros; 16-byte chunk
+      // (row, k-chunk) at k-chunk * 2048 + row * 16 (no-swizzle core matrices)
+      uint8_t* abuf = smem + A_OFF + (i & 1) * 4096;
+      const float* x = pcm + static_cast<int64_t>(b) * n;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          umma_f16(tmem + h * 256, smem_desc(sa, 2048, 128, kSwizzleNone), smem_desc(sb + h * 256 * 16, 8192, 128,
-                   kSwizzleNone), idesc, 0u);
-        umma_commit(accf);
-      } else {
-        atomicOr(err, kErrWaitMma);
+      for (int u = 0; u < 8; ++u) {
+        const int idx = u * 32 + lane;
+        const int row = idx >> 1, kc = idx & 1;
+        const int t = f0 + row;
+        const float* xr = x + static_cast<int64_t>(kHop) * t;
+        uint32_t hv[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; e2 += 2) {
+          const int j = kc * 8 + e2;
+          const float v0 = (t < t0 && j < kTaps) ? xr[j] : 0.f;
+          const float v1 = (t < t0 && j + 1 < kTaps) ? xr[j + 1] : 0.f;
+          __half2 h = __floats2half2_rn(v0, v1);
+          hv[e2 / 2] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(abuf + kc * 2048 + row * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        // the accumulator is free once the epilogue of tile i - 1 has read it
+        if (ok && i == 0) ok = mbar_wait(w_full, 0);
+        if (ok && i >= 1) ok = mbar_wait(tmem_empty, (i - 1) & 1);
+        if (ok) {
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_f16_f32(128, 256);
+          const uint32_t sa = smem_u32(abuf);
+          const uint32_t sb = smem_u32(smem + B_OFF);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            umma_f16(tmem + h * 256, smem_desc(sa, 2048, 128, kSwizzleNone),
+                     smem_desc(sb + h * 256 * 16, 8192, 128, kSwizzleNone), idesc, 0u);
+          umma_commit(accf);
+          umma_commit(&a_free[i & 1]);
+        } else {
+          atomicOr(err, kErrWaitMma);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
     }
   } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
     const int q = warp & 3;              // TMEM lane quarter
     const int sl = (warp - 2) >> 2;      // channel slice [kCols sl, kCols sl + kCols)
     const int r = q * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16) + sl * kCols;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
-    if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
-    tc_fence_after();
-    // Per element: pre-activation a = v * A + B with per-channel (A, B) pairs:
-    // GroupNorm (scale, shift), or for LayerNorm A = rstd gamma and
-    // B = (bias - mean) rstd gamma + beta, folded per 4-channel group below.
-    float mean = 0.f, rstd = 1.f;
-    if (layer_norm) {
-      // Per-frame LayerNorm statistics over all 512 channels (two passes; the
-      // four slices of a row meet in shared memory).
-      float s1 = 0.f;
-      if (ok) {
-#pragma unroll 1
-        for (int c = 0; c < kCols; c += 32) {
-          float v[32];
-          tmem_ld32(trow + c, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s1 += v[i] + bias[sl * kCols + c + i];
-        }
-      }
-      red[sl * 128 + r] = s1;
-      named_barrier_sync(1, 32 * kEpiWarps);
-      mean = ((red[r] + red[128 + r]) + (red[256 + r] + red[384 + r])) * (1.0f / kC0);
-      named_barrier_sync(1, 32 * kEpiWarps);
-      float s2 = 0.f;
-      if (ok) {
-#pragma unroll 1
-        for (int c = 0; c < kCols; c += 32) {
-          float v[32];
-          tmem_ld32(trow + c, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float d = v[i] + bias[sl * kCols + c + i] - mean;
-            s2 += d * d;
-          }
-        }
-      }
-      red[sl * 128 + r] = s2;
-      named_barrier_sync(1, 32 * kEpiWarps);
-      rstd = rsqrtf(((red[r] + red[128 + r]) + (red[256 + r] + red[384 + r])) * (1.0f / kC0) + eps);
-    }
     uint8_t* stage = smem + STG_OFF + (warp - 2) * (kCols / 32) * 2048;
-#pragma unroll 1
-    for (int cb = 0; cb < kCols / 32; ++cb) {
-      const int c = cb * 32;
-      const int ch = sl * kCols + c;
-      uint32_t hv[16];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float v[16];
-        if (ok) tmem_ld16(trow + c + hh * 16, v);
-#pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-          const int cc = ch + hh * 16 + i;
-          // Warp-uniform addresses: broadcast loads of 4 channels' parameters.
-          const float4 A4 = *reinterpret_cast<const float4*>(pa + cc);
-          const float4 B4 = *reinterpret_cast<const float4*>(pb + cc);
-          float2 a01, a23;
-          if (layer_norm) {
-            const float4 c4 = *reinterpret_cast<const float4*>(bias + cc);
-            // ((v + bias) - mean) * rstd * gamma + beta
-            const float2 m2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
-            a01 = fmul2(fadd2(fadd2(make_float2(v[i], v[i + 1]), make_float2(c4.x, c4.y)), m2), r2);
-            a23 = fmul2(fadd2(fadd2(make_float2(v[i + 2], v[i + 3]), make_float2(c4.z, c4.w)), m2), r2);
-            a01 = ffma2(a01, make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
-            a23 = ffma2(a23, make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
-          } else {
-            a01 = ffma2(make_float2(v[i], v[i + 1]), make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
-            a23 = ffma2(make_float2(v[i + 2], v[i + 3]), make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
-          }
-          if (ACT == 2) {
-            a01 = gelu_tanh2(a01);
-            a23 = gelu_tanh2(a23);
-          } else if (ACT == 1) {
-            a01 = make_float2(gelu_erf(a01.x), gelu_erf(a01.y));
-            a23 = make_float2(gelu_erf(a23.x), gelu_erf(a23.y));
-          }
-          __half2 h01 = __floats2half2_rn(a01.x, a01.y), h23 = __floats2half2_rn(a23.x, a23.y);
-          hv[hh * 8 + i / 2] = *reinterpret_cast<uint32_t*>(&h01);
-          hv[hh * 8 + i / 2 + 1] = *reinterpret_cast<uint32_t*>(&h23);
+    bool ok = true;
+    int cur_b = -1;
+    int i = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int b = tile / tiles_per_clip;
+      const int f0 = (tile - b * tiles_per_clip) * 128;
+      if (!layer_norm && b != cur_b) {
+        // GroupNorm scale/shift of this clip (every epilogue warp walks the
+        // same tiles, so all of them take this branch together)
+        named_barrier_sync(2, kEpiThreads);
+        for (int c = threadIdx.x - 64; c < kC0; c += kEpiThreads) {
+          const float2 ss = scale_shift[b * kC0 + c];
+          pa[c] = ss.x;
+          pb[c] = ss.y;
         }
+        named_barrier_sync(2, kEpiThreads);
+        cur_b = b;
       }
-      // 32 rows x 32 channels box, 64-byte rows, 64-byte swizzle.
-      uint8_t* box = stage + cb * 2048;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(accf, i & 1));
+      if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+      tc_fence_after();
+      float mean = 0.f, rstd = 1.f;
+      if (layer_norm) {
+        // Per-frame LayerNorm statistics over all 512 channels (two passes; the
+        // four slices of a row meet in shared memory).
+        float s1 = 0.f;
+        if (ok) {
+#pragma unroll 1
+          for (int c = 0; c < kCols; c += 32) {
+            float v[32];
+            tmem_ld32(trow + c, v);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
-            make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
-      fence_proxy_async_smem();
+            for (int k = 0; k < 32; ++k) s1 += v[k] + bias[sl * kCols + c + k];
+          }
+        }
+        red[sl * 128 + r] = s1;
+        named_barrier_sync(1, kEpiThreads);
+        mean = ((red[r] + red[128 + r]) + (red[256 + r] + red[384 + r])) * (1.0f / kC0);
+        named_barrier_sync(1, kEpiThreads);
+        float s2 = 0.f;
+        if (ok) {
+#pragma unroll 1
+          for (int c = 0; c < kCols; c += 32) {
+            float v[32];
+            tmem_ld32(trow + c, v);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float d = v[k] + bias[sl * kCols + c + k] - mean;
+              s2 += d * d;
+            }
+          }
+        }
+        red[sl * 128 + r] = s2;
+        named_barrier_sync(1, kEpiThreads);
+        rstd = rsqrtf(((red[r] + red[128 + r]) + (red[256 + r] + red[384 + r])) * (1.0f / kC0) + eps);
+        named_barrier_sync(1, kEpiThreads);  // red is rewritten by the next tile
+      }
+      // this warp's staging boxes: the previous tile's stores have read them
+      if (lane == 0) bulk_wait_read_all();
       __syncwarp();
-      if (lane == 0 && ok) tma_store_3d(&tmOut, box, ch, f0 + q * 32, b);
+#pragma unroll 1
+      for (int cb = 0; cb < kCols / 32; ++cb) {
+        const int c = cb * 32;
+        const int ch = sl * kCols + c;
+        uint32_t hv[16];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[16];
+          if (ok) tmem_ld16(trow + c + hh * 16, v);
+#pragma unroll
+          for (int k = 0; k < 16; k += 4) {
+            const int cc = ch + hh * 16 + k;
+            // Warp-uniform addresses: broadcast loads of 4 channels' parameters.
+            const float4 A4 = *reinterpret_cast<const float4*>(pa + cc);
+            const float4 B4 = *reinterpret_cast<const float4*>(pb + cc);
+            float2 a01, a23;
+            if (layer_norm) {
+              const float4 c4 = *reinterpret_cast<const float4*>(bias + cc);
+              // ((v + bias) - mean) * rstd * gamma + beta
+              const float2 m2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
+              a01 = fmul2(fadd2(fadd2(make_float2(v[k], v[k + 1]), make_float2(c4.x, c4.y)), m2), r2);
+              a23 = fmul2(fadd2(fadd2(make_float2(v[k + 2], v[k + 3]), make_float2(c4.z, c4.w)), m2), r2);
+              a01 = ffma2(a01, make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
+              a23 = ffma2(a23, make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
+            } else {
+              a01 = ffma2(make_float2(v[k], v[k + 1]), make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
+              a23 = ffma2(make_float2(v[k + 2], v[k + 3]), make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
+            }
+            if (ACT == 2) {
+              a01 = gelu_tanh2(a01);
+              a23 = gelu_tanh2(a23);
+            } else if (ACT == 1) {
+              a01 = make_float2(gelu_erf(a01.x), gelu_erf(a01.y));
+              a23 = make_float2(gelu_erf(a23.x), gelu_erf(a23.y));
+            }
+            __half2 h01 = __floats2half2_rn(a01.x, a01.y), h23 = __floats2half2_rn(a23.x, a23.y);
+            hv[hh * 8 + k / 2] = *reinterpret_cast<uint32_t*>(&h01);
+            hv[hh * 8 + k / 2 + 1] = *reinterpret_cast<uint32_t*>(&h23);
+          }
+        }
+        if (cb == kCols / 32 - 1) {
+          // last accumulator read of this tile: hand TMEM to the next MMA
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tmem_empty);
+        }
+        // 32 rows x 32 channels box, 64-byte rows, 64-byte swizzle.
+        uint8_t* box = stage + cb * 2048;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && ok) tma_store_3d(&tmOut, box, ch, f0 + q * 32, b);
+      }
+      if (lane == 0) bulk_commit_group();
     }
-    if (lane == 0) {
-      bulk_commit_group();
-      bulk_wait_all();
-    }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -250,10 +298,12 @@ cudaError_t launch_conv0_tc(const float* pcm, int n, int batch, int t0, int clip
   const uint32_t box[3] = {32, 32, 1};
   cudaError_t r = make_tmap(&tm, out, 3, dims, str, box, 2, 64);
   if (r != cudaSuccess) return r;
-  dim3 grid((t0 + 127) / 128, 1, batch);
+  const int tiles_per_clip = (t0 + 127) / 128;
+  const int ntiles = tiles_per_clip * batch;
+  const int grid = ntiles < kNumSMs ? ntiles : kNumSMs;
   auto k = act == 2 ? conv0_tc_kernel<2> : (act == 1 ? conv0_tc_kernel<1> : conv0_tc_kernel<0>);
-  return launch_pdl(k, grid, dim3(kThreads), SMEM, st, tm, pcm, n, t0, wpack, b0, gamma, beta, scale_shift,
-                    layer_norm, eps, err);
+  return launch_pdl(k, dim3(grid), dim3(kThreads), SMEM, st, tm, pcm, n, t0, tiles_per_clip, ntiles, wpack, b0, gamma,
+                    beta, scale_shift, layer_norm, eps, err);
 }
 
 }  // namespace w2v

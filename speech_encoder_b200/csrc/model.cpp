@@ -4,6 +4,7 @@
 // shape as a CUDA graph.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -463,7 +464,9 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   return W2V_OK;
 }
 
-int get_plan(w2v_model* m, int n, int batch, const Plan** out) {
+int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits);
+
+int get_plan(w2v_model* m, int n, int batch, const Plan** out, const float* pcm, float* logits) {
   auto key = std::make_pair(n, batch);
   auto it = m->plans.find(key);
   if (it != m->plans.end()) {
@@ -472,6 +475,7 @@ int get_plan(w2v_model* m, int n, int batch, const Plan** out) {
   }
   std::unique_ptr<Plan> p(new Plan());
   int rc = build_plan(m, n, batch, p.get());
+  if (rc == W2V_OK) rc = refine_plan(m, p.get(), pcm, logits);
   if (rc != W2V_OK) return rc;
   *out = p.get();
   m->plans[key] = std::move(p);
@@ -880,6 +884,103 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   return W2V_OK;
 }
 
+// The per-layer GEMMs (QKV, out-projection, FFN1, FFN2) are re-chosen on the
+// whole forward: tiles timed on their own are only a starting point, since a
+// GEMM launched back to back with itself behaves differently from one inside
+// the forward's chain.  For each role in turn every candidate (tile width and
+// split-K factor) replaces the current one, the forward is captured as a CUDA
+// graph and timed (best of 3 replays), and the fastest is kept (coordinate
+// descent; the incumbent wins ties within 0.5 %).
+namespace {
+int apply_role(w2v_model* m, Plan* p, int role, int bn, int splits) {
+  const int d = m->cfg.d_model, F = m->cfg.d_ffn;
+  std::vector<CUtensorMap>* maps[4] = {&p->qkvB, &p->oB, &p->f1B, &p->f2B};
+  int* bns[4] = {&p->qkvBN, &p->oBN, &p->f1BN, &p->f2BN};
+  GemmShape* shapes[4] = {&p->qkvS, &p->oS, &p->f1S, &p->f2S};
+  *bns[role] = bn;
+  shapes[role]->splits = splits;
+  for (int l = 0; l < m->cfg.n_layers; ++l) {
+    const LayerDev& w = m->L[l];
+    const __half* W = role == 0 ? w.wqkv : role == 1 ? w.wo : role == 2 ? w.w1 : w.w2;
+    const int N = role == 0 ? 3 * d : role == 2 ? F : d;
+    const int K = role == 3 ? F : d;
+    CUDA_OR(m, map_matrix(&(*maps[role])[l], W, N, K, bn));
+  }
+  return W2V_OK;
+}
+
+float time_forward_us(w2v_model* m, const Plan& p, const float* pcm, float* logits) {
+  cudaStream_t st = m->cap_stream;
+  cudaGraph_t g = nullptr;
+  cudaGraphExec_t ge = nullptr;
+  if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return 1e30f;
+  const int rc = enqueue_forward(m, p, pcm, logits, st, nullptr);
+  const cudaError_t ec = cudaStreamEndCapture(st, &g);
+  if (rc != W2V_OK || ec != cudaSuccess || cudaGraphInstantiate(&ge, g, 0) != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return 1e30f;
+  }
+  cudaGraphDestroy(g);
+  float best = 1e30f;
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) == cudaSuccess && cudaEventCreate(&e1) == cudaSuccess) {
+    cudaGraphLaunch(ge, st);
+    for (int i = 0; i < 3; ++i) {
+      cudaEventRecord(e0, st);
+      cudaGraphLaunch(ge, st);
+      cudaEventRecord(e1, st);
+      float ms = 0.f;
+      if (cudaEventSynchronize(e1) == cudaSuccess && cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess)
+        best = std::min(best, ms * 1000.f);
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+  }
+  cudaGraphExecDestroy(ge);
+  cudaGetLastError();
+  return best;
+}
+
+int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
+  const char* env = std::getenv("W2V_AUTOTUNE");
+  if ((env && env[0] == '0') || m->cfg.n_layers == 0 || !pcm || !logits) return W2V_OK;
+  const int d = m->cfg.d_model, F = m->cfg.d_ffn;
+  const bool log = std::getenv("W2V_TUNE_LOG") != nullptr;
+  float best = time_forward_us(m, *p, pcm, logits);
+  if (log) std::fprintf(stderr, "w2v tune: forward %.1f us with the per-GEMM choices\n", best);
+  const char* names[4] = {"QKV", "out-proj", "FFN1", "FFN2"};
+  for (int role = 0; role < 4; ++role) {
+    const int N = role == 0 ? 3 * d : role == 2 ? F : d;
+    const int K = role == 3 ? F : d;
+    const int nk = K / 64;
+    GemmShape* sh = role == 0 ? &p->qkvS : role == 1 ? &p->oS : role == 2 ? &p->f1S : &p->f2S;
+    int cur_bn = role == 0 ? p->qkvBN : role == 1 ? p->oBN : role == 2 ? p->f1BN : p->f2BN;
+    int cur_s = sh->splits;
+    for (int bn : {32, 64, 128, 192, 256}) {
+      if (bn == 32 ? N > 32 : N <= bn / 2) continue;
+      if (role == 0 && d % bn != 0) continue;
+      for (int sp : {1, 2, 3, 4, 6}) {
+        if (sp > 1 && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
+        if (bn == cur_bn && sp == cur_s) continue;
+        int rc = apply_role(m, p, role, bn, sp);
+        if (rc != W2V_OK) return rc;
+        const float t = time_forward_us(m, *p, pcm, logits);
+        if (t < best * 0.995f) {
+          best = t;
+          cur_bn = bn;
+          cur_s = sp;
+        }
+      }
+    }
+    int rc = apply_role(m, p, role, cur_bn, cur_s);
+    if (rc != W2V_OK) return rc;
+    if (log) std::fprintf(stderr, "w2v tune: %s -> bn=%d splits=%d, forward %.1f us\n", names[role], cur_bn, cur_s, best);
+  }
+  return W2V_OK;
+}
+}  // namespace
+
 extern "C" int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev,
                            void* stream) {
   if (!m) return W2V_EINVAL;
@@ -893,7 +994,7 @@ extern "C" int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, in
   if (cudaSetDevice(m->device) != cudaSuccess) return fail(m, W2V_ECUDA, "cudaSetDevice failed");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Plan* p = nullptr;
-  int rc = get_plan(m, n_samples, batch, &p);
+  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev);
   if (rc != W2V_OK) return rc;
   m->last_plan = p;
   if (!m->cfg.use_cuda_graph) {
@@ -1014,7 +1115,7 @@ extern "C" int w2v_profile_forward(w2v_model* m, const float* pcm_dev, int n_sam
   CUDA_OR(m, cudaSetDevice(m->device));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Plan* p = nullptr;
-  int rc = get_plan(m, n_samples, batch, &p);
+  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev);
   if (rc != W2V_OK) return rc;
   m->last_plan = p;
   Prof prof;
@@ -1057,7 +1158,7 @@ extern "C" int w2v_time_class(w2v_model* m, const float* pcm_dev, int n_samples,
   CUDA_OR(m, cudaSetDevice(m->device));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Plan* p = nullptr;
-  int rc = get_plan(m, n_samples, batch, &p);
+  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev);
   if (rc != W2V_OK) return rc;
   // Record `reps` passes of only this class's launches as one graph.
   Prof filt;

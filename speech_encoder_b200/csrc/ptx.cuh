@@ -120,6 +120,12 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // Waits until every bulk store this thread committed has been performed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Waits until every committed bulk store of this thread has finished reading
+// its shared-memory source (the writes to global memory may still be in flight).
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Plain (untiled) bulk copy global -> shared.  Both addresses 16-byte aligned,
 // size a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -331,6 +337,38 @@ __device__ __forceinline__ uint32_t exp2_affine_f16x2(float s0, float s1, float 
       "cvt.rn.f16x2.f32 h, x1, x0;\n\tex2.approx.f16x2 %0, h;\n\t}"
       : "=r"(out)
       : "f"(s0), "f"(s1), "f"(c), "f"(b));
+  return out;
+}
+
+// The same pair on the FMA and ALU pipes instead of the exponent unit
+// (softmax offloads part of its exponentials here): x = s c + b rounded to
+// fp16 and clamped to [-15, 8] (the caller keeps x <= 8), split as x = j + f
+// with j = round(x) (adding 1536 leaves j in the low mantissa bits) and
+// |f| <= 1/2; 2^f by a cubic whose coefficients were fitted to 2^f on
+// [-1/2, 1/2] by iteratively reweighted least squares (relative error 1.5e-4
+// with the coefficients in fp16, 7e-4 with fp16 Horner steps); 2^j as the
+// fp16 whose biased exponent field is j + 15 (j = -15 gives +0, so values
+// below 2^-15 flush to zero).
+__device__ __forceinline__ uint32_t exp2_affine_poly_f16x2(float s0, float s1, float c, float b) {
+  uint32_t out;
+  asm("{\n\t.reg .b64 sv, cv, bv, xv;\n\t.reg .f32 x0, x1;\n\t.reg .b32 h, t, r, f, p, e;\n\t"
+      "mov.b64 sv, {%1, %2};\n\tmov.b64 cv, {%3, %3};\n\tmov.b64 bv, {%4, %4};\n\t"
+      "fma.rn.f32x2 xv, sv, cv, bv;\n\tmov.b64 {x0, x1}, xv;\n\t"
+      "cvt.rn.f16x2.f32 h, x1, x0;\n\t"
+      "max.f16x2 h, h, %5;\n\t"
+      "add.rn.f16x2 t, h, %6;\n\t"
+      "sub.rn.f16x2 r, t, %6;\n\t"
+      "sub.rn.f16x2 f, h, r;\n\t"
+      "fma.rn.f16x2 p, f, %7, %8;\n\t"
+      "fma.rn.f16x2 p, p, f, %9;\n\t"
+      "fma.rn.f16x2 p, p, f, %10;\n\t"
+      "sub.u32 e, t, %11;\n\t"
+      "shl.b32 e, e, 10;\n\t"
+      "mul.rn.f16x2 %0, p, e;\n\t}"
+      : "=r"(out)
+      : "f"(s0), "f"(s1), "f"(c), "f"(b), "r"(0xCB80CB80u) /* -15 */, "r"(0x66006600u) /* 1536 */,
+        "r"(0x2B102B10u) /* 0.0551758 */, "r"(0x33C333C3u) /* 0.2425537 */, "r"(0x398C398Cu) /* 0.6933594 */,
+        "r"(0x3C003C00u) /* 1 */, "r"(0x65F165F1u) /* bits of 1536 - 15 */);
   return out;
 }
 

@@ -66,6 +66,9 @@ struct GemmEpilogue {
   int t_len = 0;                   // frames per clip (rows are clip-major)
 };
 
+// Streaming multiprocessors of a B200: the grid of the persistent kernels.
+constexpr int kNumSMs = 148;
+
 struct GemmShape {
   int M = 0;        // valid rows per batch item
   int N = 0;        // valid output columns
