@@ -151,13 +151,18 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16_f32(128, 128);
       constexpr uint32_t idO = idesc_f16_f32(128, 80);
-      const uint32_t sQ = smem_u32(smem + AttnSmem::Q);
+      // Descriptors built once; a buffer or K step only moves the 14-bit
+      // start-address field (16-byte units; addresses stay below 256 KB).
+      const uint64_t dQ = desc_sw128(smem_u32(smem + AttnSmem::Q));
+      const uint64_t dK0 = desc_sw128(smem_u32(smem + AttnSmem::K0));
+      const uint64_t dP0 = desc_sw128(smem_u32(smem + AttnSmem::P));
+      const uint64_t dV0 = desc_sw128(smem_u32(smem + AttnSmem::V0));
       auto issue_s = [&](int j) {
         const int b = j % kKvStages;
-        const uint32_t sK = smem_u32(smem + AttnSmem::K0 + b * 16384);
+        const uint64_t dK = dK0 + static_cast<uint64_t>(b * (16384 >> 4));
         const uint32_t tS = tmem + b * 128;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_f16(tS, desc_sw128(sQ + kk * 32), desc_sw128(sK + kk * 32), idS, kk);
+        for (int kk = 0; kk < 4; ++kk) umma_f16(tS, dQ + 2 * kk, dK + 2 * kk, idS, kk);
         umma_commit(&s_full[b]);
       };
       bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
@@ -188,13 +193,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t sP = smem_u32(smem + AttnSmem::P + (j & 1) * 32768);
-        const uint32_t sV = smem_u32(smem + AttnSmem::V0 + (j % kKvStages) * 2 * AttnSmem::kVHalf);
+        const uint64_t dP = dP0 + static_cast<uint64_t>((j & 1) * (32768 >> 4));
+        const uint64_t dV = dV0 + static_cast<uint64_t>((j % kKvStages) * (2 * AttnSmem::kVHalf >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a = sP + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t bv = sV + (kk >> 2) * AttnSmem::kVHalf + (kk & 3) * 32;
-          umma_f16(tO, desc_sw128(a), desc_sw128(bv), idO, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t a = dP + static_cast<uint64_t>((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
+          const uint64_t bv = dV + static_cast<uint64_t>((kk >> 2) * (AttnSmem::kVHalf >> 4) + (kk & 3) * 2);
+          umma_f16(tO, a, bv, idO, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[j & 1]);
         umma_commit(&kv_empty[j % kKvStages]);

@@ -202,21 +202,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, BN);
+      // The issuing thread's own instruction latency paces the MMAs, so the
+      // shared-memory descriptors are built once: stage st, K step kk is the
+      // stage-0 descriptor with (st * STAGE + kk * 32) / 16 added to its
+      // 14-bit start-address field (addresses stay below 256 KB: no carry).
+      const uint64_t dA0 = desc_sw128(smem_u32(smem));
+      const uint64_t dB0 = desc_sw128(smem_u32(smem) + C::A_BYTES);
       bool ok = true;
+      int st = 0;
+      uint32_t ph = 0;
       for (int i = 0; i < nkl; ++i) {
-        const int st = i % C::STAGES;
-        if (!mbar_wait(&full[st], (i / C::STAGES) & 1)) {
+        if (!mbar_wait(&full[st], ph)) {
           atomicOr(err, kErrWaitMma);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + st * C::STAGE);
-        const uint32_t sb = sa + C::A_BYTES;
+        const uint64_t off = static_cast<uint64_t>(st * (C::STAGE >> 4));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16(tmem, desc_sw128(sa + kk * 32), desc_sw128(sb + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
+          umma_f16(tmem, dA0 + off + 2 * kk, dB0 + off + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
         umma_commit(&empty[st]);
+        if (++st == C::STAGES) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
       if (ok) umma_commit(accf);
     }

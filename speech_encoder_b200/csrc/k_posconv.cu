@@ -112,7 +112,10 @@ posconv_kernel(const __grid_constant__ CUtensorMap tmX, const __half* x, const _
       constexpr uint32_t idesc = idesc_f16_f32(128, MG);
       bool ok = mbar_wait(a_full, 0);
       if (!ok) atomicOr(err, kErrWaitMma);
-      const uint32_t a0 = smem_u32(sA);
+      // Descriptors built once; a tap or stage step only moves the 14-bit
+      // start-address field (16-byte units; addresses stay below 256 KB).
+      const uint64_t dA0 = smem_desc(smem_u32(sA), kWin * 16, 128, kSwizzleNone);
+      const uint64_t dB0 = smem_desc(smem_u32(sB), MG * 16, 128, kSwizzleNone);
       for (int it = 0; ok && it < C::ITERS; ++it) {
         const int st = it % C::STAGES;
         if (!mbar_wait(&full[st], (it / C::STAGES) & 1)) {
@@ -121,16 +124,15 @@ posconv_kernel(const __grid_constant__ CUtensorMap tmX, const __half* x, const _
           break;
         }
         tc_fence_after();
-        const uint32_t b0 = smem_u32(sB + st * C::STAGE);
-#pragma unroll 1
+        const uint64_t bst = dB0 + static_cast<uint64_t>(st * (C::STAGE >> 4));
+#pragma unroll 4
         for (int tt = 0; tt < C::TAPS; ++tt) {
           const int j = it * C::TAPS + tt;
+          const uint64_t ad = dA0 + static_cast<uint64_t>(j);                        // window row j
+          const uint64_t bd = bst + static_cast<uint64_t>(tt * (C::TAP_BYTES >> 4));  // tap tt's block
 #pragma unroll
-          for (int kk = 0; kk < MG / 16; ++kk) {
-            const uint64_t ad = smem_desc(a0 + j * 16 + kk * 2 * (kWin * 16), kWin * 16, 128, kSwizzleNone);
-            const uint64_t bd = smem_desc(b0 + tt * C::TAP_BYTES + kk * 2 * (MG * 16), MG * 16, 128, kSwizzleNone);
-            umma_f16(tmem, ad, bd, idesc, (j | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < MG / 16; ++kk)
+            umma_f16(tmem, ad + kk * 2 * kWin, bd + kk * 2 * MG, idesc, (j | kk) != 0 ? 1u : 0u);
         }
         umma_commit(&empty[st]);
       }
