@@ -41,12 +41,13 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 }  // namespace
 
-template <int ACT>
+template <int ACT, bool LN>
 __global__ void __launch_bounds__(kThreads, 1)
 conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int n, int t0, int tiles_per_clip,
                 int ntiles, const __half* __restrict__ wpack, const float* __restrict__ b0,
                 const float* __restrict__ gamma, const float* __restrict__ beta, const float2* scale_shift,
-                int layer_norm, float eps, int* err) {
+                float eps, int* err) {
+  constexpr bool layer_norm = LN;
   // pcm and scale_shift may be written by the previous kernel (programmatic
   // dependent launch): plain coherent loads after pdl_wait() only.
   extern __shared__ uint8_t smem_raw[];
@@ -213,61 +214,95 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
       // this warp's staging boxes: the previous tile's stores have read them
       if (lane == 0) bulk_wait_read_all();
       __syncwarp();
-#pragma unroll 1
-      for (int cb = 0; cb < kCols / 32; ++cb) {
-        const int c = cb * 32;
-        const int ch = sl * kCols + c;
-        uint32_t hv[16];
+      // 8 chunks of 16 columns; the TMEM load of chunk k + 1 is in flight
+      // while chunk k is processed (two register buffers, alternating).
+      auto process = [&](uint32_t(&cur)[16], int k16) {
+        const int cb = k16 >> 1, hh = k16 & 1;
+        const int ch = sl * kCols + cb * 32;
+        uint32_t hv[8];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float v[16];
-          if (ok) tmem_ld16(trow + c + hh * 16, v);
-#pragma unroll
-          for (int k = 0; k < 16; k += 4) {
-            const int cc = ch + hh * 16 + k;
-            // Warp-uniform addresses: broadcast loads of 4 channels' parameters.
-            const float4 A4 = *reinterpret_cast<const float4*>(pa + cc);
-            const float4 B4 = *reinterpret_cast<const float4*>(pb + cc);
-            float2 a01, a23;
-            if (layer_norm) {
-              const float4 c4 = *reinterpret_cast<const float4*>(bias + cc);
-              // ((v + bias) - mean) * rstd * gamma + beta
-              const float2 m2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
-              a01 = fmul2(fadd2(fadd2(make_float2(v[k], v[k + 1]), make_float2(c4.x, c4.y)), m2), r2);
-              a23 = fmul2(fadd2(fadd2(make_float2(v[k + 2], v[k + 3]), make_float2(c4.z, c4.w)), m2), r2);
-              a01 = ffma2(a01, make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
-              a23 = ffma2(a23, make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
-            } else {
-              a01 = ffma2(make_float2(v[k], v[k + 1]), make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
-              a23 = ffma2(make_float2(v[k + 2], v[k + 3]), make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
-            }
-            if (ACT == 2) {
-              a01 = gelu_tanh2(a01);
-              a23 = gelu_tanh2(a23);
-            } else if (ACT == 1) {
-              a01 = make_float2(gelu_erf(a01.x), gelu_erf(a01.y));
-              a23 = make_float2(gelu_erf(a23.x), gelu_erf(a23.y));
-            }
-            __half2 h01 = __floats2half2_rn(a01.x, a01.y), h23 = __floats2half2_rn(a23.x, a23.y);
-            hv[hh * 8 + k / 2] = *reinterpret_cast<uint32_t*>(&h01);
-            hv[hh * 8 + k / 2 + 1] = *reinterpret_cast<uint32_t*>(&h23);
+        for (int k = 0; k < 16; k += 4) {
+          const int cc = ch + hh * 16 + k;
+          const float v0 = __uint_as_float(cur[k]), v1 = __uint_as_float(cur[k + 1]);
+          const float v2 = __uint_as_float(cur[k + 2]), v3 = __uint_as_float(cur[k + 3]);
+          // Warp-uniform addresses: broadcast loads of 4 channels' parameters.
+          const float4 A4 = *reinterpret_cast<const float4*>(pa + cc);
+          const float4 B4 = *reinterpret_cast<const float4*>(pb + cc);
+          float2 a01, a23;
+          if (layer_norm) {
+            const float4 c4 = *reinterpret_cast<const float4*>(bias + cc);
+            // ((v + bias) - mean) * rstd * gamma + beta
+            const float2 m2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
+            a01 = fmul2(fadd2(fadd2(make_float2(v0, v1), make_float2(c4.x, c4.y)), m2), r2);
+            a23 = fmul2(fadd2(fadd2(make_float2(v2, v3), make_float2(c4.z, c4.w)), m2), r2);
+            a01 = ffma2(a01, make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
+            a23 = ffma2(a23, make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
+          } else {
+            a01 = ffma2(make_float2(v0, v1), make_float2(A4.x, A4.y), make_float2(B4.x, B4.y));
+            a23 = ffma2(make_float2(v2, v3), make_float2(A4.z, A4.w), make_float2(B4.z, B4.w));
           }
+          if (ACT == 2) {
+            a01 = gelu_tanh2(a01);
+            a23 = gelu_tanh2(a23);
+          } else if (ACT == 1) {
+            a01 = make_float2(gelu_erf(a01.x), gelu_erf(a01.y));
+            a23 = make_float2(gelu_erf(a23.x), gelu_erf(a23.y));
+          }
+          __half2 h01 = __floats2half2_rn(a01.x, a01.y), h23 = __floats2half2_rn(a23.x, a23.y);
+          hv[k / 2] = *reinterpret_cast<uint32_t*>(&h01);
+          hv[k / 2 + 1] = *reinterpret_cast<uint32_t*>(&h23);
         }
-        if (cb == kCols / 32 - 1) {
-          // last accumulator read of this tile: hand TMEM to the next MMA
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tmem_empty);
-        }
-        // 32 rows x 32 channels box, 64-byte rows, 64-byte swizzle.
+        // 32 rows x 32 channels box, 64-byte rows, 64-byte swizzle: this half
+        // fills the row's 16-byte chunks 2 hh and 2 hh + 1.
         uint8_t* box = stage + cb * 2048;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+        for (int k = 0; k < 2; ++k)
+          *reinterpret_cast<uint4*>(box + lane * 64 + (((2 * hh + k) ^ ((lane >> 1) & 3)) << 4)) =
               make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && ok) tma_store_3d(&tmOut, box, ch, f0 + q * 32, b);
+        if (hh == 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && ok) tma_store_3d(&tmOut, box, ch, f0 + q * 32, b);
+        }
+      };
+      uint32_t b0[16], b1[16];
+      if (!(ACT == 1 && LN)) {
+        if (ok) tmem_ld16_issue(trow, b0);
+#pragma unroll 1
+        for (int k16 = 0; k16 < kCols / 16; k16 += 2) {
+          if (ok) {
+            tmem_wait16(b0);
+            tmem_ld16_issue(trow + (k16 + 1) * 16, b1);
+          }
+          process(b0, k16);
+          if (ok) {
+            tmem_wait16(b1);
+            if (k16 + 2 < kCols / 16) tmem_ld16_issue(trow + (k16 + 2) * 16, b0);
+          }
+          if (k16 + 2 == kCols / 16) {
+            // last accumulator read of this tile: hand TMEM to the next MMA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_empty);
+          }
+          process(b1, k16 + 1);
+        }
+      } else {
+        // The erf + LayerNorm variant has no registers to spare for a second
+        // buffer at this thread count: one load at a time.
+#pragma unroll 1
+        for (int k16 = 0; k16 < kCols / 16; ++k16) {
+          if (ok) {
+            tmem_ld16_issue(trow + k16 * 16, b0);
+            tmem_wait16(b0);
+          }
+          if (k16 + 1 == kCols / 16) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_empty);
+          }
+          process(b0, k16);
+        }
       }
       if (lane == 0) bulk_commit_group();
     }
@@ -281,10 +316,18 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
   }
 }
 
+template <int ACT, bool LN>
+static cudaError_t prepare_one() {
+  return cudaFuncSetAttribute(conv0_tc_kernel<ACT, LN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+}
+
 cudaError_t conv0_prepare() {
-  cudaError_t r = cudaFuncSetAttribute(conv0_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (r == cudaSuccess) r = cudaFuncSetAttribute(conv0_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (r == cudaSuccess) r = cudaFuncSetAttribute(conv0_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t r = prepare_one<0, false>();
+  if (r == cudaSuccess) r = prepare_one<1, false>();
+  if (r == cudaSuccess) r = prepare_one<2, false>();
+  if (r == cudaSuccess) r = prepare_one<0, true>();
+  if (r == cudaSuccess) r = prepare_one<1, true>();
+  if (r == cudaSuccess) r = prepare_one<2, true>();
   return r;
 }
 
@@ -301,9 +344,11 @@ cudaError_t launch_conv0_tc(const float* pcm, int n, int batch, int t0, int clip
   const int tiles_per_clip = (t0 + 127) / 128;
   const int ntiles = tiles_per_clip * batch;
   const int grid = ntiles < kNumSMs ? ntiles : kNumSMs;
-  auto k = act == 2 ? conv0_tc_kernel<2> : (act == 1 ? conv0_tc_kernel<1> : conv0_tc_kernel<0>);
+  auto k = layer_norm ? (act == 2 ? conv0_tc_kernel<2, true> : (act == 1 ? conv0_tc_kernel<1, true> : conv0_tc_kernel<0, true>))
+                      : (act == 2 ? conv0_tc_kernel<2, false>
+                                  : (act == 1 ? conv0_tc_kernel<1, false> : conv0_tc_kernel<0, false>));
   return launch_pdl(k, dim3(grid), dim3(kThreads), SMEM, st, tm, pcm, n, t0, tiles_per_clip, ntiles, wpack, b0, gamma,
-                    beta, scale_shift, layer_norm, eps, err);
+                    beta, scale_shift, eps, err);
 }
 
 }  // namespace w2v
