@@ -24,8 +24,11 @@ extern "C" {
  * the encoder blocks (README "Recipe" table: q/k/v/out projections,
  * intermediate_dense, output_dense) and of the CTC head.  bn = 0 picks the
  * tile width and split-K factor; otherwise bn (32/64/128/192/256) and splits
- * (1..8, <= K/64: the K blocks are divided among a cluster of `splits` CTAs
- * whose partial sums are reduced in distributed shared memory) are forced. */
+ * are forced: splits 1..8 (<= K/64) divides the K blocks among a cluster of
+ * `splits` CTAs whose partial sums are reduced in distributed shared memory;
+ * splits -2 or -4 (bn >= 64) reduces 2 or 4 splits through an fp32 scratch in
+ * L2 (TMA stores and loads; the call allocates and frees it on the stream),
+ * summed in split order.  Invalid combinations return W2V_EINVAL. */
 int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, const float* bias, const void* residual,
                 int res_f32, void* out, int out_f32, int act, int bn, int splits, int* err_dev, void* stream);
 

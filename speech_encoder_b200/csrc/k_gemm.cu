@@ -76,7 +76,7 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // (from shared memory), GELU, residual, store.  `vec` selects 16-/8-byte
 // accesses (row starts and pointers 16-byte aligned, full 4-vector in range).
 __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, int lcol, int grow, int col, int nv,
-                                        int bzb, const GemmEpilogue& e, void* outp, int ocol0, bool vec) {
+                                        int bzb, const GemmEpiArgs& e, void* outp, int ocol0, bool vec) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) x[i] = apply_act(x[i] + bias_s[lcol + i], e.act);
   if (e.residual) {
@@ -118,11 +118,13 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, int 
 }
 
 // mode: 0 generic, 1 direct (TMA store), 2 split-K
-template <int BN>
+// SPLIT: the instantiation for split-K launches (modes 2 and 3); the other one
+// runs modes 0 and 1 only.
+template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
-               const __grid_constant__ CUtensorMap tmV, GemmShape s, GemmEpilogue e, int vec_ok, int mode, int* err) {
+               const __grid_constant__ CUtensorMap tmV, GemmDims s, GemmEpiArgs e, int vec_ok, int mode, int* err) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,7 +132,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* peer_bar = accf + 1;  // [8] mode 3: one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_bar + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -150,6 +153,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(&empty[i], 1);
     }
     mbar_init(accf, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&peer_bar[i], 1);
     fence_mbar_init();
     pdl_launch_dependents();
     tma_prefetch_desc(&tmA);
@@ -298,10 +302,73 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     tc_fence_before();
     __syncthreads();
-  } else if (mode == 1) {
+  } else if (mode == 1 || (SPLIT && mode == 3)) {
     // ------------------------------------------------------------- direct
-    if (epi) {
-      named_barrier_sync(1, kEpiThreads);  // bias staged
+    // mode 3 = split-K through L2: the S = 2 or 4 CTAs of a tile (a cluster
+    // along z) split K; split k owns the 32-row quarters q with q S / 4 = k.
+    // Warps whose quarter another split owns TMA-store their fp32 partial
+    // boxes to that split's plane of the scratch (map in tmV's slot); after a
+    // cluster barrier the owning warps TMA-load the other splits' boxes of
+    // their rows (into the drained staging of the non-owning warps), add them
+    // in split order (deterministic) and finish as in the direct form.
+    constexpr int kChunks = BN / 2 / 32;  // 32-column boxes per warp
+    const bool m3 = SPLIT && mode == 3;
+    const bool owner = !m3 || (q * S) / 4 == split;
+    // Staging region of the non-owner warp that holds peer pi's boxes for the
+    // owner warp (q, half): the same half, quarter q ^ 2 (S = 2) or the pi-th
+    // quarter other than q (S = 4); epilogue warp w has quarter (w + 2) & 3
+    // and half w >> 2.
+    auto peer_region = [&](int pi) -> uint8_t* {
+      const int q2 = S == 2 ? (q ^ 2) : (pi < q ? pi : pi + 1);
+      const int w = half * 4 + ((q2 - 2) & 3);
+      return smem + w * kChunks * 4096;
+    };
+    if (m3) {
+      if (epi && !owner && ok) {
+        uint8_t* stg = smem + (warp - 2) * kChunks * 4096;
+#pragma unroll 1
+        for (int cb = 0; cb < kChunks; ++cb) {
+          const int c = half * (BN / 2) + cb * 32;
+          float v[32];
+          tmem_ld32(trow + c, v);
+          uint8_t* box = stg + cb * 4096;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(box + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tma_store_3d(&tmV, box, n0 + c, m0 + q * 32, split);
+        }
+        if (lane == 0) {
+          bulk_commit_group();
+          bulk_wait_all();
+        }
+      }
+      __threadfence();
+      tc_fence_before();
+      __syncwarp();
+      cluster_sync();  // every partial box of the cluster is in the scratch
+      tc_fence_after();
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      if (epi && owner && ok) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&peer_bar[warp - 2], static_cast<uint32_t>((S - 1) * kChunks * 4096));
+          int pi = 0;
+          for (int k = 0; k < S; ++k) {
+            if (k == split) continue;
+            uint8_t* dst = peer_region(pi);
+            for (int cb = 0; cb < kChunks; ++cb)
+              tma_load_3d(dst + cb * 4096, &tmV, &peer_bar[warp - 2], n0 + half * (BN / 2) + cb * 32, m0 + q * 32, k);
+            ++pi;
+          }
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(&peer_bar[warp - 2], 0));
+        if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+      }
+    }
+    if (epi && owner) {
+      if (mode == 1) named_barrier_sync(1, kEpiThreads);  // bias staged (mode 3: the cluster barrier)
       const int grow = m0 + r;
       void* outp = region == 1 ? e.out_k : e.out;
       const int ocol0 = region > 0 ? region * e.qkv_d : 0;
@@ -313,6 +380,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
         float v[32];
         if (ok) tmem_ld32(trow + c, v);
+        if (m3 && ok) {
+          // partials in split order 0..S-1, this CTA's own (TMEM) in its place
+          const int cb = (c - half * (BN / 2)) / 32;
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+          int pi = 0;
+          for (int k = 0; k < S; ++k) {
+            if (k == split) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc[i] += v[i];
+              continue;
+            }
+            const uint8_t* src = peer_region(pi) + cb * 4096;
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 pv = *reinterpret_cast<const float4*>(src + lane * 128 + ((k4 ^ (lane & 7)) << 4));
+              acc[4 * k4] += pv.x; acc[4 * k4 + 1] += pv.y; acc[4 * k4 + 2] += pv.z; acc[4 * k4 + 3] += pv.w;
+            }
+            ++pi;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = acc[i];
+        }
         const int col = n0 + c;
         if (e.residual && grow < s.M) {
           const int64_t roff =
@@ -386,7 +477,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     tc_fence_before();
     __syncthreads();
-  } else if (mode == 2) {
+  } else if (SPLIT && mode == 2) {
     // ------------------------------------------------------------ split-K
     const int rows_max = (C::BM + S - 1) / S;
     const uint32_t slot_bytes = static_cast<uint32_t>(rows_max) * C::ROW_CHUNKS * 16;
@@ -581,7 +672,11 @@ int gemm_pick(GemmShape* s, int bn_divides) {
 
 template <int BN>
 static cudaError_t prepare_bn() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM);
+  cudaError_t r =
+      cudaFuncSetAttribute(gemm_tc_kernel<BN, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(gemm_tc_kernel<BN, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM);
+  return r;
 }
 
 cudaError_t gemm_prepare() {
@@ -602,7 +697,7 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
                              const GemmEpilogue& e, int vec_ok, int mode, int* err, cudaStream_t st) {
   using C = GemmCfg<BN>;
   const int S = s.splits;
-  dim3 grid((s.M + 127) / 128, (s.N + BN - 1) / BN, S > 1 ? S : s.batch);
+  dim3 grid((s.M + 127) / 128, (s.N + BN - 1) / BN, S > 1 ? S : s.batch);  // modes 2 and 3: S > 1
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kGemmThreads);
@@ -614,10 +709,13 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = 1;
   attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = S > 1 ? S : 1;
+  attr[1].val.clusterDim.z = S > 1 ? S : 1;  // modes 2 and 3
   cfg.attrs = attr;
   cfg.numAttrs = S > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, tmA, tmB, tmO, tmO2, tmV, s, e, vec_ok, mode, err);
+  const GemmDims sd = s;      // the kernel's parameter block holds only
+  const GemmEpiArgs ea = e;   // what it reads
+  return S > 1 ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, true>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok, mode, err)
+               : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok, mode, err);
 }
 
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
@@ -643,7 +741,12 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   std::memset(&tmO2, 0, sizeof tmO2);
   std::memset(&tmV, 0, sizeof tmV);
   int mode = s.splits > 1 ? 2 : 0;
-  const bool tma_ok = s.splits == 1 && bn >= 64 && vec && (e.ldo * esz_out) % 16 == 0 &&
+  // split-K through L2 (mode 3): S = 2 or 4, the scratch, and a TMA-storable output
+  const bool l2split = s.split_l2 && (s.splits == 2 || s.splits == 4) && e.part_ws && e.qkv_d == 0 &&
+                       s.N <= e.ws_ld && e.ws_ld % 4 == 0 && e.ws_rows >= 128L * ((s.M + 127) / 128) &&
+                       (reinterpret_cast<uintptr_t>(e.part_ws) % 16) == 0;
+  if (s.split_l2 && !l2split) return cudaErrorInvalidValue;
+  const bool tma_ok = (s.splits == 1 || l2split) && bn >= 64 && vec && (e.ldo * esz_out) % 16 == 0 &&
                       (e.residual == nullptr || (e.ldr * esz_res) % 16 == 0);
   if (tma_ok) {
     const uint64_t cols = e.qkv_d > 0 ? static_cast<uint64_t>(e.qkv_d) : static_cast<uint64_t>(s.N);
@@ -664,8 +767,16 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
       built = built && !e.out_f32 && e.t_pad % 8 == 0 &&
               make_tmap(&tmV, e.vt, 2, vd, vs, vb, 2, 64) == cudaSuccess;
     }
-    if (built) mode = 1;
+    if (built && l2split) {
+      // the scratch planes [S][ws_rows][ws_ld] fp32, 32 x 32 boxes, 128-byte swizzle
+      const uint64_t wd[3] = {static_cast<uint64_t>(e.ws_ld), static_cast<uint64_t>(e.ws_rows),
+                              static_cast<uint64_t>(s.splits)};
+      const uint64_t ws[2] = {static_cast<uint64_t>(e.ws_ld) * 4, static_cast<uint64_t>(e.ws_rows * e.ws_ld) * 4};
+      built = make_tmap(&tmV, e.part_ws, 3, wd, ws, box, 4, 128) == cudaSuccess;
+    }
+    if (built) mode = l2split ? 3 : 1;
   }
+  if (l2split && mode != 3) return cudaErrorInvalidValue;
   switch (bn) {
     case 32: return launch_bn<32>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
     case 64: return launch_bn<64>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);

@@ -189,6 +189,8 @@ struct w2v_model {
   int* err_word = nullptr;
   int32_t* ids = nullptr;
   float* tune_logits = nullptr;  // output of the lm_head GEMM while tuning
+  float* part_ws = nullptr;      // split-K through L2: fp32 [4][ws_rows][ws_ld]
+  int64_t ws_rows = 0, ws_ld = 0;
   int max_rows = 0;
   std::map<std::pair<int, int>, std::unique_ptr<Plan>> plans;
   std::map<std::tuple<int, int, const void*, void*>, cudaGraphExec_t> graphs;
@@ -244,8 +246,18 @@ cudaError_t map_a(CUtensorMap* t, const void* base, int64_t cols, int64_t rows, 
 }
 
 // ------------------------------------------------ epilogues of each GEMM role
-GemmEpilogue epi_conv(const w2v_model* m, const Plan& p, int i) {
+// Every GEMM epilogue carries the split-K scratch (used only when split
+// through L2).
+GemmEpilogue epi_base(const w2v_model* m) {
   GemmEpilogue e;
+  e.part_ws = m->part_ws;
+  e.ws_rows = m->ws_rows;
+  e.ws_ld = m->ws_ld;
+  return e;
+}
+
+GemmEpilogue epi_conv(const w2v_model* m, const Plan& p, int i) {
+  GemmEpilogue e = epi_base(m);
   e.bias = m->cb[i];
   e.out = (i % 2 == 0) ? m->act_a : m->act_b;
   e.ldo = kC;
@@ -255,7 +267,7 @@ GemmEpilogue epi_conv(const w2v_model* m, const Plan& p, int i) {
 }
 
 GemmEpilogue epi_proj(const w2v_model* m) {
-  GemmEpilogue e;
+  GemmEpilogue e = epi_base(m);
   e.bias = m->bp;
   e.out = m->x;
   e.ldo = m->cfg.d_model;
@@ -263,7 +275,7 @@ GemmEpilogue epi_proj(const w2v_model* m) {
 }
 
 GemmEpilogue epi_qkv(const w2v_model* m, const Plan& p, int l) {
-  GemmEpilogue e;
+  GemmEpilogue e = epi_base(m);
   e.bias = m->L[l].bqkv;
   e.out = m->q;
   e.ldo = m->cfg.d_model;
@@ -278,7 +290,7 @@ GemmEpilogue epi_qkv(const w2v_model* m, const Plan& p, int l) {
 
 // out_proj (ffn = false) or FFN2 (ffn = true): bias + residual into the fp32 stream
 GemmEpilogue epi_resid(const w2v_model* m, int l, bool ffn) {
-  GemmEpilogue e;
+  GemmEpilogue e = epi_base(m);
   e.bias = ffn ? m->L[l].b2 : m->L[l].bo;
   if (m->cfg.stable_layer_norm) {
     e.residual = m->r;
@@ -295,7 +307,7 @@ GemmEpilogue epi_resid(const w2v_model* m, int l, bool ffn) {
 }
 
 GemmEpilogue epi_ffn1(const w2v_model* m, int l) {
-  GemmEpilogue e;
+  GemmEpilogue e = epi_base(m);
   e.bias = m->L[l].b1;
   e.act = m->cfg.gelu_tanh ? 2 : 1;
   e.out = m->f;
@@ -304,7 +316,7 @@ GemmEpilogue epi_ffn1(const w2v_model* m, int l) {
 }
 
 GemmEpilogue epi_lm(const w2v_model* m, float* logits) {
-  GemmEpilogue e;
+  GemmEpilogue e = epi_base(m);
   e.bias = m->blm;
   e.out = logits;
   e.out_f32 = 1;
@@ -316,6 +328,12 @@ GemmEpilogue epi_lm(const w2v_model* m, float* logits) {
 // candidates on the plan's own buffers (CUDA events on a private stream), or
 // by the analytic model when W2V_AUTOTUNE=0.  Every candidate computes the
 // same result; without split-K even bit for bit.
+// Whether a GEMM may split K by `sp` (2 or 4) through the L2 scratch.
+bool l2_split_ok(const w2v_model* m, const GemmShape& s, int N, int bn, int sp) {
+  return s.batch == 1 && bn >= 64 && N <= m->ws_ld && 128L * ((s.M + 127) / 128) <= m->ws_rows &&
+         s.K / 64 >= 2 * sp;
+}
+
 int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* W, int N, int K,
               const GemmEpilogue& e, int bn_divides, int* bn_out) {
   const char* env = std::getenv("W2V_AUTOTUNE");
@@ -335,10 +353,14 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     if (bn_divides > 0 && bn_divides % bn != 0) continue;
     CUtensorMap tmB;
     CUDA_OR(m, map_matrix(&tmB, W, N, K, bn));
-    for (int sp : {1, 2, 3, 4, 6}) {
+    // sp > 1: K splits reduced through distributed shared memory; sp < 0:
+    // -sp splits reduced through the L2 scratch
+    for (int sp : {1, 2, 3, 4, 6, -2, -4}) {
       if (sp > 1 && (s->batch != 1 || nk < 16 || sp > nk)) continue;
+      if (sp < 0 && !l2_split_ok(m, *s, N, bn, -sp)) continue;
       GemmShape c = *s;
-      c.splits = sp;
+      c.splits = sp < 0 ? -sp : sp;
+      c.split_l2 = sp < 0;
       CUDA_OR(m, launch_gemm(tmA, tmB, c, bn, e, m->err_word, st));
       CUDA_OR(m, cudaEventRecord(e0, st));
       for (int it = 0; it < 3; ++it) CUDA_OR(m, launch_gemm(tmA, tmB, c, bn, e, m->err_word, st));
@@ -356,7 +378,8 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
   if (!best_bn) return fail(m, W2V_ECUDA, "no GEMM configuration for N=%d K=%d", N, K);
-  s->splits = best_s;
+  s->splits = best_s < 0 ? -best_s : best_s;
+  s->split_l2 = best_s < 0;
   *bn_out = best_bn;
   return W2V_OK;
 }
@@ -862,6 +885,11 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   wtake(reinterpret_cast<void**>(&m->err_word), 256);
   wtake(reinterpret_cast<void**>(&m->ids), 3 * rows * 4);
   wtake(reinterpret_cast<void**>(&m->tune_logits), rows * static_cast<size_t>(V) * 4);  // ids, plus token scratch of the profiler
+  // Split-K scratch: GEMMs of at most 2048 rows (128-row tiles) and at most
+  // max(d, 512) columns may split K through L2.
+  m->ws_rows = std::min<int64_t>((static_cast<int64_t>(B) * tf + 127) / 128 * 128, 2048);
+  m->ws_ld = std::max(d, kC);
+  wtake(reinterpret_cast<void**>(&m->part_ws), static_cast<size_t>(4) * m->ws_rows * m->ws_ld * 4);
   const size_t wsbytes = round_up(cursor, 1 << 20);
   if (cudaMalloc(&m->ws, wsbytes) != cudaSuccess) {
     cudaFree(m->wmem);
@@ -892,13 +920,15 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
 // graph and timed (best of 3 replays), and the fastest is kept (coordinate
 // descent; the incumbent wins ties within 0.5 %).
 namespace {
-int apply_role(w2v_model* m, Plan* p, int role, int bn, int splits) {
+int apply_role(w2v_model* m, Plan* p, int role, int bn, int sp) {
+  const int splits = sp < 0 ? -sp : sp;
   const int d = m->cfg.d_model, F = m->cfg.d_ffn;
   std::vector<CUtensorMap>* maps[4] = {&p->qkvB, &p->oB, &p->f1B, &p->f2B};
   int* bns[4] = {&p->qkvBN, &p->oBN, &p->f1BN, &p->f2BN};
   GemmShape* shapes[4] = {&p->qkvS, &p->oS, &p->f1S, &p->f2S};
   *bns[role] = bn;
   shapes[role]->splits = splits;
+  shapes[role]->split_l2 = sp < 0;
   for (int l = 0; l < m->cfg.n_layers; ++l) {
     const LayerDev& w = m->L[l];
     const __half* W = role == 0 ? w.wqkv : role == 1 ? w.wo : role == 2 ? w.w1 : w.w2;
@@ -956,12 +986,13 @@ int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
     const int nk = K / 64;
     GemmShape* sh = role == 0 ? &p->qkvS : role == 1 ? &p->oS : role == 2 ? &p->f1S : &p->f2S;
     int cur_bn = role == 0 ? p->qkvBN : role == 1 ? p->oBN : role == 2 ? p->f1BN : p->f2BN;
-    int cur_s = sh->splits;
+    int cur_s = sh->split_l2 ? -sh->splits : sh->splits;
     for (int bn : {32, 64, 128, 192, 256}) {
       if (bn == 32 ? N > 32 : N <= bn / 2) continue;
       if (role == 0 && d % bn != 0) continue;
-      for (int sp : {1, 2, 3, 4, 6}) {
+      for (int sp : {1, 2, 3, 4, 6, -2, -4}) {
         if (sp > 1 && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
+        if (sp < 0 && !l2_split_ok(m, *sh, N, bn, -sp)) continue;
         if (bn == cur_bn && sp == cur_s) continue;
         int rc = apply_role(m, p, role, bn, sp);
         if (rc != W2V_OK) return rc;
@@ -1256,15 +1287,18 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return W2V_EINVAL;
   if (act < 0 || act > 2) return W2V_EINVAL;
   if (gemm_prepare() != cudaSuccess) return W2V_ECUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   GemmShape s;
   s.M = M; s.N = N; s.K = K; s.a_kwrap = K; s.batch = 1;
   if (bn == 0) {
     bn = gemm_pick(&s, 0);
   } else {
-    s.splits = splits;
+    s.splits = splits < 0 ? -splits : splits;
+    s.split_l2 = splits < 0;
   }
   if (bn != 32 && bn != 64 && bn != 128 && bn != 192 && bn != 256) return W2V_EINVAL;
   if (s.splits < 1 || s.splits > 8 || s.splits > K / 64) return W2V_EINVAL;
+  if (s.split_l2 && ((s.splits != 2 && s.splits != 4) || bn < 64)) return W2V_EINVAL;
   CUtensorMap ta, tb;
   if (map_a(&ta, A, K, M, K, 1, 0) != cudaSuccess) return W2V_ECUDA;
   if (map_matrix(&tb, B, N, K, bn) != cudaSuccess) return W2V_ECUDA;
@@ -1277,8 +1311,17 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   e.out_f32 = out_f32;
   e.ldo = N;
   e.act = act;
-  return launch_gemm(ta, tb, s, bn, e, err_dev, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W2V_OK
-                                                                                                    : W2V_ECUDA;
+  void* ws = nullptr;
+  if (s.split_l2) {
+    e.ws_rows = 128L * ((M + 127) / 128);
+    e.ws_ld = (N + 3) / 4 * 4;
+    if (cudaMallocAsync(&ws, static_cast<size_t>(s.splits) * e.ws_rows * e.ws_ld * 4, st) != cudaSuccess)
+      return W2V_ENOMEM;
+    e.part_ws = static_cast<float*>(ws);
+  }
+  const cudaError_t r = launch_gemm(ta, tb, s, bn, e, err_dev, st);
+  if (ws) cudaFreeAsync(ws, st);
+  return r == cudaSuccess ? W2V_OK : (r == cudaErrorInvalidValue ? W2V_EINVAL : W2V_ECUDA);
 }
 
 extern "C" int w2v_op_attention(const void* q, const void* k, const void* vt, void* out, int batch, int T, int H,

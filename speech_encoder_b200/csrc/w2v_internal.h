@@ -44,7 +44,11 @@ cudaError_t make_tmap(CUtensorMap* out, const void* base, int rank, const uint64
 // K block starting at k is fetched from column (k % a_kwrap) of row
 // (m0 + k / a_kwrap) — a_kwrap = K for an ordinary matrix, or the width of a
 // pair of frames for the stride-2 conv layers (implicit GEMM).
-struct GemmEpilogue {
+// The kernel's own copy of the epilogue arguments.  It is kept exactly this
+// size: growing the by-value parameter block of the GEMM kernel (even by
+// fields it never reads) measured 30-50 % slower mainloops on B200, so
+// host-only additions go into GemmEpilogue below.
+struct GemmEpiArgs {
   const float* bias = nullptr;     // [N] or null
   const void* residual = nullptr;  // [rows, ldr], fp16 or fp32 per res_f32, or null
   int res_f32 = 0;
@@ -66,10 +70,20 @@ struct GemmEpilogue {
   int t_len = 0;                   // frames per clip (rows are clip-major)
 };
 
+struct GemmEpilogue : GemmEpiArgs {
+  // Split-K scratch for GemmShape::split_l2: fp32 [splits][ws_rows][ws_ld],
+  // ws_rows >= the row tiles' extent (128 * ceil(M / 128)), ws_ld >= N.  The
+  // kernel reaches it through a tensor map only.
+  float* part_ws = nullptr;
+  int64_t ws_rows = 0;
+  int64_t ws_ld = 0;
+};
+
 // Streaming multiprocessors of a B200: the grid of the persistent kernels.
 constexpr int kNumSMs = 148;
 
-struct GemmShape {
+// The kernel's copy of the problem shape (see GemmEpiArgs on its size).
+struct GemmDims {
   int M = 0;        // valid rows per batch item
   int N = 0;        // valid output columns
   int K = 0;        // multiple of 64
@@ -77,7 +91,12 @@ struct GemmShape {
   int batch = 1;
   int splits = 1;   // split-K factor (batch must be 1 when > 1): the splits of
                     // one output tile form a thread-block cluster and reduce
-                    // their fp32 partials through distributed shared memory
+                    // their fp32 partials through distributed shared memory,
+};
+
+struct GemmShape : GemmDims {
+  bool split_l2 = false;  // or, with splits 2 or 4, through the L2 scratch of
+                          // GemmEpilogue (TMA stores and loads of fp32 boxes)
 };
 
 // Chooses the N tile width (returned) and the split-K factor (s->splits) for

@@ -77,9 +77,14 @@ def test_small_model_stages_match_oracle():
         model.close()
 
 
-def test_graph_replay_equals_direct_launch_and_is_deterministic():
+def test_graph_replay_equals_direct_launch_and_is_deterministic(monkeypatch):
+    # Two models only share a launch plan when neither times candidates (a
+    # measured choice of split-K changes the summation order), so the
+    # graph-versus-direct comparison runs on the analytic plan; a tuned model
+    # must still replay bit-identically.
     shape = S.small_shape()
     pcm = S.synth_pcm(30000, 9)[None]
+    monkeypatch.setenv("W2V_AUTOTUNE", "0")
     m1 = U.make_model(shape, 48000, 1, use_cuda_graph=False)
     m2 = U.make_model(shape, 48000, 1, use_cuda_graph=True)
     a = _run(m1, pcm)
@@ -88,6 +93,12 @@ def test_graph_replay_equals_direct_launch_and_is_deterministic():
     assert np.array_equal(a, b) and np.array_equal(b, c)
     m1.close()
     m2.close()
+    monkeypatch.delenv("W2V_AUTOTUNE")
+    m3 = U.make_model(shape, 48000, 1, use_cuda_graph=True)
+    d = _run(m3, pcm)
+    e = _run(m3, pcm)
+    assert np.array_equal(d, e)
+    m3.close()
 
 
 def test_forward_rejects_bad_shapes_without_launching():

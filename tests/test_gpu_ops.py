@@ -41,6 +41,13 @@ GEMM_CASES = [
     (130, 96, 512, (64, 8), 2, None, 0),
     (1, 2341, 1024, (256, 5), 0, None, 1),
     (799, 512, 1024, (192, 3), 1, "f16", 0),
+    # split-K through the L2 scratch (splits -2 / -4)
+    (799, 768, 3072, (128, -4), 0, "f16", 1),
+    (799, 768, 3072, (256, -2), 0, "f32", 1),
+    (799, 768, 768, (64, -2), 0, "f16", 1),
+    (130, 96, 512, (64, -4), 2, None, 0),
+    (257, 512, 1536, (192, -4), 1, "f16", 0),
+    (1, 640, 1024, (256, -2), 0, None, 1),
 ]
 
 
@@ -77,7 +84,8 @@ def test_gemm_every_tile_width_same_result():
     A = torch.randn(M, K, generator=g).half().cuda()
     W = (torch.randn(N, K, generator=g) * 0.05).half().cuda()
     outs = []
-    for bn, sp in ((32, 1), (64, 1), (128, 1), (192, 1), (256, 1), (256, 2), (128, 8), (64, 3)):
+    for bn, sp in ((32, 1), (64, 1), (128, 1), (192, 1), (256, 1), (256, 2), (128, 8), (64, 3), (256, -2),
+                   (128, -4), (192, -4)):
         out = torch.empty(M, N, dtype=torch.float32, device="cuda")
         assert B.w2v_op_gemm(A, W, M, N, K, None, None, 0, out, 1, 0, _err(), bn=bn, splits=sp) == 0
         outs.append(out)
