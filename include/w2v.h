@@ -111,7 +111,12 @@ int w2v_create(const w2v_config* cfg, const float* host_weights, size_t n_floats
  * then re-chooses the per-layer GEMMs by timing the whole forward with each
  * candidate (a few hundred milliseconds, synchronous; W2V_AUTOTUNE=0 in the
  * environment uses a cost model instead, W2V_TUNE_LOG=1 prints the choices),
- * so make that first call outside any stream capture.
+ * so make that first call outside any stream capture.  With W2V_PLAN_FILE set
+ * to a path, a plan tuned for this model shape, n_samples and batch is
+ * appended to that text file, and a later process that finds its line there
+ * launches exactly those GEMM configurations without timing anything (the
+ * same kernels, hence bit-identical logits, across processes); a line whose
+ * choices do not fit the shapes makes the call fail with W2V_EINVAL.
  * Errors: W2V_ESHAPE if n_samples < 400 or > max_samples or batch outside
  * [1, max_batch]; W2V_EINVAL for null/misaligned pointers. */
 int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, void* stream);

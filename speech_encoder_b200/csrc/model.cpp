@@ -189,6 +189,10 @@ struct w2v_model {
   int* err_word = nullptr;
   int32_t* ids = nullptr;
   float* tune_logits = nullptr;  // output of the lm_head GEMM while tuning
+  // GEMM choices read from W2V_PLAN_FILE for the plan being built, consumed in
+  // tune_gemm's call order (see plan_file_key); empty when tuning.
+  std::vector<std::pair<int, int>> forced;
+  size_t forced_i = 0;
   float* part_ws = nullptr;      // split-K through L2: fp32 [4][ws_rows][ws_ld]
   int64_t ws_rows = 0, ws_ld = 0;
   int max_rows = 0;
@@ -336,12 +340,26 @@ bool l2_split_ok(const w2v_model* m, const GemmShape& s, int N, int bn, int sp) 
 
 int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* W, int N, int K,
               const GemmEpilogue& e, int bn_divides, int* bn_out) {
+  const int nk = K / 64;
+  if (m->forced_i < m->forced.size()) {
+    const int bn = m->forced[m->forced_i].first, sp = m->forced[m->forced_i].second;
+    ++m->forced_i;
+    const int splits = sp < 0 ? -sp : sp;
+    const bool bn_ok = (bn == 32 || bn == 64 || bn == 128 || bn == 192 || bn == 256) &&
+                       (bn_divides <= 0 || bn_divides % bn == 0);
+    const bool sp_ok = sp == 1 || (sp > 1 && sp <= 8 && s->batch == 1 && sp <= nk) ||
+                       ((sp == -2 || sp == -4) && l2_split_ok(m, *s, N, bn, -sp));
+    if (!bn_ok || !sp_ok) return fail(m, W2V_EINVAL, "plan file: bn=%d splits=%d invalid for N=%d K=%d", bn, sp, N, K);
+    s->splits = splits;
+    s->split_l2 = sp < 0;
+    *bn_out = bn;
+    return W2V_OK;
+  }
   const char* env = std::getenv("W2V_AUTOTUNE");
   if (env && env[0] == '0') {
     *bn_out = gemm_pick(s, bn_divides);
     return W2V_OK;
   }
-  const int nk = K / 64;
   cudaStream_t st = m->cap_stream;
   cudaEvent_t e0, e1;
   CUDA_OR(m, cudaEventCreate(&e0));
@@ -489,6 +507,57 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
 
 int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits);
 
+// Plan file (W2V_PLAN_FILE): one line per (model shape, n_samples, batch),
+//   <key> bn:sp bn:sp ...
+// with the GEMM choices in build order: conv layers 1-6, projection, then
+// (with encoder layers) QKV, out-projection, FFN1, FFN2, then the lm_head.
+// sp > 1 splits K through distributed shared memory, sp < 0 through L2.  A
+// process that finds its key reuses the choices instead of timing anything,
+// so that separate processes (a benchmark and a profiler run of it) launch the
+// same kernels; one that does not appends the plan it tuned.
+std::string plan_file_key(const w2v_model* m, int n, int batch) {
+  const w2v_config& c = m->cfg;
+  char buf[192];
+  std::snprintf(buf, sizeof buf, "w2v-plan-1:d%d:f%d:h%d:l%d:v%d:norm%d:st%d:n%d:b%d", c.d_model, c.d_ffn, c.n_heads,
+                c.n_layers, c.vocab, c.conv_norm, c.stable_layer_norm, n, batch);
+  return buf;
+}
+
+void plan_file_read(const char* path, const std::string& key, std::vector<std::pair<int, int>>* out) {
+  FILE* f = std::fopen(path, "r");
+  if (!f) return;
+  char line[1024];
+  while (std::fgets(line, sizeof line, f)) {
+    char* save = nullptr;
+    char* tok = strtok_r(line, " \t\n", &save);
+    if (!tok || key != tok) continue;
+    out->clear();
+    while ((tok = strtok_r(nullptr, " \t\n", &save))) {
+      int bn = 0, sp = 0;
+      if (std::sscanf(tok, "%d:%d", &bn, &sp) == 2) out->emplace_back(bn, sp);
+    }
+  }
+  std::fclose(f);
+}
+
+void plan_file_append(const char* path, const std::string& key, const Plan& p, bool layers) {
+  FILE* f = std::fopen(path, "a");
+  if (!f) return;
+  auto put = [&](int bn, const GemmShape& s) { std::fprintf(f, " %d:%d", bn, s.split_l2 ? -s.splits : s.splits); };
+  std::fputs(key.c_str(), f);
+  for (int i = 1; i < 7; ++i) put(p.convBN[i], p.convS[i]);
+  put(p.projBN, p.projS);
+  if (layers) {
+    put(p.qkvBN, p.qkvS);
+    put(p.oBN, p.oS);
+    put(p.f1BN, p.f1S);
+    put(p.f2BN, p.f2S);
+  }
+  put(p.lmBN, p.lmS);
+  std::fputc('\n', f);
+  std::fclose(f);
+}
+
 int get_plan(w2v_model* m, int n, int batch, const Plan** out, const float* pcm, float* logits) {
   auto key = std::make_pair(n, batch);
   auto it = m->plans.find(key);
@@ -497,9 +566,20 @@ int get_plan(w2v_model* m, int n, int batch, const Plan** out, const float* pcm,
     return W2V_OK;
   }
   std::unique_ptr<Plan> p(new Plan());
+  const char* pf = std::getenv("W2V_PLAN_FILE");
+  const std::string pkey = plan_file_key(m, n, batch);
+  m->forced.clear();
+  m->forced_i = 0;
+  if (pf && *pf) plan_file_read(pf, pkey, &m->forced);
+  const bool pinned = !m->forced.empty();
   int rc = build_plan(m, n, batch, p.get());
-  if (rc == W2V_OK) rc = refine_plan(m, p.get(), pcm, logits);
+  if (rc == W2V_OK && pinned && m->forced_i != m->forced.size())
+    rc = fail(m, W2V_EINVAL, "plan file: %zu GEMM choices for %s, %zu used", m->forced.size(), pkey.c_str(),
+              m->forced_i);
+  m->forced.clear();
+  if (rc == W2V_OK && !pinned) rc = refine_plan(m, p.get(), pcm, logits);
   if (rc != W2V_OK) return rc;
+  if (pf && *pf && !pinned) plan_file_append(pf, pkey, *p, m->cfg.n_layers > 0);
   *out = p.get();
   m->plans[key] = std::move(p);
   return W2V_OK;

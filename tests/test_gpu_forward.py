@@ -212,3 +212,34 @@ def test_c4_large_true_length_clips_sampled():
     for i in (int(np.argmin(lens)), int(np.argmax(lens))):
         print("c4", i, lens[i], U.compare_logits(outs[i][0], U.oracle_workload_clip("c4", i, 0), f"c4 clip {i}"))
     m.close()
+
+
+def test_plan_file_pins_the_gemm_choices_across_models(tmp_path, monkeypatch):
+    # The first model tunes and appends its plan; the second finds the line,
+    # launches the same GEMM configurations without timing, and so reproduces
+    # the logits bit for bit.  A line that does not fit the shapes is refused.
+    shape = S.small_shape()
+    pcm = S.synth_pcm(30000, 9)[None]
+    path = tmp_path / "plans.txt"
+    monkeypatch.setenv("W2V_PLAN_FILE", str(path))
+    m1 = U.make_model(shape, 48000, 1)
+    a = _run(m1, pcm)
+    m1.close()
+    lines = path.read_text().splitlines()
+    assert len(lines) == 1
+    key, *choices = lines[0].split()
+    assert key.startswith("w2v-plan-1:") and len(choices) == 6 + 1 + 4 + 1
+    for c in choices:
+        bn, sp = (int(x) for x in c.split(":"))
+        assert bn in (32, 64, 128, 192, 256) and sp != 0
+    m2 = U.make_model(shape, 48000, 1)
+    b = _run(m2, pcm)
+    m2.close()
+    assert np.array_equal(a, b)
+    assert len(path.read_text().splitlines()) == 1  # found, not re-tuned
+    bad = " ".join([key] + ["96:1"] * len(choices))
+    path.write_text(bad + "\n")
+    m3 = U.make_model(shape, 48000, 1)
+    with pytest.raises(B.W2VError):
+        _run(m3, pcm)
+    m3.close()
