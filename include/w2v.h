@@ -117,6 +117,11 @@ int w2v_create(const w2v_config* cfg, const float* host_weights, size_t n_floats
  * launches exactly those GEMM configurations without timing anything (the
  * same kernels, hence bit-identical logits, across processes); a line whose
  * choices do not fit the shapes makes the call fail with W2V_EINVAL.
+ * Post-norm models (stable_layer_norm = 0) with encoder layers run the two
+ * LayerNorms of every block inside the neighbouring GEMMs (gamma folded into
+ * the next weights at w2v_create, row statistics as partial sums written by
+ * the GEMM that produces the rows); W2V_LN_FOLD=0 in the environment at
+ * w2v_create keeps them as separate kernels.
  * Errors: W2V_ESHAPE if n_samples < 400 or > max_samples or batch outside
  * [1, max_batch]; W2V_EINVAL for null/misaligned pointers. */
 int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, float* logits_dev, void* stream);

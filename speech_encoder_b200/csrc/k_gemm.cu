@@ -52,7 +52,9 @@ struct GemmCfg {
   static constexpr int CHUNK = BN >= 64 ? 32 : 16;  // TMEM columns per load
   static constexpr int ROW_CHUNKS = BN / 4;         // 16-byte fp32 chunks per row
   static constexpr int BIAS_OFF = RING;
-  static constexpr int BAR_OFF = BIAS_OFF + BN * 4;
+  static constexpr int VEC_OFF = BIAS_OFF + BN * 4;   // LN column vectors, 2 x BN floats
+  static constexpr int ROWLN_OFF = VEC_OFF + 2 * BN * 4;  // per-row LN factors, 128 float2
+  static constexpr int BAR_OFF = ROWLN_OFF + 128 * 8;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
   static_assert(BM * BN * 4 <= RING, "parked tile must fit in the operand ring");
   static_assert(ROW_CHUNKS >= 8, "row swizzle needs >= 8 chunks");
@@ -60,6 +62,7 @@ struct GemmCfg {
 
 constexpr int kGemmThreads = 320;
 constexpr int kEpiThreads = 256;
+static_assert(sizeof(GemmEpiArgs) <= 128, "the GEMM kernel's parameter block must stay within 808 bytes");
 
 // fp32 tile rows of `row_chunks` 16-byte chunks; chunk j of row r lives at
 // chunk (j ^ (r & 7)) so that 8 consecutive rows hit 8 different bank groups.
@@ -75,19 +78,29 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // Final epilogue for 4 consecutive columns [col, col+4) of row grow: bias
 // (from shared memory), GELU, residual, store.  `vec` selects 16-/8-byte
 // accesses (row starts and pointers 16-byte aligned, full 4-vector in range).
-__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, int lcol, int grow, int col, int nv,
-                                        int bzb, const GemmEpiArgs& e, void* outp, int ocol0, bool vec) {
+// lnr: the row's LayerNorm factors (rstd, -mean * rstd) when e.ln_mode != 0;
+// vec_s: the LN column vectors of this tile (ln_mode 1: column sums; 2: gamma,
+// then beta at vec_s + BN).
+__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, const float* vec_s, int bn, float2 lnr,
+                                        int lcol, int grow, int col, int nv, int bzb, const GemmEpiArgs& e,
+                                        void* outp, int ocol0, bool vec) {
+  const int ln_mode = e.ln_cfg & 255;
+  if (ln_mode == 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = fmaf(lnr.x, x[i], lnr.y * vec_s[lcol + i]);
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) x[i] = apply_act(x[i] + bias_s[lcol + i], e.act);
   if (e.residual) {
     const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+    float rv[4] = {0.f, 0.f, 0.f, 0.f};
     if (e.res_f32) {
       const float* rp = static_cast<const float*>(e.residual) + roff;
       if (vec && nv == 4) {
-        const float4 rv = *reinterpret_cast<const float4*>(rp);
-        x[0] += rv.x; x[1] += rv.y; x[2] += rv.z; x[3] += rv.w;
+        const float4 t = *reinterpret_cast<const float4*>(rp);
+        rv[0] = t.x; rv[1] = t.y; rv[2] = t.z; rv[3] = t.w;
       } else {
-        for (int i = 0; i < nv; ++i) x[i] += rp[i];
+        for (int i = 0; i < nv; ++i) rv[i] = rp[i];
       }
     } else {
       const __half* rp = static_cast<const __half*>(e.residual) + roff;
@@ -95,11 +108,17 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, int 
         const uint2 u = *reinterpret_cast<const uint2*>(rp);
         const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
         const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-        x[0] += a.x; x[1] += a.y; x[2] += b.x; x[3] += b.y;
+        rv[0] = a.x; rv[1] = a.y; rv[2] = b.x; rv[3] = b.y;
       } else {
-        for (int i = 0; i < nv; ++i) x[i] += __half2float(rp[i]);
+        for (int i = 0; i < nv; ++i) rv[i] = __half2float(rp[i]);
       }
     }
+    if (ln_mode == 2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rv[i] = fmaf(fmaf(rv[i], lnr.x, lnr.y), vec_s[lcol + i], vec_s[bn + lcol + i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] += rv[i];
   }
   const int64_t ooff = static_cast<int64_t>(bzb) * e.out_batch_stride + static_cast<int64_t>(grow) * e.ldo + (col - ocol0);
   if (e.out_f32) {
@@ -129,6 +148,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + C::BIAS_OFF);
+  float* vec_s = reinterpret_cast<float*>(smem + C::VEC_OFF);
+  float2* rowln_s = reinterpret_cast<float2*>(smem + C::ROWLN_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
@@ -244,13 +265,102 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
   const int region = e.qkv_d > 0 ? n0 / e.qkv_d : -1;
   const bool vec = vec_ok != 0;
+  const int ln_mode = e.ln_cfg & 255;
   bool ok = true;
   if (epi) {
     for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (e.bias && n0 + i < s.N) ? e.bias[n0 + i] : 0.f;
+    if (ln_mode == 1) {
+      for (int i = et; i < BN; i += kEpiThreads) vec_s[i] = n0 + i < s.N ? e.ln_vec[n0 + i] : 0.f;
+    } else if (ln_mode == 2) {
+      for (int i = et; i < BN; i += kEpiThreads) {
+        vec_s[i] = n0 + i < s.N ? e.ln_vec[n0 + i] : 0.f;
+        vec_s[BN + i] = n0 + i < s.N ? e.ln_vec[s.N + n0 + i] : 0.f;
+      }
+    }
+    if (ln_mode != 0) {
+      // Row statistics from the partial sums the producing GEMM stored (it is
+      // a previous kernel: wait for it here, while the mainloop runs), added
+      // in partial order: rowln_s[row] = (rstd, -mean * rstd).  The width is
+      // the A row (mode 1) or the output row (mode 2).
+      pdl_wait();
+      if (et < C::BM) {
+        const int grow = m0 + et;
+        float2 f = make_float2(1.f, 0.f);
+        if (grow < s.M) {
+          const int parts = e.ln_cfg >> 8;
+          float s1 = 0.f, s2 = 0.f;
+          for (int p = 0; p < parts; ++p) {
+            const float2 t = e.ln_in[static_cast<int64_t>(p) * s.M + grow];
+            s1 += t.x;
+            s2 += t.y;
+          }
+          const float inv = 1.f / static_cast<float>(ln_mode == 1 ? s.K : s.N);
+          const float mean = s1 * inv;
+          const float rstd = rsqrtf(fmaxf(fmaf(s2, inv, -mean * mean), 0.f) + e.ln_eps);
+          f = make_float2(rstd, -mean * rstd);
+        }
+        rowln_s[et] = f;
+      }
+    }
     ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
     if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
     tc_fence_after();
   }
+  // The LayerNorm factors (rstd, -mean * rstd) of tile row lrow.
+  auto row_lnr = [&](int lrow) -> float2 { return ln_mode != 0 ? rowln_s[lrow] : make_float2(1.f, 0.f); };
+  // Modes 0 and 2 with partial row sums to store: each epilogue warp takes
+  // whole rows (lr0 + lr, lr < nrows, tile rows r0 + lr) and its lanes the
+  // rows' 16-byte chunks, so that a row's two half-tile sums reduce inside the
+  // warp in a fixed order.  fetch4(lr, j) gives chunk j of the row's fp32 sums.
+  auto finish_rows_stats = [&](int r0, int nrows, void* outp, int ocol0, auto&& fetch4) {
+    constexpr int RC = C::ROW_CHUNKS;
+    constexpr int RPW = RC >= 32 ? 1 : 32 / RC;  // rows per warp pass
+    constexpr int JSTEP = RC >= 32 ? 32 : RC;
+    const int ew = et >> 5;
+    const int sub = RC >= 32 ? 0 : lane / RC;
+    const int j0 = RC >= 32 ? lane : lane % RC;
+#pragma unroll 1
+    for (int lb = ew * RPW; lb < nrows; lb += (kEpiThreads / 32) * RPW) {
+      const int lr = lb + sub;
+      const int grow = m0 + r0 + lr;
+      const bool live = lr < nrows && grow < s.M;
+      float a1 = 0.f, a2 = 0.f, b1 = 0.f, b2 = 0.f;
+      if (live) {
+        const float2 lnr = row_lnr(r0 + lr);
+        for (int j = j0; j < RC; j += JSTEP) {
+          const int col = n0 + 4 * j;
+          if (col >= s.N) continue;
+          const int nv = min(4, s.N - col);
+          const float4 v = fetch4(lr, j);
+          float x[4] = {v.x, v.y, v.z, v.w};
+          finish4(x, bias_s, vec_s, BN, lnr, 4 * j, grow, col, nv, bzb, e, outp, ocol0, vec);
+          float p1 = 0.f, p2 = 0.f;
+          for (int i = 0; i < nv; ++i) {
+            p1 += x[i];
+            p2 = fmaf(x[i], x[i], p2);
+          }
+          if (4 * j < BN / 2) {
+            a1 += p1;
+            a2 += p2;
+          } else {
+            b1 += p1;
+            b2 += p2;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = (RC >= 32 ? 16 : RC / 2); o > 0; o >>= 1) {
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+        b1 += __shfl_xor_sync(0xffffffffu, b1, o);
+        b2 += __shfl_xor_sync(0xffffffffu, b2, o);
+      }
+      if (live && j0 == 0) {
+        e.ln_out[static_cast<int64_t>(2 * blockIdx.y) * s.M + grow] = make_float2(a1, a2);
+        e.ln_out[static_cast<int64_t>(2 * blockIdx.y + 1) * s.M + grow] = make_float2(b1, b2);
+      }
+    }
+  };
 
   if (mode == 1 && region == 2) {
     // ------------------------------------------- direct, V^T of fused QKV
@@ -271,10 +381,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int t = grow - clip * e.t_len;
       uint8_t* stage = smem + (warp - 2) * (BN / 2 / 32) * 4096;
       int nbox = 0;
+      const float2 lnr = row_lnr(r);
 #pragma unroll 1
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
         float v[32];
         if (ok) tmem_ld32(trow + c, v);
+        if (ln_mode == 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaf(lnr.x, v[i], lnr.y * vec_s[c + i]);
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i] + bias_s[c + i], e.act);
         const int cc = n0 + c - 2 * e.qkv_d;  // column within V: head * 64 + dim
@@ -376,6 +491,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // Staging: this warp's boxes of 32 rows x 32 columns, 4 KB apart.
       uint8_t* stage = smem + (warp - 2) * (BN / 2 / 32) * 4096;
       int nbox = 0;
+      const float2 lnr = row_lnr(r);
+      float st1 = 0.f, st2 = 0.f;
 #pragma unroll 1
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
         float v[32];
@@ -403,6 +520,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = acc[i];
+        }
+        if (ln_mode == 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaf(lnr.x, v[i], lnr.y * vec_s[c + i]);
         }
         const int col = n0 + c;
         if (e.residual && grow < s.M) {
@@ -434,20 +555,37 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                  const float2 f = __half22float2(h[k]);
+                  float2 f = __half22float2(h[k]);
+                  if (ln_mode == 2) {
+                    const int cc = c + i + 2 * k;
+                    f.x = fmaf(fmaf(f.x, lnr.x, lnr.y), vec_s[cc], vec_s[BN + cc]);
+                    f.y = fmaf(fmaf(f.y, lnr.x, lnr.y), vec_s[cc + 1], vec_s[BN + cc + 1]);
+                  }
                   v[i + 2 * k] = apply_act(v[i + 2 * k] + bias_s[c + i + 2 * k], e.act) + f.x;
                   v[i + 2 * k + 1] = apply_act(v[i + 2 * k + 1] + bias_s[c + i + 2 * k + 1], e.act) + f.y;
                 }
               }
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + (i < nv ? __half2float(rp[i]) : 0.f);
+              for (int i = 0; i < 32; ++i) {
+                float f = i < nv ? __half2float(rp[i]) : 0.f;
+                if (ln_mode == 2) f = fmaf(fmaf(f, lnr.x, lnr.y), vec_s[c + i], vec_s[BN + c + i]);
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + f;
+              }
             }
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i] + bias_s[c + i], e.act);
+        }
+        if (e.ln_out) {  // this row's partial sums over this warp's half of the tile
+          const int nvs = min(32, s.N - col);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nvs) {
+              st1 += v[i];
+              st2 = fmaf(v[i], v[i], st2);
+            }
         }
         uint8_t* box = stage + nbox * 4096;
         if (e.out_f32) {
@@ -469,6 +607,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (lane == 0 && ok && col < s.N) tma_store_3d(om, box, col - ocol0, m0 + q * 32, bzb);
         ++nbox;
       }
+      if (e.ln_out && ok && grow < s.M)
+        e.ln_out[static_cast<int64_t>(2 * blockIdx.y + half) * s.M + grow] = make_float2(st1, st2);
       if (lane == 0) {
         bulk_commit_group();
         bulk_wait_all();
@@ -540,7 +680,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       } else {
         void* outp = region == 1 ? e.out_k : e.out;
         const int ocol0 = region > 0 ? region * e.qkv_d : 0;
-        const int total = nrows * C::ROW_CHUNKS;
+        const int total = e.ln_out ? 0 : nrows * C::ROW_CHUNKS;
+        if (e.ln_out) finish_rows_stats(r0, nrows, outp, ocol0, fetch);
 #pragma unroll 2
         for (int idx = et; idx < total; idx += kEpiThreads) {
           const int lr = idx / C::ROW_CHUNKS;
@@ -550,7 +691,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (grow >= s.M || col >= s.N) continue;
           const float4 v = fetch(lr, j);
           float x[4] = {v.x, v.y, v.z, v.w};
-          finish4(x, bias_s, 4 * j, grow, col, min(4, s.N - col), bzb, e, outp, ocol0, vec);
+          finish4(x, bias_s, vec_s, BN, row_lnr(r0 + lr), 4 * j, grow, col, min(4, s.N - col), bzb, e, outp,
+                  ocol0, vec);
         }
       }
     }
@@ -590,7 +732,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const int col = n0 + 4 * j;
           if (grow >= s.M || col >= s.N) continue;
           const float4 v = *reinterpret_cast<const float4*>(park + swz_off(C::ROW_CHUNKS, rr, j));
-          const float x[4] = {v.x, v.y, v.z, v.w};
+          float x[4] = {v.x, v.y, v.z, v.w};
+          if (ln_mode == 1) {
+            const float2 lnr = rowln_s[rr];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[i] = fmaf(lnr.x, x[i], lnr.y * vec_s[4 * j + i]);
+          }
           const int cc = col - 2 * e.qkv_d;
           const int clip = grow / e.t_len;
           const int t = grow - clip * e.t_len;
@@ -603,8 +750,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       } else {
         void* outp = region == 1 ? e.out_k : e.out;
         const int ocol0 = region > 0 ? region * e.qkv_d : 0;
+        if (e.ln_out)
+          finish_rows_stats(0, C::BM, outp, ocol0, [&](int rr, int j) -> float4 {
+            return *reinterpret_cast<const float4*>(park + swz_off(C::ROW_CHUNKS, rr, j));
+          });
 #pragma unroll 2
-        for (int idx = et; idx < total; idx += kEpiThreads) {
+        for (int idx = et; idx < (e.ln_out ? 0 : total); idx += kEpiThreads) {
           const int rr = idx / C::ROW_CHUNKS;
           const int j = idx - rr * C::ROW_CHUNKS;
           const int grow = m0 + rr;
@@ -612,7 +763,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (grow >= s.M || col >= s.N) continue;
           const float4 v = *reinterpret_cast<const float4*>(park + swz_off(C::ROW_CHUNKS, rr, j));
           float x[4] = {v.x, v.y, v.z, v.w};
-          finish4(x, bias_s, 4 * j, grow, col, min(4, s.N - col), bzb, e, outp, ocol0, vec);
+          finish4(x, bias_s, vec_s, BN, row_lnr(rr), 4 * j, grow, col, min(4, s.N - col), bzb, e, outp, ocol0,
+                  vec);
         }
       }
     }
@@ -725,6 +877,13 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   if (s.splits < 1 || s.splits > 8 || s.splits > s.K / 64 || (s.splits > 1 && s.batch != 1))
     return cudaErrorInvalidValue;
   if (e.qkv_d > 0 && (e.qkv_d % bn != 0 || s.N != 3 * e.qkv_d || e.t_len <= 0)) return cudaErrorInvalidValue;
+  // Folded LayerNorm: row statistics come as partial sums indexed by row
+  // (one clip batch); the normalised residual must be fp16.
+  const int ln_mode = e.ln_cfg & 255;
+  if (ln_mode > 2 || (ln_mode != 0 && (!e.ln_vec || !e.ln_in || (e.ln_cfg >> 8) < 1 || s.batch != 1)))
+    return cudaErrorInvalidValue;
+  if (ln_mode == 2 && (!e.residual || e.res_f32)) return cudaErrorInvalidValue;
+  if (e.ln_out && (s.batch != 1 || e.qkv_d > 0)) return cudaErrorInvalidValue;
   // Vector loads/stores need 16-byte aligned bases and 4-element-aligned rows.
   const int esz_out = e.out_f32 ? 4 : 2;
   const int esz_res = e.res_f32 ? 4 : 2;

@@ -131,6 +131,10 @@ struct LayerDev {
   __half *wqkv = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr;
   float *bqkv = nullptr, *bo = nullptr, *b1 = nullptr, *b2 = nullptr;
   float *ln1g = nullptr, *ln1b = nullptr, *ln2g = nullptr, *ln2b = nullptr;
+  // Folded post-norm LayerNorms (w2v_model::fold): column sums of the
+  // gamma-scaled QKV (layers >= 1) and FFN1 weights, and [gamma; beta] of the
+  // two norms for the residual epilogues.
+  float *cs_qkv = nullptr, *cs1 = nullptr, *gb1 = nullptr, *gb2 = nullptr;
 };
 
 struct Plan {
@@ -145,7 +149,7 @@ struct Plan {
   GemmShape projS;
   int projBN = 0;
   CUtensorMap posX;
-  CUtensorMap aH, aAO, aF;
+  CUtensorMap aH, aAO, aF, aRa;
   std::vector<CUtensorMap> qkvB, oB, f1B, f2B;
   GemmShape qkvS, oS, f1S, f2S;
   int qkvBN = 0, oBN = 0, f1BN = 0, f2BN = 0;
@@ -179,10 +183,21 @@ struct w2v_model {
   std::vector<LayerDev> L;
   __half* wlm = nullptr;
   float* blm = nullptr;
+  // Post-norm blocks with their LayerNorms folded into the GEMMs: the
+  // out-projection writes the un-normalised sum to `ra` and its partial row
+  // sums to stats_a, FFN2 writes its sum to `h` and partial sums to stats_f;
+  // the GEMMs that read those rows as A (FFN1, the next QKV, the lm_head)
+  // normalise in their epilogues with gamma-scaled weights (cs_* = column
+  // sums), and the residual epilogues of FFN2 / the next out-projection
+  // normalise their residual, all from the partial sums.
+  bool fold = false;
+  float* cs_lm = nullptr;
   // workspace
   __half *act_a = nullptr, *act_b = nullptr, *ln512 = nullptr, *x = nullptr, *h = nullptr, *q = nullptr,
          *k = nullptr, *vt = nullptr, *ao = nullptr, *f = nullptr;
   float* r = nullptr;
+  __half* ra = nullptr;
+  float2 *stats_a = nullptr, *stats_f = nullptr;
   double* gn_partial = nullptr;   // [max_batch][<=296][65] per-block window moments
   unsigned* gn_ticket = nullptr;  // [max_batch] last-block tickets (zero between calls)
   float2* gn_ss = nullptr;        // [max_batch][512] GroupNorm scale/shift
@@ -278,9 +293,20 @@ GemmEpilogue epi_proj(const w2v_model* m) {
   return e;
 }
 
+// Partial row sums stored by a GEMM of N columns in tiles of bn (two per
+// column tile), and the ln_cfg word of a GEMM that reads them.
+int ln_parts(int N, int bn) { return 2 * ((N + bn - 1) / bn); }
+int ln_cfg(int mode, int parts) { return mode | (parts << 8); }
+
 GemmEpilogue epi_qkv(const w2v_model* m, const Plan& p, int l) {
   GemmEpilogue e = epi_base(m);
   e.bias = m->L[l].bqkv;
+  if (m->fold && l > 0) {  // A = the previous block's un-normalised FFN sum
+    e.ln_cfg = ln_cfg(1, ln_parts(m->cfg.d_model, p.f2BN));
+    e.ln_vec = m->L[l].cs_qkv;
+    e.ln_in = m->stats_f;
+    e.ln_eps = m->cfg.ln_eps;
+  }
   e.out = m->q;
   e.ldo = m->cfg.d_model;
   e.qkv_d = m->cfg.d_model;
@@ -293,9 +319,27 @@ GemmEpilogue epi_qkv(const w2v_model* m, const Plan& p, int l) {
 }
 
 // out_proj (ffn = false) or FFN2 (ffn = true): bias + residual into the fp32 stream
-GemmEpilogue epi_resid(const w2v_model* m, int l, bool ffn) {
+GemmEpilogue epi_resid(const w2v_model* m, const Plan& p, int l, bool ffn) {
   GemmEpilogue e = epi_base(m);
   e.bias = ffn ? m->L[l].b2 : m->L[l].bo;
+  if (m->fold) {
+    // residual: LN_attn(ra) for FFN2; LN_ffn of the previous block (h) for the
+    // out-projection, or the materialised encoder LN output h in block 0
+    e.residual = ffn ? m->ra : m->h;
+    e.res_f32 = 0;
+    e.ldr = m->cfg.d_model;
+    if (ffn || l > 0) {
+      e.ln_cfg = ln_cfg(2, ln_parts(m->cfg.d_model, ffn ? p.oBN : p.f2BN));
+      e.ln_vec = ffn ? m->L[l].gb1 : m->L[l - 1].gb2;
+      e.ln_in = ffn ? m->stats_a : m->stats_f;
+      e.ln_eps = m->cfg.ln_eps;
+    }
+    e.ln_out = ffn ? m->stats_f : m->stats_a;  // partial sums of the new un-normalised rows
+    e.out = ffn ? m->h : m->ra;
+    e.out_f32 = 0;
+    e.ldo = m->cfg.d_model;
+    return e;
+  }
   if (m->cfg.stable_layer_norm) {
     e.residual = m->r;
     e.res_f32 = 1;
@@ -310,18 +354,30 @@ GemmEpilogue epi_resid(const w2v_model* m, int l, bool ffn) {
   return e;
 }
 
-GemmEpilogue epi_ffn1(const w2v_model* m, int l) {
+GemmEpilogue epi_ffn1(const w2v_model* m, const Plan& p, int l) {
   GemmEpilogue e = epi_base(m);
   e.bias = m->L[l].b1;
+  if (m->fold) {  // A = the un-normalised attention sum ra
+    e.ln_cfg = ln_cfg(1, ln_parts(m->cfg.d_model, p.oBN));
+    e.ln_vec = m->L[l].cs1;
+    e.ln_in = m->stats_a;
+    e.ln_eps = m->cfg.ln_eps;
+  }
   e.act = m->cfg.gelu_tanh ? 2 : 1;
   e.out = m->f;
   e.ldo = m->cfg.d_ffn;
   return e;
 }
 
-GemmEpilogue epi_lm(const w2v_model* m, float* logits) {
+GemmEpilogue epi_lm(const w2v_model* m, const Plan& p, float* logits) {
   GemmEpilogue e = epi_base(m);
   e.bias = m->blm;
+  if (m->fold) {  // A = the last block's un-normalised FFN sum
+    e.ln_cfg = ln_cfg(1, ln_parts(m->cfg.d_model, p.f2BN));
+    e.ln_vec = m->cs_lm;
+    e.ln_in = m->stats_f;
+    e.ln_eps = m->cfg.ln_eps;
+  }
   e.out = logits;
   e.out_f32 = 1;
   e.ldo = m->cfg.vocab;
@@ -453,6 +509,7 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   CUDA_OR(m, map_a(&p->aH, m->h, d, rows, d, 1, 0));
   CUDA_OR(m, map_a(&p->aAO, m->ao, d, rows, d, 1, 0));
   CUDA_OR(m, map_a(&p->aF, m->f, F, rows, F, 1, 0));
+  CUDA_OR(m, map_a(&p->aRa, m->ra, d, rows, d, 1, 0));
   auto shp = [&](int N, int K) {
     GemmShape s;
     s.M = rows; s.N = N; s.K = K; s.a_kwrap = K; s.batch = 1;
@@ -464,9 +521,10 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   p->f2S = shp(d, F);
   if (c.n_layers > 0) {
     int rc = tune_gemm(m, &p->qkvS, p->aH, m->L[0].wqkv, 3 * d, d, epi_qkv(m, *p, 0), d, &p->qkvBN);
-    if (rc == W2V_OK) rc = tune_gemm(m, &p->oS, p->aAO, m->L[0].wo, d, d, epi_resid(m, 0, false), 0, &p->oBN);
-    if (rc == W2V_OK) rc = tune_gemm(m, &p->f1S, p->aH, m->L[0].w1, F, d, epi_ffn1(m, 0), 0, &p->f1BN);
-    if (rc == W2V_OK) rc = tune_gemm(m, &p->f2S, p->aF, m->L[0].w2, d, F, epi_resid(m, 0, true), 0, &p->f2BN);
+    if (rc == W2V_OK) rc = tune_gemm(m, &p->oS, p->aAO, m->L[0].wo, d, d, epi_resid(m, *p, 0, false), 0, &p->oBN);
+    if (rc == W2V_OK)
+      rc = tune_gemm(m, &p->f1S, m->fold ? p->aRa : p->aH, m->L[0].w1, F, d, epi_ffn1(m, *p, 0), 0, &p->f1BN);
+    if (rc == W2V_OK) rc = tune_gemm(m, &p->f2S, p->aF, m->L[0].w2, d, F, epi_resid(m, *p, 0, true), 0, &p->f2BN);
     if (rc != W2V_OK) return rc;
   }
   p->qkvB.resize(c.n_layers);
@@ -492,7 +550,7 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   }
   p->lmS = shp(V, d);
   {
-    const int rc = tune_gemm(m, &p->lmS, p->aH, m->wlm, V, d, epi_lm(m, m->tune_logits), 0, &p->lmBN);
+    const int rc = tune_gemm(m, &p->lmS, p->aH, m->wlm, V, d, epi_lm(m, *p, m->tune_logits), 0, &p->lmBN);
     if (rc != W2V_OK) return rc;
   }
   // Tuning wrote garbage into the activation buffers: nothing reads them before
@@ -693,29 +751,31 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
     LAUNCH(W2V_K_ATTENTION, 4.0 * B * double(p.Tf) * p.Tf * D, 8.0 * R * D,
            launch_attention(p.attQ, p.attK, p.attVt, p.Tf, B, H, m->ao, m->err_word, st));
     {
-      const GemmEpilogue e = epi_resid(m, l, false);
+      const GemmEpilogue e = epi_resid(m, p, l, false);
       LAUNCH(W2V_K_OUT_GEMM, 2.0 * R * D * D, 2.0 * R * D + 2.0 * D * D + res_bytes + 4.0 * R * D,
              launch_gemm(p.aAO, p.oB[l], p.oS, p.oBN, e, m->err_word, st));
     }
-    LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes,
-           launch_layernorm(m->r, 1, m->h, rows, d, stable ? w.ln2g : w.ln1g, stable ? w.ln2b : w.ln1b, eps, 0, st));
+    if (!m->fold)
+      LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes,
+             launch_layernorm(m->r, 1, m->h, rows, d, stable ? w.ln2g : w.ln1g, stable ? w.ln2b : w.ln1b, eps, 0, st));
     {
-      const GemmEpilogue e = epi_ffn1(m, l);
+      const GemmEpilogue e = epi_ffn1(m, p, l);
       LAUNCH(W2V_K_FFN1_GEMM, 2.0 * R * FF * D, 2.0 * R * D + 2.0 * FF * D + 2.0 * R * FF,
-             launch_gemm(p.aH, p.f1B[l], p.f1S, p.f1BN, e, m->err_word, st));
+             launch_gemm(m->fold ? p.aRa : p.aH, p.f1B[l], p.f1S, p.f1BN, e, m->err_word, st));
     }
     {
-      const GemmEpilogue e = epi_resid(m, l, true);
+      const GemmEpilogue e = epi_resid(m, p, l, true);
       LAUNCH(W2V_K_FFN2_GEMM, 2.0 * R * D * FF, 2.0 * R * FF + 2.0 * D * FF + res_bytes + 4.0 * R * D,
              launch_gemm(p.aF, p.f2B[l], p.f2S, p.f2BN, e, m->err_word, st));
     }
-    if (!stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, w.ln2g, w.ln2b, eps, 0, st));
+    if (!stable && !m->fold)
+      LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, w.ln2g, w.ln2b, eps, 0, st));
   }
   if (stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, m->encg, m->encb, eps, 0, st));
 
   // --- CTC head, fp32 logits
   {
-    const GemmEpilogue e = epi_lm(m, logits);
+    const GemmEpilogue e = epi_lm(m, p, logits);
     LAUNCH(W2V_K_LM_HEAD, 2.0 * R * VV * D, 2.0 * R * D + 2.0 * VV * D + 4.0 * R * VV,
            launch_gemm(p.aH, p.lmB, p.lmS, p.lmBN, e, m->err_word, st));
   }
@@ -833,6 +893,31 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     fix.push_back({o, dst});
   };
 
+  // A gamma-scaled fp16 weight W[n][k] * g[k] ([N][K]), its bias plus W beta,
+  // and the column sums of the stored fp16 values (what the tensor core
+  // multiplies), both accumulated in double.
+  auto put_f16_folded = [&](void** wdst, void** bdst, void** csdst, int N, int K, auto&& wget, const float* bias,
+                            const float* g, const float* beta) {
+    put_f16(wdst, static_cast<size_t>(N) * K, [&](size_t i) { return wget(i) * g[i % K]; });
+    std::vector<float> cs(N), bp(N);
+    {
+      const __half* hp = reinterpret_cast<const __half*>(host.data() + fix.back().first);
+      for (int n = 0; n < N; ++n) {
+        double a = 0.0, b = bias[n];
+        for (int k = 0; k < K; ++k) {
+          a += static_cast<double>(__half2float(hp[static_cast<size_t>(n) * K + k]));
+          b += static_cast<double>(wget(static_cast<size_t>(n) * K + k)) * beta[k];
+        }
+        cs[n] = static_cast<float>(a);
+        bp[n] = static_cast<float>(b);
+      }
+    }
+    put_f32(bdst, bp.data(), N);
+    put_f32(csdst, cs.data(), N);
+  };
+  const bool fold = !c.stable_layer_norm && NL > 0 && !(std::getenv("W2V_LN_FOLD") && std::getenv("W2V_LN_FOLD")[0] == '0');
+  m->fold = fold;
+  auto lname = [&](int l, const char* what) { return "layers." + std::to_string(l) + "." + what; };
   put_f32(reinterpret_cast<void**>(&m->c0w), src("conv0.weight"), kC * 10);
   {
     const float* w = src("conv0.weight");  // [512][1][10]
@@ -894,15 +979,18 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     const float* wk = src(p + "attn.k.weight");
     const float* wv = src(p + "attn.v.weight");
     const size_t dd = static_cast<size_t>(d) * d;
-    put_f16(reinterpret_cast<void**>(&L.wqkv), 3 * dd, [&](size_t i) {
-      return i < dd ? wq[i] : (i < 2 * dd ? wk[i - dd] : wv[i - 2 * dd]);
-    });
-    {
-      size_t o = take(3 * d * 4);
-      std::memcpy(host.data() + o, src(p + "attn.q.bias"), d * 4);
-      std::memcpy(host.data() + o + d * 4, src(p + "attn.k.bias"), d * 4);
-      std::memcpy(host.data() + o + 2 * d * 4, src(p + "attn.v.bias"), d * 4);
-      fix.push_back({o, reinterpret_cast<void**>(&L.bqkv)});
+    auto wqkv = [&](size_t i) { return i < dd ? wq[i] : (i < 2 * dd ? wk[i - dd] : wv[i - 2 * dd]); };
+    std::vector<float> bqkv(3 * d);
+    std::memcpy(bqkv.data(), src(p + "attn.q.bias"), d * 4);
+    std::memcpy(bqkv.data() + d, src(p + "attn.k.bias"), d * 4);
+    std::memcpy(bqkv.data() + 2 * d, src(p + "attn.v.bias"), d * 4);
+    if (fold && l > 0) {  // input: LN_ffn of block l - 1
+      put_f16_folded(reinterpret_cast<void**>(&L.wqkv), reinterpret_cast<void**>(&L.bqkv),
+                     reinterpret_cast<void**>(&L.cs_qkv), 3 * d, d, wqkv, bqkv.data(),
+                     src(lname(l - 1, "ffn_norm.weight")), src(lname(l - 1, "ffn_norm.bias")));
+    } else {
+      put_f16(reinterpret_cast<void**>(&L.wqkv), 3 * dd, wqkv);
+      put_f32(reinterpret_cast<void**>(&L.bqkv), bqkv.data(), 3 * d);
     }
     const float* wo = src(p + "attn.out.weight");
     put_f16(reinterpret_cast<void**>(&L.wo), dd, [&](size_t i) { return wo[i]; });
@@ -910,8 +998,21 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     put_f32(reinterpret_cast<void**>(&L.ln1g), src(p + "attn_norm.weight"), d);
     put_f32(reinterpret_cast<void**>(&L.ln1b), src(p + "attn_norm.bias"), d);
     const float* w1 = src(p + "ffn.in.weight");
-    put_f16(reinterpret_cast<void**>(&L.w1), static_cast<size_t>(F) * d, [&](size_t i) { return w1[i]; });
-    put_f32(reinterpret_cast<void**>(&L.b1), src(p + "ffn.in.bias"), F);
+    if (fold) {  // input: LN_attn of this block
+      put_f16_folded(reinterpret_cast<void**>(&L.w1), reinterpret_cast<void**>(&L.b1), reinterpret_cast<void**>(&L.cs1),
+                     F, d, [&](size_t i) { return w1[i]; }, src(p + "ffn.in.bias"), src(p + "attn_norm.weight"),
+                     src(p + "attn_norm.bias"));
+      std::vector<float> gb(2 * d);
+      std::memcpy(gb.data(), src(p + "attn_norm.weight"), d * 4);
+      std::memcpy(gb.data() + d, src(p + "attn_norm.bias"), d * 4);
+      put_f32(reinterpret_cast<void**>(&L.gb1), gb.data(), 2 * d);
+      std::memcpy(gb.data(), src(p + "ffn_norm.weight"), d * 4);
+      std::memcpy(gb.data() + d, src(p + "ffn_norm.bias"), d * 4);
+      put_f32(reinterpret_cast<void**>(&L.gb2), gb.data(), 2 * d);
+    } else {
+      put_f16(reinterpret_cast<void**>(&L.w1), static_cast<size_t>(F) * d, [&](size_t i) { return w1[i]; });
+      put_f32(reinterpret_cast<void**>(&L.b1), src(p + "ffn.in.bias"), F);
+    }
     const float* w2 = src(p + "ffn.out.weight");
     put_f16(reinterpret_cast<void**>(&L.w2), static_cast<size_t>(F) * d, [&](size_t i) { return w2[i]; });
     put_f32(reinterpret_cast<void**>(&L.b2), src(p + "ffn.out.bias"), d);
@@ -920,10 +1021,17 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   }
   {
     const float* w = src("lm_head.weight");
-    put_f16(reinterpret_cast<void**>(&m->wlm), static_cast<size_t>(V) * d, [&](size_t i) { return w[i]; });
+    if (fold) {  // input: LN_ffn of the last block
+      put_f16_folded(reinterpret_cast<void**>(&m->wlm), reinterpret_cast<void**>(&m->blm),
+                     reinterpret_cast<void**>(&m->cs_lm), V, d, [&](size_t i) { return w[i]; }, src("lm_head.bias"),
+                     src(lname(NL - 1, "ffn_norm.weight")), src(lname(NL - 1, "ffn_norm.bias")));
+    } else {
+      put_f16(reinterpret_cast<void**>(&m->wlm), static_cast<size_t>(V) * d, [&](size_t i) { return w[i]; });
+      put_f32(reinterpret_cast<void**>(&m->blm), src("lm_head.bias"), V);
+    }
   }
-  put_f32(reinterpret_cast<void**>(&m->blm), src("lm_head.bias"), V);
   (void)put_f32_zero;
+  (void)put_f16_folded;
 
   const size_t wbytes = round_up(cursor, 256);
   if (cudaMalloc(&m->wmem, wbytes) != cudaSuccess) return W2V_ENOMEM;
@@ -959,6 +1067,11 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   wtake(reinterpret_cast<void**>(&m->ao), rows * d * 2);
   wtake(reinterpret_cast<void**>(&m->f), rows * F * 2);
   wtake(reinterpret_cast<void**>(&m->r), rows * d * 4);
+  wtake(reinterpret_cast<void**>(&m->ra), rows * d * 2);
+  // partial row sums of the folded LayerNorms: up to 2 per 32 columns
+  const size_t ln_parts_max = 2 * static_cast<size_t>((d + 31) / 32);
+  wtake(reinterpret_cast<void**>(&m->stats_a), ln_parts_max * rows * 8);
+  wtake(reinterpret_cast<void**>(&m->stats_f), ln_parts_max * rows * 8);
   wtake(reinterpret_cast<void**>(&m->gn_partial), static_cast<size_t>(B) * 296 * 65 * 8);
   wtake(reinterpret_cast<void**>(&m->gn_ticket), static_cast<size_t>(B) * 4);
   wtake(reinterpret_cast<void**>(&m->gn_ss), static_cast<size_t>(B) * 512 * 8);
@@ -1178,7 +1291,16 @@ extern "C" int w2v_debug_read(w2v_model* m, int which, void* dst_dev, size_t dst
     case 0: srcp = m->act_a; sz = rows * kC * 2; break;
     case 1: srcp = m->x; sz = rows * m->cfg.d_model * 2; break;
     case 2: srcp = m->r; sz = rows * m->cfg.d_model * 4; break;
-    case 3: srcp = m->h; sz = rows * m->cfg.d_model * 2; break;
+    case 3:
+      srcp = m->h;
+      sz = rows * m->cfg.d_model * 2;
+      if (m->fold) {  // h holds the last block's un-normalised sum: apply its LN into ra
+        const LayerDev& w = m->L[m->cfg.n_layers - 1];
+        CUDA_OR(m, launch_layernorm(m->h, 0, m->ra, p->rows, m->cfg.d_model, w.ln2g, w.ln2b, m->cfg.ln_eps, 0,
+                                    static_cast<cudaStream_t>(stream)));
+        srcp = m->ra;
+      }
+      break;
     default: return fail(m, W2V_EINVAL, "unknown buffer %d", which);
   }
   if (bytes) *bytes = sz;

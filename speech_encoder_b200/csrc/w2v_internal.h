@@ -44,19 +44,21 @@ cudaError_t make_tmap(CUtensorMap* out, const void* base, int rank, const uint64
 // K block starting at k is fetched from column (k % a_kwrap) of row
 // (m0 + k / a_kwrap) — a_kwrap = K for an ordinary matrix, or the width of a
 // pair of frames for the stride-2 conv layers (implicit GEMM).
-// The kernel's own copy of the epilogue arguments.  It is kept exactly this
-// size: growing the by-value parameter block of the GEMM kernel (even by
-// fields it never reads) measured 30-50 % slower mainloops on B200, so
+// The kernel's own copy of the epilogue arguments.  Its size is capped: the
+// GEMM kernel's by-value parameter block (5 tensor maps, GemmDims, this struct
+// and 16 bytes more) measured the same speed up to 808 bytes and 30-50 %
+// slower launches from 816 bytes on (direct TMA-store epilogues), so this
+// struct stays at or below 128 bytes (static_assert in k_gemm.cu) and
 // host-only additions go into GemmEpilogue below.
 struct GemmEpiArgs {
   const float* bias = nullptr;     // [N] or null
   const void* residual = nullptr;  // [rows, ldr], fp16 or fp32 per res_f32, or null
   int res_f32 = 0;
-  int64_t ldr = 0;
+  int ldr = 0;
   int64_t res_batch_stride = 0;    // elements between batch items
   void* out = nullptr;             // [rows, ldo], fp16 or fp32 per out_f32
   int out_f32 = 0;
-  int64_t ldo = 0;
+  int ldo = 0;
   int64_t out_batch_stride = 0;
   int act = 0;                     // 0 none, 1 exact GELU, 2 tanh GELU
   // QKV split: when qkv_d > 0 the N = 3*qkv_d columns go to three places:
@@ -68,6 +70,23 @@ struct GemmEpiArgs {
   int t_pad = 0;
   int n_heads = 0;
   int t_len = 0;                   // frames per clip (rows are clip-major)
+  // LayerNorm folded into the GEMMs (post-norm encoder blocks).  Row
+  // statistics travel as partial sums: a GEMM with ln_out set stores, for each
+  // output row and each half of each column tile (2 N / BN partials), the sum
+  // and the sum of squares of its final values at ln_out[p * M + row].  A GEMM
+  // reading such rows gets (ln_cfg >> 8) partials per row at ln_in and
+  //  ln_mode 1 (ln_cfg & 255): A holds the un-normalised rows x and B holds
+  //    W diag(gamma); the epilogue turns the accumulator into LN(x) W^T + bias
+  //    as rstd * (acc - mean * ln_vec[n]) + bias[n], with ln_vec = the column
+  //    sums of the scaled weight and bias = the original bias + W beta;
+  //  ln_mode 2: the fp16 residual is un-normalised; the epilogue adds
+  //    LN(residual) = (res - mean) * rstd * gamma[n] + beta[n], with
+  //    gamma = ln_vec[n], beta = ln_vec[N + n].
+  int ln_cfg = 0;
+  const float* ln_vec = nullptr;
+  const float2* ln_in = nullptr;
+  float2* ln_out = nullptr;
+  float ln_eps = 0.f;
 };
 
 struct GemmEpilogue : GemmEpiArgs {

@@ -47,6 +47,21 @@ def test_small_model_matches_oracle(layout, n):
     model.close()
 
 
+@pytest.mark.parametrize("layout", ["group_post", "group_post_tanh"])
+def test_unfolded_post_norm_matches_oracle(layout, monkeypatch):
+    # W2V_LN_FOLD=0 at create time keeps the post-norm LayerNorms as their own
+    # kernels (the folded form is the default and is covered above).
+    monkeypatch.setenv("W2V_LN_FOLD", "0")
+    shape = S.small_shape(**LAYOUTS[layout])
+    model = U.make_model(shape, max_samples=48000, max_batch=2, seed=3, affine_noise=True)
+    pcm = np.stack([S.synth_pcm(41234, 21), S.synth_pcm(41234, 22)])
+    got = _run(model, pcm)
+    for b in range(2):
+        ref = U.oracle_logits(shape, pcm[b], seed=3, affine_noise=True)
+        U.compare_logits(got[b], ref, f"{layout} unfolded clip {b}")
+    model.close()
+
+
 def test_small_model_stages_match_oracle():
     # Intermediate activations (conv encoder output, projection, encoder output)
     # of a 0-layer and a 2-layer model, to localise any disagreement.
