@@ -287,12 +287,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int grow = m0 + et;
         float2 f = make_float2(1.f, 0.f);
         if (grow < s.M) {
+          // loads issued eight at a time (independent L2 reads), added in
+          // partial order
           const int parts = e.ln_cfg >> 8;
           float s1 = 0.f, s2 = 0.f;
-          for (int p = 0; p < parts; ++p) {
-            const float2 t = e.ln_in[static_cast<int64_t>(p) * s.M + grow];
-            s1 += t.x;
-            s2 += t.y;
+          for (int p0 = 0; p0 < parts; p0 += 8) {
+            float2 t[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              t[k] = p0 + k < parts ? e.ln_in[static_cast<int64_t>(p0 + k) * s.M + grow] : make_float2(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              s1 += t[k].x;
+              s2 += t[k].y;
+            }
           }
           const float inv = 1.f / static_cast<float>(ln_mode == 1 ? s.K : s.N);
           const float mean = s1 * inv;
