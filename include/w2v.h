@@ -96,6 +96,38 @@ int w2v_weight_num_entries(const w2v_config* cfg);
 int w2v_weight_entry(const w2v_config* cfg, int index, char* name, size_t name_len, int* ndim, int64_t shape[3],
                      size_t* offset);
 
+/* Packs a single-file safetensors checkpoint into the float32 weight blob
+ * (blob: host float[n_floats], n_floats == w2v_weight_count(cfg); owned by the
+ * caller).  Host only, no device work.  Format: 8-byte little-endian header
+ * length, JSON header {name: {dtype, shape, data_offsets}}, raw data; dtypes
+ * F32, F16, BF16, F64 (converted to float32).  Each manifest entry is looked
+ * up under its own name, then under the checkpoint module path, with or
+ * without a "wav2vec2." prefix:
+ *   conv{i}.weight/.bias    feature_extractor.conv_layers.{i}.conv.weight/.bias
+ *   conv{i}.norm.*          feature_extractor.conv_layers.{i}.layer_norm.*
+ *   fp.norm.* / fp.proj.*   feature_projection.layer_norm.* / .projection.*
+ *   pos_conv.*              encoder.pos_conv_embed.conv.*
+ *   enc.norm.*              encoder.layer_norm.*
+ *   layers.{l}.attn.{q,k,v,out}.*  encoder.layers.{l}.attention.{q,k,v,out}_proj.*
+ *   layers.{l}.attn_norm.*  encoder.layers.{l}.layer_norm.*
+ *   layers.{l}.ffn.in.* / ffn.out.*  encoder.layers.{l}.feed_forward.
+ *                           intermediate_dense.* / output_dense.*
+ *   layers.{l}.ffn_norm.*   encoder.layers.{l}.final_layer_norm.*
+ *   lm_head.*               lm_head.*
+ * The positional conv weight may be stored weight-normalised, as weight_g /
+ * weight_v or parametrizations.weight.original0 / original1 (g, v): it is
+ * folded to g * v / ||v||, the norm (float64) taken over the axes where g has
+ * extent 1 (the pages' "pos_conv weight-norm folded into a static weight").
+ * Errors: W2V_EINVAL (unreadable or malformed file, missing tensor,
+ * unsupported dtype, bad config), W2V_ESHAPE (a tensor's shape differs from
+ * the manifest, or n_floats is wrong); err (err_len bytes, may be NULL)
+ * receives a message naming the tensor. */
+int w2v_pack_safetensors(const char* path, const w2v_config* cfg, float* blob, size_t n_floats, char* err,
+                         size_t err_len);
+/* w2v_pack_safetensors then w2v_create; *out is NULL on error. */
+int w2v_create_from_safetensors(const char* path, const w2v_config* cfg, w2v_model** out, char* err,
+                                size_t err_len);
+
 /* Creates a model on the current CUDA device: validates cfg, converts the host
  * float32 blob (n_floats == w2v_weight_count(cfg)) to the device layouts (fp16
  * matrices, repacked conv and positional-conv weights, fp32 vectors) and

@@ -59,6 +59,9 @@ def lib() -> ctypes.CDLL:
         "w2v_weight_entry": (I, [ctypes.POINTER(w2v_config), I, ctypes.c_char_p, SZ, ctypes.POINTER(I),
                                  ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(SZ)]),
         "w2v_create": (I, [ctypes.POINTER(w2v_config), VP, SZ, ctypes.POINTER(VP)]),
+        "w2v_pack_safetensors": (I, [ctypes.c_char_p, ctypes.POINTER(w2v_config), VP, SZ, ctypes.c_char_p, SZ]),
+        "w2v_create_from_safetensors": (I, [ctypes.c_char_p, ctypes.POINTER(w2v_config), ctypes.POINTER(VP),
+                                            ctypes.c_char_p, SZ]),
         "w2v_forward": (I, [VP, VP, I, I, VP, VP]),
         "w2v_ctc_greedy": (I, [VP, VP, I, I, I, VP, VP, VP]),
         "w2v_sync": (I, [VP, VP]),
@@ -135,6 +138,25 @@ def w2v_weight_manifest(cfg: w2v_config):
             raise W2VError(rc, "w2v_weight_entry")
         out.append((buf.value.decode(), tuple(int(shp[j]) for j in range(nd.value)), int(off.value)))
     return out
+
+
+def w2v_pack_safetensors(path: str, cfg: w2v_config) -> np.ndarray:
+    """The float32 weight blob of a single-file safetensors checkpoint (host only)."""
+    blob = np.empty(w2v_weight_count(cfg), dtype=np.float32)
+    err = ctypes.create_string_buffer(512)
+    rc = lib().w2v_pack_safetensors(os.fsencode(path), ctypes.byref(cfg), blob.ctypes.data, blob.size, err, 512)
+    if rc != W2V_OK:
+        raise W2VError(rc, f"w2v_pack_safetensors: {err.value.decode(errors='replace')}")
+    return blob
+
+
+def w2v_create_from_safetensors(path: str, cfg: w2v_config) -> int:
+    h = VP()
+    err = ctypes.create_string_buffer(512)
+    rc = lib().w2v_create_from_safetensors(os.fsencode(path), ctypes.byref(cfg), ctypes.byref(h), err, 512)
+    if rc != W2V_OK:
+        raise W2VError(rc, f"w2v_create_from_safetensors: {err.value.decode(errors='replace')}")
+    return h.value
 
 
 def _check(rc: int, handle=None, what: str = ""):
@@ -256,10 +278,18 @@ def w2v_op_wait_probe(err, limit_ns: int, stream=None) -> int:
 class Model:
     """Owns one w2v_model handle.  Tensors are torch CUDA tensors."""
 
-    def __init__(self, shape, blob: np.ndarray, max_samples: int, max_batch: int = 1, use_cuda_graph: bool = True):
+    def __init__(self, shape, blob: Optional[np.ndarray], max_samples: int, max_batch: int = 1,
+                 use_cuda_graph: bool = True, safetensors: Optional[str] = None):
+        """Weights from `blob` (float32, manifest order) or, with blob None,
+        from the single-file safetensors checkpoint at `safetensors`."""
         self.shape = shape
         self.cfg = make_config(shape, max_samples, max_batch, use_cuda_graph)
-        self.handle = w2v_create(self.cfg, blob)
+        if blob is None:
+            if safetensors is None:
+                raise ValueError("give a weight blob or a safetensors path")
+            self.handle = w2v_create_from_safetensors(safetensors, self.cfg)
+        else:
+            self.handle = w2v_create(self.cfg, blob)
 
     def forward(self, pcm, logits=None, stream=None):
         """pcm: float32 CUDA tensor [batch, n].  Returns logits [batch, T, vocab]."""

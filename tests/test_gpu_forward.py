@@ -258,3 +258,43 @@ def test_plan_file_pins_the_gemm_choices_across_models(tmp_path, monkeypatch):
     with pytest.raises(B.W2VError):
         _run(m3, pcm)
     m3.close()
+
+
+def test_model_from_safetensors_equals_model_from_blob(tmp_path, monkeypatch):
+    # The loader's blob (checkpoint names, fp16 tensors, weight-normalised
+    # positional conv) gives the same logits as the same blob handed to
+    # w2v_create directly (the analytic plan on both sides: bit for bit).
+    from test_safetensors import _fixture, write_safetensors
+    monkeypatch.setenv("W2V_AUTOTUNE", "0")
+    shape = S.small_shape()
+    cfg = B.make_config(shape, 48000, 1)
+    tensors, want, _ = _fixture(cfg)
+    # keep the random checkpoint in a numerically sane range for a forward
+    tensors = {k: (dt, (a * 0.05).astype(a.dtype) if dt != "BF16" else a) for k, (dt, a) in tensors.items()}
+    path = tmp_path / "model.safetensors"
+    write_safetensors(path, tensors)
+    blob = B.w2v_pack_safetensors(str(path), cfg)
+    m1 = B.Model(shape, None, 48000, 1, safetensors=str(path))
+    m2 = B.Model(shape, blob, 48000, 1)
+    pcm = S.synth_pcm(30000, 9)[None]
+    a = _run(m1, pcm)
+    b = _run(m2, pcm)
+    assert np.isfinite(a).all()
+    assert np.array_equal(a, b)
+    m1.close()
+    m2.close()
+
+
+def test_sharded_transcription_single_rank_matches_per_clip_decode():
+    from speech_encoder_b200.shard import transcribe_clips
+    shape = S.small_shape()
+    model = U.make_model(shape, 48000, 1)
+    clips = [S.synth_pcm(n, 30 + i) for i, n in enumerate((41234, 16000, 30000))]
+    got = transcribe_clips(model, clips, rank=0, world=1)
+    for c, tok in zip(clips, got):
+        logits = _run(model, c[None])
+        T = O.num_frames(len(c))
+        # the same tokens as the oracle's decode of this model's own logits
+        ref = np.asarray(O.ctc_greedy(logits[0], T, shape.blank_id), dtype=np.int32)
+        assert np.array_equal(tok, ref)
+    model.close()
