@@ -96,6 +96,21 @@ int w2v_weight_num_entries(const w2v_config* cfg);
 int w2v_weight_entry(const w2v_config* cfg, int index, char* name, size_t name_len, int* ndim, int64_t shape[3],
                      size_t* offset);
 
+/* Raw PCM to forward-pass windows (the fixed-window form of the pages: a clip
+ * zero-padded to the window and decoded over its valid frames).  pcm_dev:
+ * float32 [n_samples] on the device, one clip at the model's sample rate.
+ * It is cut into w2v_num_windows(n_samples, window) = ceil(n_samples / window)
+ * consecutive windows; window w holds samples [w*window, w*window + valid_w),
+ * valid_w = min(window, n_samples - w*window), normalised over those valid
+ * samples to (x - mean) / sqrt(var + 1e-7) (biased variance), then zeros up
+ * to `window`.  out_dev: float32 [num_windows][window] on the device, owned by
+ * the caller, ready for w2v_forward(batch = num_windows, n_samples = window);
+ * decode window w over w2v_num_frames(valid_w) frames.  Asynchronous on
+ * `stream`.  Errors: W2V_EINVAL (null pointer), W2V_ESHAPE (n_samples or
+ * window < 1), W2V_ECUDA (launch failure). */
+int w2v_num_windows(int n_samples, int window);
+int w2v_window_pcm(const float* pcm_dev, int n_samples, int window, float* out_dev, void* stream);
+
 /* Packs a single-file safetensors checkpoint into the float32 weight blob
  * (blob: host float[n_floats], n_floats == w2v_weight_count(cfg); owned by the
  * caller).  Host only, no device work.  Format: 8-byte little-endian header

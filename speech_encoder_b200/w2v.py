@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         "w2v_weight_entry": (I, [ctypes.POINTER(w2v_config), I, ctypes.c_char_p, SZ, ctypes.POINTER(I),
                                  ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(SZ)]),
         "w2v_create": (I, [ctypes.POINTER(w2v_config), VP, SZ, ctypes.POINTER(VP)]),
+        "w2v_num_windows": (I, [I, I]),
+        "w2v_window_pcm": (I, [VP, I, I, VP, VP]),
         "w2v_pack_safetensors": (I, [ctypes.c_char_p, ctypes.POINTER(w2v_config), VP, SZ, ctypes.c_char_p, SZ]),
         "w2v_create_from_safetensors": (I, [ctypes.c_char_p, ctypes.POINTER(w2v_config), ctypes.POINTER(VP),
                                             ctypes.c_char_p, SZ]),
@@ -137,6 +139,22 @@ def w2v_weight_manifest(cfg: w2v_config):
         if rc:
             raise W2VError(rc, "w2v_weight_entry")
         out.append((buf.value.decode(), tuple(int(shp[j]) for j in range(nd.value)), int(off.value)))
+    return out
+
+
+def w2v_num_windows(n_samples: int, window: int) -> int:
+    return lib().w2v_num_windows(int(n_samples), int(window))
+
+
+def w2v_window_pcm(pcm, window: int, out=None, stream=None):
+    """pcm: float32 CUDA tensor [n] of one raw clip.  Returns the normalised,
+    zero-padded windows [num_windows, window] (see include/w2v.h)."""
+    import torch
+    n = pcm.numel()
+    nw = w2v_num_windows(n, window)
+    if out is None:
+        out = torch.empty((nw, window), dtype=torch.float32, device=pcm.device)
+    _check(lib().w2v_window_pcm(_ptr(pcm), int(n), int(window), _ptr(out), _stream(stream)), None, "w2v_window_pcm")
     return out
 
 

@@ -100,3 +100,11 @@ def test_create_without_gpu_reports_device_error():
     L = B.lib()
     h = ctypes.c_void_p()
     assert L.w2v_create(ctypes.byref(cfg), blob.ctypes.data, blob.size, ctypes.byref(h)) == B.W2V_EDEVICE
+
+
+def test_num_windows_host_arithmetic():
+    assert B.w2v_num_windows(256000, 256000) == 1
+    assert B.w2v_num_windows(256001, 256000) == 2
+    assert B.w2v_num_windows(1, 160000) == 1
+    assert B.w2v_num_windows(0, 160000) == 0
+    assert B.w2v_num_windows(10, 0) == 0

@@ -167,3 +167,22 @@ def test_bounded_wait_reports_instead_of_hanging():
     assert B.w2v_op_gemm(A, A[:64], 128, 64, 64, None, None, 0, out, 1, 0, err2) == 0
     torch.cuda.synchronize()
     assert int(err2.item()) == 0 and float(out[0, 0]) == 64.0
+
+
+@pytest.mark.parametrize("n,window", [(130000, 48000), (96000, 48000), (48001, 48000), (1000, 48000), (7, 3)])
+def test_window_pcm_matches_per_window_normalisation(n, window):
+    # raw (un-normalised) PCM: offset sinusoids plus noise
+    rng = np.random.default_rng(n)
+    t = np.arange(n)
+    raw = (0.3 * np.sin(2 * np.pi * 440 * t / 16000) + 0.2 * np.sin(2 * np.pi * 97 * t / 16000 + 1.0) + 0.5 +
+           0.05 * rng.standard_normal(n)).astype(np.float32)
+    nw = B.w2v_num_windows(n, window)
+    assert nw == -(-n // window)
+    got = B.w2v_window_pcm(torch.from_numpy(raw).cuda(), window).cpu().numpy()
+    assert got.shape == (nw, window)
+    for w in range(nw):
+        seg = raw[w * window:(w + 1) * window].astype(np.float64)
+        ref = np.zeros(window)
+        ref[:len(seg)] = (seg - seg.mean()) / np.sqrt(seg.var() + 1e-7)
+        np.testing.assert_allclose(got[w], ref, atol=3e-5, rtol=0)
+        assert (got[w, len(seg):] == 0).all()
