@@ -136,7 +136,8 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, cons
   }
 }
 
-// mode: 0 generic, 1 direct (TMA store), 2 split-K
+// mode: 0 generic, 1 direct (TMA store), 2 split-K through distributed shared
+// memory, 3 split-K through an L2 scratch (with the direct stores)
 // SPLIT: the instantiation for split-K launches (modes 2 and 3); the other one
 // runs modes 0 and 1 only.
 template <int BN, bool SPLIT>

@@ -322,15 +322,6 @@ __device__ __forceinline__ void st_dsmem_f4(uint32_t addr, float4 v) {
                : "memory");
 }
 
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start while the
 // previous kernel on the stream is still running.  pdl_wait() blocks until that
@@ -399,12 +390,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
 }
 
 // GELU, exact form x * Phi(x) through the CUDA erff, or the tanh form.
@@ -479,9 +464,5 @@ __device__ __forceinline__ float apply_act(float x, int act) {
   if (act == 2) return gelu_tanh(x);
   return x;
 }
-
-__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
-
-__device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace w2v
