@@ -200,3 +200,41 @@ def test_missing_tensor_wrong_shape_and_bad_files_are_refused(cfg, tmp_path):
     write_safetensors(path, t4)
     with pytest.raises(B.W2VError, match="unsupported dtype"):
         B.w2v_pack_safetensors(str(path), cfg)
+
+
+@pytest.mark.parametrize("layout", ["group_post", "layer_stable"])
+def test_loader_on_a_transformers_checkpoint_reproduces_its_logits(tmp_path, layout):
+    # An independent pin of the name map and the weight-norm fold: a randomly
+    # initialised transformers Wav2Vec2ForCTC (its own parameter names, its
+    # positional conv under weight normalisation, g perturbed away from ||v||)
+    # saved as safetensors, packed by the loader, run through the oracle,
+    # gives the module's own logits.
+    torch = pytest.importorskip("torch")
+    from oracle import w2v_oracle as O
+    from test_oracle_pins import _hf_model
+    group = layout.startswith("group")
+    shape = S.small_shape(conv_norm="group" if group else "layer", stable=not group, conv_bias=not group)
+    torch.manual_seed(3)
+    model = _hf_model(shape)
+    sd = model.state_dict()
+    gk = [k for k in sd if k.endswith("parametrizations.weight.original0") or k.endswith("weight_g")]
+    assert len(gk) == 1
+    with torch.no_grad():
+        sd[gk[0]].mul_(1.0 + 0.5 * torch.rand_like(sd[gk[0]]))
+        for k, v in sd.items():  # make biases and norm affines non-trivial too
+            if k.endswith("bias") or "layer_norm" in k:
+                v.add_(0.1 * torch.randn_like(v))
+    model.load_state_dict(sd)
+    tensors = {k: ("F32", v.float().numpy()) for k, v in sd.items()}
+    path = tmp_path / "model.safetensors"
+    write_safetensors(path, tensors)
+    B.lib()
+    cfg = B.make_config(shape, 48000, 1)
+    blob = B.w2v_pack_safetensors(str(path), cfg)
+    W = {name: blob[off:off + int(np.prod(shp))].reshape(shp) for name, shp, off in B.w2v_weight_manifest(cfg)}
+    pcm = S.synth_pcm(6000, 12)
+    with torch.no_grad():
+        ref = model(torch.tensor(pcm.astype(np.float64))[None]).logits[0].numpy()
+    got = O.forward(shape, O.to_f64(W), pcm)
+    # the checkpoint went through fp32: agreement to fp32 rounding of the weights
+    assert np.abs(got - ref).max() < 1e-4 * max(1.0, np.abs(ref).max())
