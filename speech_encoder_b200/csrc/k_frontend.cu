@@ -80,8 +80,18 @@ gn_moments_kernel(const float* pcm, int n, int t0, const float* __restrict__ w0,
     const double* pb = partial + static_cast<int64_t>(b) * gridDim.x * kMom;
     const int mi = threadIdx.x % kMom, grp = threadIdx.x / kMom;  // 260 slots > 256 threads: grp 3 has 61
     if (grp < 4) {
+      // loads issued eight at a time (independent L2 reads), added in block order
       double sum = 0.0;
-      for (unsigned k = grp; k < gridDim.x; k += 4) sum += __ldcg(pb + k * kMom + mi);
+      for (unsigned k0 = grp; k0 < gridDim.x; k0 += 32) {
+        double v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const unsigned k = k0 + 4u * u;
+          v[u] = k < gridDim.x ? __ldcg(pb + k * kMom + mi) : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sum += v[u];
+      }
       part[grp][mi] = sum;
     }
     __syncthreads();
@@ -89,8 +99,18 @@ gn_moments_kernel(const float* pcm, int n, int t0, const float* __restrict__ w0,
       // threads 195..255 cover moments 0..60 of group 3; moments 61..64 of
       // group 3 were not visited: add their blocks here.
       double s3 = threadIdx.x < 256 - 3 * kMom ? part[3][threadIdx.x] : 0.0;
-      if (threadIdx.x >= 256 - 3 * kMom)
-        for (unsigned k = 3; k < gridDim.x; k += 4) s3 += __ldcg(pb + k * kMom + threadIdx.x);
+      if (threadIdx.x >= 256 - 3 * kMom) {
+        for (unsigned k0 = 3; k0 < gridDim.x; k0 += 32) {
+          double v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const unsigned k = k0 + 4u * u;
+            v[u] = k < gridDim.x ? __ldcg(pb + k * kMom + threadIdx.x) : 0.0;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) s3 += v[u];
+        }
+      }
       mom[threadIdx.x] = ((part[0][threadIdx.x] + part[1][threadIdx.x]) + part[2][threadIdx.x]) + s3;
     }
   }
