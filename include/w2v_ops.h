@@ -50,6 +50,19 @@ int w2v_op_layernorm(const void* x, int in_f32, void* y, int rows, int cols, con
  * that the timeout path reports instead of hanging. */
 int w2v_op_wait_probe(int* err_dev, uint64_t limit_ns, void* stream);
 
+/* Host only: the weights of LayerNorm(x) -> Linear(W, bias) folded so that
+ * the GEMM runs on the un-normalised x (the post-norm LayerNorm fold of
+ * w2v_create).  W: float [N][K] (PyTorch Linear layout), bias: float [N] or
+ * NULL, gamma / beta: float [K].  Outputs (caller-owned host arrays):
+ * w_fp16 [N][K] = fp16 bits of W[n][k] * gamma[k] (product in float32, rounded
+ * to nearest even); bias_out [N] = bias[n] + sum_k W[n][k] beta[k] and
+ * colsum_out [N] = sum_k fp16 value of w_fp16[n][k], both accumulated in
+ * float64.  Then LN(x) W^T + bias = rstd (x W''^T - mean * colsum) + bias_out
+ * for every row x with mean and rstd = 1 / sqrt(var + eps), up to the fp16
+ * rounding of W''.  Errors: W2V_EINVAL (null pointer), W2V_ESHAPE (N or K < 1). */
+int w2v_fold_layernorm_linear(const float* W, int N, int K, const float* bias, const float* gamma, const float* beta,
+                              uint16_t* w_fp16, float* bias_out, float* colsum_out);
+
 #ifdef __cplusplus
 }
 #endif

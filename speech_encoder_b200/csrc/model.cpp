@@ -798,6 +798,25 @@ __half to_half(float v) { return __float2half_rn(v); }
 
 // =================================================================== C ABI
 
+extern "C" int w2v_fold_layernorm_linear(const float* W, int N, int K, const float* bias, const float* gamma,
+                                         const float* beta, uint16_t* w_fp16, float* bias_out, float* colsum_out) {
+  if (!W || !gamma || !beta || !w_fp16 || !bias_out || !colsum_out) return W2V_EINVAL;
+  if (N < 1 || K < 1) return W2V_ESHAPE;
+  for (int n = 0; n < N; ++n) {
+    double a = 0.0, b = bias ? static_cast<double>(bias[n]) : 0.0;
+    for (int k = 0; k < K; ++k) {
+      const size_t i = static_cast<size_t>(n) * K + k;
+      const __half h = to_half(W[i] * gamma[k]);
+      std::memcpy(&w_fp16[i], &h, 2);
+      a += static_cast<double>(__half2float(h));
+      b += static_cast<double>(W[i]) * beta[k];
+    }
+    colsum_out[n] = static_cast<float>(a);
+    bias_out[n] = static_cast<float>(b);
+  }
+  return W2V_OK;
+}
+
 extern "C" int w2v_num_frames(int n_samples) { return n_samples >= 400 ? (n_samples - 400) / 320 + 1 : 0; }
 
 extern "C" size_t w2v_weight_count(const w2v_config* cfg) {
@@ -896,22 +915,13 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   // A gamma-scaled fp16 weight W[n][k] * g[k] ([N][K]), its bias plus W beta,
   // and the column sums of the stored fp16 values (what the tensor core
   // multiplies), both accumulated in double.
-  auto put_f16_folded = [&](void** wdst, void** bdst, void** csdst, int N, int K, auto&& wget, const float* bias,
+  auto put_f16_folded = [&](void** wdst, void** bdst, void** csdst, int N, int K, const float* W, const float* bias,
                             const float* g, const float* beta) {
-    put_f16(wdst, static_cast<size_t>(N) * K, [&](size_t i) { return wget(i) * g[i % K]; });
+    const size_t o = take(static_cast<size_t>(N) * K * 2);
+    fix.push_back({o, wdst});
     std::vector<float> cs(N), bp(N);
-    {
-      const __half* hp = reinterpret_cast<const __half*>(host.data() + fix.back().first);
-      for (int n = 0; n < N; ++n) {
-        double a = 0.0, b = bias[n];
-        for (int k = 0; k < K; ++k) {
-          a += static_cast<double>(__half2float(hp[static_cast<size_t>(n) * K + k]));
-          b += static_cast<double>(wget(static_cast<size_t>(n) * K + k)) * beta[k];
-        }
-        cs[n] = static_cast<float>(a);
-        bp[n] = static_cast<float>(b);
-      }
-    }
+    w2v_fold_layernorm_linear(W, N, K, bias, g, beta, reinterpret_cast<uint16_t*>(host.data() + o), bp.data(),
+                              cs.data());
     put_f32(bdst, bp.data(), N);
     put_f32(csdst, cs.data(), N);
   };
@@ -985,8 +995,10 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     std::memcpy(bqkv.data() + d, src(p + "attn.k.bias"), d * 4);
     std::memcpy(bqkv.data() + 2 * d, src(p + "attn.v.bias"), d * 4);
     if (fold && l > 0) {  // input: LN_ffn of block l - 1
+      std::vector<float> wcat(3 * dd);
+      for (size_t i = 0; i < 3 * dd; ++i) wcat[i] = wqkv(i);
       put_f16_folded(reinterpret_cast<void**>(&L.wqkv), reinterpret_cast<void**>(&L.bqkv),
-                     reinterpret_cast<void**>(&L.cs_qkv), 3 * d, d, wqkv, bqkv.data(),
+                     reinterpret_cast<void**>(&L.cs_qkv), 3 * d, d, wcat.data(), bqkv.data(),
                      src(lname(l - 1, "ffn_norm.weight")), src(lname(l - 1, "ffn_norm.bias")));
     } else {
       put_f16(reinterpret_cast<void**>(&L.wqkv), 3 * dd, wqkv);
@@ -1000,8 +1012,7 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     const float* w1 = src(p + "ffn.in.weight");
     if (fold) {  // input: LN_attn of this block
       put_f16_folded(reinterpret_cast<void**>(&L.w1), reinterpret_cast<void**>(&L.b1), reinterpret_cast<void**>(&L.cs1),
-                     F, d, [&](size_t i) { return w1[i]; }, src(p + "ffn.in.bias"), src(p + "attn_norm.weight"),
-                     src(p + "attn_norm.bias"));
+                     F, d, w1, src(p + "ffn.in.bias"), src(p + "attn_norm.weight"), src(p + "attn_norm.bias"));
       std::vector<float> gb(2 * d);
       std::memcpy(gb.data(), src(p + "attn_norm.weight"), d * 4);
       std::memcpy(gb.data() + d, src(p + "attn_norm.bias"), d * 4);
@@ -1023,7 +1034,7 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     const float* w = src("lm_head.weight");
     if (fold) {  // input: LN_ffn of the last block
       put_f16_folded(reinterpret_cast<void**>(&m->wlm), reinterpret_cast<void**>(&m->blm),
-                     reinterpret_cast<void**>(&m->cs_lm), V, d, [&](size_t i) { return w[i]; }, src("lm_head.bias"),
+                     reinterpret_cast<void**>(&m->cs_lm), V, d, w, src("lm_head.bias"),
                      src(lname(NL - 1, "ffn_norm.weight")), src(lname(NL - 1, "ffn_norm.bias")));
     } else {
       put_f16(reinterpret_cast<void**>(&m->wlm), static_cast<size_t>(V) * d, [&](size_t i) { return w[i]; });

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         "w2v_op_attention": (I, [VP, VP, VP, VP, I, I, I, I, VP, VP]),
         "w2v_op_layernorm": (I, [VP, I, VP, I, I, VP, VP, ctypes.c_float, I, VP]),
         "w2v_op_wait_probe": (I, [VP, ctypes.c_uint64, VP]),
+        "w2v_fold_layernorm_linear": (I, [VP, I, I, VP, VP, VP, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -287,6 +288,23 @@ def w2v_op_attention(q, k, vt, out, batch, T, H, t_pad, err, stream=None) -> int
 def w2v_op_layernorm(x, in_f32, y, rows, cols, gamma, beta, eps, act, stream=None) -> int:
     return lib().w2v_op_layernorm(_ptr(x), in_f32, _ptr(y), rows, cols, _ptr(gamma), _ptr(beta), float(eps), act,
                                   _stream(stream))
+
+
+def w2v_fold_layernorm_linear(W: np.ndarray, bias, gamma: np.ndarray, beta: np.ndarray):
+    """Host-side LayerNorm -> Linear fold (see include/w2v_ops.h): returns
+    (fp16 weight W diag(gamma), bias + W beta, column sums of the fp16 weight)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    bt = np.ascontiguousarray(beta, dtype=np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    wf = np.empty((N, K), dtype=np.float16)
+    bo = np.empty(N, dtype=np.float32)
+    cs = np.empty(N, dtype=np.float32)
+    rc = lib().w2v_fold_layernorm_linear(W.ctypes.data, N, K, None if b is None else b.ctypes.data, g.ctypes.data,
+                                         bt.ctypes.data, wf.ctypes.data, bo.ctypes.data, cs.ctypes.data)
+    _check(rc, None, "w2v_fold_layernorm_linear")
+    return wf, bo, cs
 
 
 def w2v_op_wait_probe(err, limit_ns: int, stream=None) -> int:
