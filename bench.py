@@ -319,6 +319,10 @@ def oracle_sample(seconds_budget: float):
     return runs * AUDIO_SEC / wall, runs, wall
 
 
+# timed oracle work of the reference arm (seconds); tests shorten it
+REFERENCE_BUDGET_S = float(os.environ.get("W2V_BENCH_REFERENCE_BUDGET_S", "90"))
+
+
 def run_reference(args, world):
     from oracle import w2v_oracle as O
     from synth import inputs as S
@@ -330,22 +334,30 @@ def run_reference(args, world):
         z = O.forward(w.model, W64, pcm)
         O.ctc_greedy(z, z.shape[0], 0)
 
-    for _ in range(args.warmup):
-        step()
+    # The oracle needs seconds per step: one warm-up step (BLAS thread start-up
+    # is its only warm-up effect), then as many of the requested timed steps
+    # as fit in REFERENCE_BUDGET_S, at least one, so that the run stays within
+    # a few minutes whatever --steps / --warmup ask for.
+    t0 = time.perf_counter()
+    step()
+    est = time.perf_counter() - t0
+    warmup = 1
+    steps = max(1, min(args.steps, int(REFERENCE_BUDGET_S // max(est, 1e-3))))
     times = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         t0 = time.perf_counter()
         step()
         times.append(time.perf_counter() - t0)
     total = sum(times)
-    value = args.steps * AUDIO_SEC / total
+    value = steps * AUDIO_SEC / total
     cores = blas_threads()
+    sample = (f"{steps} timed step(s) of the {args.steps} requested (+{warmup} warm-up), each the full 16 s clip: "
+              f"fp64 numpy forward + greedy CTC")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+            "steps": steps, "warmup": warmup, "ms_per_step": 1000 * total / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded sinusoids + noise PCM, random-init weights)", "config": config_dict(world),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": "the full 16 s clip per step: fp64 numpy forward + greedy CTC"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
