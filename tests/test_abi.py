@@ -108,3 +108,38 @@ def test_num_windows_host_arithmetic():
     assert B.w2v_num_windows(1, 160000) == 1
     assert B.w2v_num_windows(0, 160000) == 0
     assert B.w2v_num_windows(10, 0) == 0
+
+
+def _prototypes():
+    """name -> parameter count of every w2v_* function declared in include/*.h."""
+    protos = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for m in re.finditer(r"\b(w2v_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", txt, flags=re.S):
+            params = m.group(2).strip()
+            protos[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_signatures_match_the_headers():
+    # every entry point the binding types must take as many arguments as the
+    # header declares (guards the ctypes table against drift)
+    protos = _prototypes()
+    L = B.lib()
+    typed = [n for n in protos if getattr(getattr(L, n), "argtypes", None) is not None]
+    assert len(typed) >= 20
+    for n in typed:
+        assert len(getattr(L, n).argtypes) == protos[n], (n, len(getattr(L, n).argtypes), protos[n])
+
+
+def test_host_side_argument_checks_need_no_device():
+    L = B.lib()
+    assert L.w2v_window_pcm(None, 10, 4, None, None) == B.W2V_EINVAL
+    buf = ctypes.create_string_buffer(64)
+    cfg = B.make_config(S.small_shape(), 48000, 1)
+    h = ctypes.c_void_p()
+    assert L.w2v_create_from_safetensors(b"/nonexistent/model.safetensors", ctypes.byref(cfg), ctypes.byref(h),
+                                         buf, 64) == B.W2V_EINVAL
+    assert h.value is None and b"cannot open" in buf.value
+    blob = np.zeros(B.w2v_weight_count(cfg), dtype=np.float32)
+    assert L.w2v_pack_safetensors(b"x", ctypes.byref(cfg), blob.ctypes.data, blob.size - 1, buf, 64) == B.W2V_ESHAPE
