@@ -192,12 +192,16 @@ int w2v_ctc_greedy(w2v_model* m, const float* logits_dev, int batch, int T, int 
  * merged, blank_id dropped; tokens_dev int32 [batch][t_valid] (clip b's
  * tokens first), n_tokens_dev int32 [batch].  The caller owns logits and
  * outputs; the per-frame argmax scratch is a fixed array of
- * W2V_CTC_STATIC_MAX_ROWS int32 in the library's device memory, which every
- * GPU that loads the library holds until the process exits.
+ * W2V_CTC_STATIC_MAX_ROWS int32 (4 MiB) in the library's device memory.
  *  - batch * T must not exceed W2V_CTC_STATIC_MAX_ROWS (1048576 frames, e.g.
  *    16 clips of 30 s): larger requests return W2V_ESHAPE and launch nothing.
- *  - The first call on a device looks up the array's device address with that
- *    device current; make that first call before any stream capture.
+ *  - CUDA loads device code lazily by default, so the array is placed on a
+ *    GPU by the first call of this entry point on that device: that first
+ *    call may allocate device memory and block like any module load.  Make
+ *    it at start-up (a call with t_valid = 0 is enough), before any stream
+ *    capture; the GPU then holds the 4 MiB until the process exits.  Every
+ *    call looks the array's address up for the current device, which
+ *    allocates nothing once the array is loaded.
  *  - All calls share the one array, so calls whose work overlaps on the GPU
  *    (on different streams, or from different threads) race and may return
  *    wrong tokens; serialise them.  Nothing in the array needs clearing: each

@@ -50,6 +50,24 @@ int w2v_op_layernorm(const void* x, int in_f32, void* y, int rows, int cols, con
  * that the timeout path reports instead of hanging. */
 int w2v_op_wait_probe(int* err_dev, uint64_t limit_ns, void* stream);
 
+/* Element-wise evaluation of the library's device math helpers, so that each
+ * hand-written approximation can be checked against its stated error bound on
+ * its own (inside the model they only show through the logits).  x_dev, y_dev:
+ * float [n] on the device.  fn:
+ *   0  y = 2^(c x + b) through fp16x2 rounding of the argument and the fp16x2
+ *      exponent instruction (the softmax's exponent-unit path);
+ *   1  the same through the cubic on the FMA/ALU pipes (the softmax's
+ *      polynomial path; argument clamped to [-15, 8], results below 2^-15
+ *      flush to zero);
+ *   2  tanh-GELU of a pair with the fp16x2 exponent (conv/FFN epilogues);
+ *   3  tanh-GELU, fp32 sigmoid form;  4  exact GELU (erff);
+ *   5  CUDA's exp2f(c x + b), the comparison point for 0 and 1.
+ * Forms 0-2 take elements 2i and 2i+1 as one pair: n must be even.  The
+ * softmax is the LiteRT discussion's plain SDPA and the tanh-GELU its first GPU
+ * rewrite.  Errors: W2V_EINVAL (null pointer, unknown fn), W2V_ESHAPE (n < 0,
+ * or odd for a pair form), W2V_ECUDA (launch failure). */
+int w2v_op_pointwise(int fn, const float* x_dev, int n, float c, float b, float* y_dev, void* stream);
+
 /* Host only: the weights of LayerNorm(x) -> Linear(W, bias) folded so that
  * the GEMM runs on the un-normalised x (the post-norm LayerNorm fold of
  * w2v_create).  W: float [N][K] (PyTorch Linear layout), bias: float [N] or

@@ -27,12 +27,20 @@ what a library matmul does internally.  Sources for each step:
 * Attention is plain SDPA with no mask: LiteRT discussion, fourth bullet.
 * lm_head, per-frame argmax and CTC collapse: README, "Results" (CTC ids).
 
-Readings where the pages are silent (each also listed in the design notes):
-eps 1e-5 with biased variance for every norm; for post-norm the encoder LN sits
-once after the positional-conv add and before block 1; the positional conv pads
-64 zeros on each side and drops the last output frame; attention scale
-1/sqrt(64); argmax ties go to the lowest index; collapse merges repeats first
-and then drops blank.
+Readings taken where the pages are silent:
+* eps 1e-5 with biased variance for every norm;
+* for post-norm the encoder LN sits once after the positional-conv add and
+  before block 1 (the pages state only that stable checkpoints apply it after
+  the blocks);
+* the positional conv pads 64 zeros on each side, drops the last output frame
+  (even kernel), has a bias, and is followed by GELU and the residual add;
+* the tanh-GELU variant replaces every GELU of the model (conv encoder,
+  positional conv, FFN);
+* attention scale 1/sqrt(64), biases on q/k/v/out, no mask, no dropout;
+* GroupNorm statistics of a zero-padded fixed window are taken over all of its
+  conv-0 frames, zeros included;
+* argmax ties go to the lowest index; collapse merges repeats first and then
+  drops blank (id 0, also for the 2341-token head).
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, invariants, brute-force loops on tiny shapes, torch fp64

@@ -10,13 +10,17 @@
 // application forbids allocations after start-up.  They pass the logits and
 // the output buffers; the library supplies the scratch.
 //
-// The array is a file-scope __device__ variable, so every GPU that loads this
-// library holds W2V_CTC_STATIC_MAX_ROWS int32 values (4 MiB) until the process
-// exits.  On the host its name is only a stand-in for the symbol, not a device
-// address: the address is looked up with cudaGetSymbolAddress once per device,
-// with that device current, on the first call made on that device.
-#include <mutex>
-
+// The array is a file-scope __device__ variable.  CUDA loads a library's
+// device code lazily by default (CUDA_MODULE_LOADING=LAZY), so the array is
+// placed on a GPU when its module is first used there: by the first call of
+// this entry point on that device.  That first call may therefore allocate
+// and block like any module load; make it at start-up, before any stream
+// capture.  From then on the GPU holds W2V_CTC_STATIC_MAX_ROWS int32 values
+// (4 MiB) until the process exits.  On the host the array's name is only a
+// stand-in for the symbol, not a device address: every call looks the address
+// up with cudaGetSymbolAddress, with the caller's device current (after the
+// module is loaded this allocates nothing), so a device reset or a new primary
+// context never leaves a stale address behind.
 #include "w2v.h"
 #include "w2v_internal.h"
 
@@ -26,24 +30,12 @@ static __device__ __align__(256) int32_t g_ctc_static_ids[W2V_CTC_STATIC_MAX_ROW
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-int32_t* g_ids_addr[kMaxDevices] = {};
-
-// Device address of g_ctc_static_ids on the current device (looked up once).
+// Device address of g_ctc_static_ids on the current device.
 cudaError_t static_ids_address(int32_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_ctc_static_ids);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_ids_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_ctc_static_ids);
-    if (e != cudaSuccess) return e;
-    g_ids_addr[dev] = static_cast<int32_t*>(p);
-  }
-  *out = g_ids_addr[dev];
+  *out = static_cast<int32_t*>(p);
   return cudaSuccess;
 }
 

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         "w2v_op_attention": (I, [VP, VP, VP, VP, I, I, I, I, VP, VP]),
         "w2v_op_layernorm": (I, [VP, I, VP, I, I, VP, VP, ctypes.c_float, I, VP]),
         "w2v_op_wait_probe": (I, [VP, ctypes.c_uint64, VP]),
+        "w2v_op_pointwise": (I, [I, VP, I, ctypes.c_float, ctypes.c_float, VP, VP]),
         "w2v_fold_layernorm_linear": (I, [VP, I, I, VP, VP, VP, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
@@ -305,6 +306,10 @@ def w2v_fold_layernorm_linear(W: np.ndarray, bias, gamma: np.ndarray, beta: np.n
                                          bt.ctypes.data, wf.ctypes.data, bo.ctypes.data, cs.ctypes.data)
     _check(rc, None, "w2v_fold_layernorm_linear")
     return wf, bo, cs
+
+
+def w2v_op_pointwise(fn: int, x, y, c: float = 1.0, b: float = 0.0, stream=None) -> int:
+    return lib().w2v_op_pointwise(int(fn), _ptr(x), int(x.numel()), float(c), float(b), _ptr(y), _stream(stream))
 
 
 def w2v_op_wait_probe(err, limit_ns: int, stream=None) -> int:

@@ -62,6 +62,44 @@ def test_unfolded_post_norm_matches_oracle(layout, monkeypatch):
     model.close()
 
 
+@pytest.mark.parametrize("offset", [10.0, 20.0])
+def test_folded_layernorm_on_rows_with_a_large_mean(offset, monkeypatch):
+    # Post-norm blocks whose attention and FFN LayerNorms have beta = offset +
+    # N(0, 0.1): every row entering a folded LayerNorm (the un-normalised sum
+    # after the FFN residual, read by the next QKV and the lm_head; the one
+    # after the attention residual of blocks >= 1, read by FFN1) then has a
+    # mean of about `offset` against a standard deviation of about 1.  The
+    # fold computes those rows' statistics from sums and sums of squares and
+    # applies the mean through the weight column sums; the unfolded path
+    # (W2V_LN_FOLD=0) normalises two-pass in a separate kernel.  Both must
+    # meet the oracle bar, and the fold must not be markedly worse.
+    shape = S.small_shape()
+    W = dict(S.init_weights(shape, 3, affine_noise=True))
+    rng = np.random.default_rng(77)
+    for l in range(shape.n_layers):
+        for nm in ("attn_norm.bias", "ffn_norm.bias"):
+            key = f"layers.{l}.{nm}"
+            W[key] = (offset + rng.normal(0.0, 0.1, W[key].shape)).astype(np.float32)
+    blob = S.pack_blob(shape, W)
+    pcm = np.stack([S.synth_pcm(41234, 21), S.synth_pcm(41234, 22)])
+    W64 = O.to_f64(W)
+    refs = [O.forward(shape, W64, pcm[b]) for b in range(2)]
+    from speech_encoder_b200 import w2v as Bm
+    folded = Bm.Model(shape, blob, max_samples=48000, max_batch=2)
+    got_f = _run(folded, pcm)
+    folded.close()
+    monkeypatch.setenv("W2V_LN_FOLD", "0")
+    plain = Bm.Model(shape, blob, max_samples=48000, max_batch=2)
+    got_u = _run(plain, pcm)
+    plain.close()
+    for b in range(2):
+        sf = U.compare_logits(got_f[b], refs[b], f"offset {offset} folded clip {b}")
+        su = U.compare_logits(got_u[b], refs[b], f"offset {offset} unfolded clip {b}")
+        print("large-mean LN fold", offset, b, sf, su)
+        assert sf["max_abs"] <= 2.0 * su["max_abs"] + 5e-3, (sf, su)
+        assert sf["mean_abs"] <= 2.0 * su["mean_abs"] + 5e-4, (sf, su)
+
+
 def test_small_model_stages_match_oracle():
     # Intermediate activations (conv encoder output, projection, encoder output)
     # of a 0-layer and a 2-layer model, to localise any disagreement.
@@ -198,14 +236,13 @@ def test_c1_base_16s_window_tanh_and_padded_short_clip():
     m.close()
 
 
-def test_c2_base_batch16_sampled_clips():
+def test_c2_base_batch16_every_clip():
+    # all 16 clips of the batch against the oracle, clip by clip
     w, m = _config_model("c2", max_batch=16)
     got = _run(m, w.calls[0][0])
     assert got.shape == (16, 499, 32)
-    for clip in (0, 7, 15):
+    for clip in range(16):
         print("c2", clip, U.compare_logits(got[clip], U.oracle_workload_clip("c2", 0, clip), f"c2 clip {clip}"))
-    # every clip's logits are finite and clips differ (no cross-clip mixing by construction of seeds)
-    assert np.isfinite(got).all()
     m.close()
 
 
@@ -217,15 +254,15 @@ def test_c3_large_stable_16s():
     m.close()
 
 
-def test_c4_large_true_length_clips_sampled():
+def test_c4_large_true_length_every_clip():
+    # each of the 8 true-length clips (its own length, its own launch plan)
+    # against the oracle
     w, m = _config_model("c4", max_samples=320000)
     lens = [p.shape[1] for p, _ in w.calls]
     outs = [_run(m, p) for p, _ in w.calls]
     for i, o in enumerate(outs):
         assert o.shape == (1, O.num_frames(lens[i]), 2341)
-        assert np.isfinite(o).all()
-    for i in (int(np.argmin(lens)), int(np.argmax(lens))):
-        print("c4", i, lens[i], U.compare_logits(outs[i][0], U.oracle_workload_clip("c4", i, 0), f"c4 clip {i}"))
+        print("c4", i, lens[i], U.compare_logits(o[0], U.oracle_workload_clip("c4", i, 0), f"c4 clip {i}"))
     m.close()
 
 

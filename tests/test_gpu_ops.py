@@ -186,3 +186,77 @@ def test_window_pcm_matches_per_window_normalisation(n, window):
         ref[:len(seg)] = (seg - seg.mean()) / np.sqrt(seg.var() + 1e-7)
         np.testing.assert_allclose(got[w], ref, atol=3e-5, rtol=0)
         assert (got[w, len(seg):] == 0).all()
+
+
+# ------------------------------------------------- device math approximations
+def _pointwise(fn, x, c=1.0, b=0.0):
+    xt = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+    y = torch.empty_like(xt)
+    assert B.w2v_op_pointwise(fn, xt, y, c, b) == B.W2V_OK
+    torch.cuda.synchronize()
+    return y.cpu().numpy().astype(np.float64)
+
+
+def test_softmax_exponentials_meet_their_error_bounds():
+    # Both exponential paths of the attention softmax round the argument
+    # x = c s + b (fp32 FMA) to fp16 first; what they then compute is 2^x16.
+    # Exponent-unit path: an fp16 result, relative error <= 2^-9 (a few fp16
+    # ulps: the hardware approximation plus the result rounding).
+    # Polynomial path: relative error <= 1e-3 (the stated 7e-4 of the cubic
+    # with fp16 Horner steps, plus the fp16 result rounding) for x16 >= -14;
+    # below that (x16 in [-15, -14)) it may flush to 0: absolute <= 2^-14.
+    # Over the whole range the softmax feeds it, [-15, 8].
+    s = np.concatenate([np.linspace(-15.0, 8.0, 400001), [-15.0, -14.5, -14.0, -1e-4, 0.0, 1e-4, 7.99, 8.0]])
+    s = s[: len(s) // 2 * 2]
+    for c, b in ((1.0, 0.0), (1.4426950408889634 * 0.125, -3.0)):
+        x32 = (s.astype(np.float64) * np.float32(c) + np.float32(b)).astype(np.float32)
+        x16 = x32.astype(np.float16).astype(np.float64)
+        keep = (x16 >= -15.0) & (x16 <= 8.0)
+        exact = np.exp2(x16)
+        mufu = _pointwise(0, s, c, b)
+        poly = _pointwise(1, s, c, b)
+        cuda = _pointwise(5, s, c, b)
+        normal = keep & (x16 >= -14.0)
+        rel_m = np.abs(mufu - exact)[normal] / exact[normal]
+        rel_p = np.abs(poly - exact)[normal] / exact[normal]
+        assert rel_m.max() <= 2.0 ** -9, rel_m.max()
+        assert rel_p.max() <= 1e-3, (rel_p.max(), x16[normal][np.argmax(rel_p)])
+        tiny = keep & (x16 < -14.0)
+        if tiny.any():
+            assert np.abs(poly - exact)[tiny].max() <= 2.0 ** -14
+        # against CUDA's own exp2f of the unrounded argument: the difference is
+        # the argument rounding (<= ln 2 * half an fp16 ulp of x, relative)
+        # plus the bounds above
+        ulp = np.spacing(np.abs(x16).astype(np.float16)).astype(np.float64)
+        arg = np.log(2.0) * 0.5 * ulp
+        sel = normal & (cuda > 0)
+        assert np.all(np.abs(poly - cuda)[sel] / cuda[sel] <= 1e-3 + arg[sel] * 1.01 + 1e-7)
+
+
+def test_gelu_approximations_meet_their_error_bounds():
+    x = np.linspace(-12.0, 12.0, 240002)
+    xd = x.astype(np.float32).astype(np.float64)
+    exact_tanh = O.gelu_tanh(xd)
+    exact_erf = O.gelu(xd)
+    # fp32 sigmoid form (ex2.approx + rcp.approx, relative ~2^-21 each)
+    g32 = _pointwise(3, x)
+    assert np.all(np.abs(g32 - exact_tanh) <= 1e-6 * np.abs(exact_tanh) + 1e-7 * np.abs(xd) + 1e-30)
+    # exact GELU through erff
+    gerf = _pointwise(4, x)
+    assert np.all(np.abs(gerf - exact_erf) <= 2e-6 * np.abs(xd) + 1e-7)
+    # packed form: the exponent argument w = -2 sqrt(2/pi) log2(e) (x + 0.044715 x^3)
+    # is rounded to fp16 and 2^w is an fp16 result, so e = 2^w carries a
+    # relative error of at most (2^-11 |w| ln 2 + 2^-10); x / (1 + e) passes it
+    # on scaled by e / (1 + e).
+    g2 = _pointwise(2, x)
+    k2 = -2.0 * 0.7978845608028654 * 1.4426950408889634
+    w = k2 * (xd + 0.044715 * xd ** 3)
+    e = np.exp2(np.minimum(w, 1000.0))
+    frac = np.where(np.isinf(e), 1.0, e / (1.0 + e))
+    bound = (2.0 ** -11 * np.abs(w) * np.log(2.0) + 2.0 ** -10) * frac * np.abs(exact_tanh) * 1.25 + 1e-6 * np.abs(xd) + 1e-7
+    over = np.abs(g2 - exact_tanh) > bound
+    # where 2^w overflows fp16 (w >= 16) the packed form returns x / inf = -0:
+    # the true value there is below 2^-16 |x|
+    overflow = w >= 15.9  # fp16 rounding of w reaches 16 within this margin
+    assert not np.any(over & ~overflow), (xd[over & ~overflow][:5], g2[over & ~overflow][:5])
+    assert np.all(np.abs(g2[overflow] - exact_tanh[overflow]) <= 2.0 ** -15 * np.abs(xd[overflow]))

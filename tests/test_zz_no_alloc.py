@@ -67,6 +67,36 @@ def test_static_ctc_matches_existing_entry_point_on_two_calls_in_a_row():
     model.close()
 
 
+def test_static_ctc_allocates_nothing_after_its_first_call():
+    # After the first call on a device has loaded the library's array, a call
+    # changes the device's free memory by nothing: the scratch is the fixed
+    # array, not an allocation.  Also covers a blank id other than 0 (against
+    # the existing entry point of a model whose blank id is 5) and an empty
+    # valid range (every count 0).
+    V = 32
+    shape = S.small_shape(vocab=V).with_(blank_id=5)
+    model = B.Model(shape, S.pack_blob(shape, S.init_weights(shape, 0)), max_samples=320000, max_batch=4)
+    lg = _logits(3, 3, 640, V)
+    out_a = _decode_static(lg, 3, 640, V, 640, blank=5)  # first call: loads the array if not yet loaded
+    torch.cuda.synchronize()
+    tok = torch.full((3, 640), -7, dtype=torch.int32, device="cuda")
+    nt = torch.full((3,), -7, dtype=torch.int32, device="cuda")
+    tok0 = torch.full((3, 1), -7, dtype=torch.int32, device="cuda")
+    nt0 = torch.full((3,), -7, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    assert B.w2v_ctc_greedy_static(lg, 3, 640, V, 640, 5, tok, nt) == B.W2V_OK
+    assert B.w2v_ctc_greedy_static(lg, 3, 640, V, 0, 5, tok0, nt0) == B.W2V_OK
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before, (free_before, free_after)
+    _same((tok, nt), out_a)
+    _same((tok, nt), _decode_existing(model, lg, 3, 640, 640))
+    assert nt0.cpu().tolist() == [0, 0, 0]
+    model.sync()
+    model.close()
+
+
 def test_static_ctc_rejects_sizes_beyond_its_array():
     lg = torch.zeros(16, dtype=torch.float32, device="cuda")
     tok = torch.zeros(16, dtype=torch.int32, device="cuda")
