@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="measure only the headline workload (c1), not c0/c2/c3/c4")
     return ap.parse_args()
 
 
@@ -290,12 +292,142 @@ def run_ours(args, rank, world, local_rank):
            "d2h_bytes_per_step": int(tok_host.numel() * 4 + nt_host.numel() * 4)}
     model.close()
 
+    # ---- the other workloads (one GPU only; the headline stays c1)
+    extra = {}
+    if world == 1 and not args.no_extra_configs:
+        for name in ("c0", "c2", "c3", "c4"):
+            extra[name] = measure_workload(name, max(5, min(args.steps, 20)), args.warmup, tc_peak, dev, flush)
+
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded sinusoids + noise PCM, random-init weights)",
            "config": config_dict(world), "frames_per_s": value / AUDIO_SEC * T, "roofline": roofline,
            "tensor_frac_all_contractions": tensor_frac_all, "kernels": kernels, "e2e": e2e,
            "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+    if extra:
+        out["other_workloads"] = extra
+    return out
+
+
+# ------------------------------------------------------- the other workloads
+OTHER_WORKLOADS = {
+    "c0": "wav2vec2-base shape, random-init, batch 1, 1 s (16000 samples -> 49 frames), exact GELU",
+    "c2": "wav2vec2-base shape, random-init, 16 clips of 10 s (160000 samples -> 499 frames each), exact GELU",
+    "c3": "wav2vec2-large stable-layer-norm shape, random-init, batch 1, 16 s (256000 samples -> 799 frames), "
+          "2341-token head, exact GELU",
+    "c4": "wav2vec2-large stable-layer-norm shape, random-init, 8 true-length clips of 2-20 s (seeded lengths), "
+          "exact GELU",
+}
+
+
+def contraction_flops(shape, n):
+    """Algorithmic FLOPs (2 per multiply-add) of the tensor-core work of one
+    clip of n samples: conv layers, projection, positional conv, QKV,
+    attention, out-projection, FFN and CTC head."""
+    ks, ss = (10, 3, 3, 3, 3, 2, 2), (5, 2, 2, 2, 2, 2, 2)
+    T, t, fl = [], n, 0.0
+    for k, st in zip(ks, ss):
+        t = (t - k) // st + 1 if t >= k else 0
+        T.append(t)
+    fl += 2.0 * 10 * 512 * T[0]
+    for i in range(1, 7):
+        fl += 2.0 * T[i] * 512 * 512 * ks[i]
+    Tf, d, F, V = T[6], shape.d_model, shape.d_ffn, shape.vocab
+    fl += 2.0 * Tf * d * 512 + 2.0 * Tf * d * (d // 16) * 128
+    fl += shape.n_layers * (2.0 * Tf * 3 * d * d + 4.0 * Tf * Tf * d + 2.0 * Tf * d * d + 4.0 * Tf * F * d)
+    fl += 2.0 * Tf * V * d
+    return fl
+
+
+def measure_workload(name, steps, warmup, tc_peak, dev, flush, cpu_budget_s=10.0):
+    """Device throughput of one of the other workloads (the clips as the
+    workload lists them, forward + greedy CTC per step, L2 flushed between
+    steps), the tensor fraction of its contractions, and the fp64 oracle on a
+    bounded sample of the same workload on the host cores."""
+    import numpy as np
+    import torch
+
+    from speech_encoder_b200 import w2v as B
+    from synth import inputs as S
+    w = S.workload(name)
+    shape = w.model
+    stream = torch.cuda.current_stream()
+    blob = S.pack_blob(shape, S.init_weights(shape, 0))
+    lens = [int(p.shape[1]) for p, _ in w.calls for _ in range(p.shape[0])]
+    audio = sum(lens) / 16000.0
+    frames = sum(B.w2v_num_frames(n) for n in lens)
+    flops = sum(contraction_flops(shape, n) for n in lens)
+    if name == "c4":
+        model = B.Model(shape, blob, max_samples=max(lens), max_batch=len(lens), use_cuda_graph=False)
+        pcm = torch.from_numpy(np.concatenate([p[0] for p, _ in w.calls])).to(dev)
+        T = [B.w2v_num_frames(n) for n in lens]
+        logits = torch.empty((sum(T), shape.vocab), dtype=torch.float32, device=dev)
+        tokens = torch.empty((sum(T),), dtype=torch.int32, device=dev)
+        ntok = torch.empty((len(T),), dtype=torch.int32, device=dev)
+
+        def step():
+            B.w2v_forward_varlen(model.handle, pcm, lens, logits, stream)
+            B.w2v_ctc_greedy_varlen(model.handle, logits, T, tokens, ntok, stream)
+        path = "varlen: 8 true-length clips in one launch set (w2v_forward_varlen + w2v_ctc_greedy_varlen)"
+    else:
+        p_np = w.calls[0][0]
+        bsz, n = p_np.shape
+        model = B.Model(shape, blob, max_samples=n, max_batch=bsz, use_cuda_graph=True)
+        pcm = torch.from_numpy(p_np).to(dev)
+        T = B.w2v_num_frames(n)
+        logits = torch.empty((bsz, T, shape.vocab), dtype=torch.float32, device=dev)
+        tokens = torch.empty((bsz, T), dtype=torch.int32, device=dev)
+        ntok = torch.empty((bsz,), dtype=torch.int32, device=dev)
+
+        def step():
+            B.w2v_forward(model.handle, pcm, n, bsz, logits, stream)
+            B.w2v_ctc_greedy(model.handle, logits, bsz, T, T, tokens, ntok, stream)
+        path = f"w2v_forward batch {bsz} x {n} samples as one CUDA graph + w2v_ctc_greedy"
+    del blob
+    for _ in range(max(warmup, 3)):
+        step()
+    model.sync()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        e0[i].record(stream)
+        step()
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    model.sync()
+    ms = sum(a.elapsed_time(b) for a, b in zip(e0, e1)) / steps
+    out = {"workload": OTHER_WORKLOADS[name], "path": path, "audio_s_per_step": audio, "ms_per_step": ms,
+           "audio_s_per_s": audio / (ms / 1000.0), "frames_per_s": frames / (ms / 1000.0),
+           "contraction_gflop_per_step": flops / 1e9,
+           "tensor_frac_of_step": flops / (ms * 1e-3) / 1e12 / tc_peak}
+    if name != "c4":
+        # per-class kernel times, as for the headline workload
+        us_t, fl_t = 0.0, 0.0
+        bsz, n = w.calls[0][0].shape
+        for cls in TENSOR_CLASSES:
+            us, nl, fl, _ = B.w2v_time_class(model.handle, pcm, n, bsz, logits, cls, reps=5, stream=stream)
+            us_t += us * nl
+            fl_t += fl * nl
+        out["tensor_frac_all_contractions"] = fl_t / (us_t * 1e-6) / 1e12 / tc_peak
+    model.close()
+    # the oracle on a bounded sample of the same workload (host cores)
+    from oracle import w2v_oracle as O
+    W64 = O.to_f64(S.init_weights(shape, 0))
+    clips = [p[i] for p, _ in w.calls for i in range(p.shape[0])]
+    clips.sort(key=len)
+    t0, done, secs = time.perf_counter(), 0, 0.0
+    for c in clips:
+        z = O.forward(shape, W64, c)
+        O.ctc_greedy(z, z.shape[0], 0)
+        done += 1
+        secs += len(c) / 16000.0
+        if time.perf_counter() - t0 >= cpu_budget_s:
+            break
+    wall = time.perf_counter() - t0
+    out["cpu_oracle"] = {"audio_s_per_s": secs / wall, "cores": blas_threads(),
+                         "sample": f"{done} of {len(clips)} clip(s), shortest first, {secs:.1f} audio s in {wall:.1f} s"}
     return out
 
 

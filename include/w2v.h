@@ -180,6 +180,42 @@ int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, int batch, fl
 int w2v_ctc_greedy(w2v_model* m, const float* logits_dev, int batch, int T, int t_valid, int32_t* tokens_dev,
                    int32_t* n_tokens_dev, void* stream);
 
+/* Varlen batched forward: `batch` clips of different lengths, each at its
+ * own true length (no padding, no attention mask across clips), in one
+ * launch set.  TensorRT-Model-Connect wav2vec2 README, "Wav2Vec2 CTC layouts"
+ * (true-length PCM input, no padded-batch attention mask) and "FP8
+ * quantization study -> When to revisit" (batches of clips give the GEMMs a
+ * larger share of the time).
+ *  - pcm_dev: float32, the clips packed back to back: clip c's n_samples[c]
+ *    samples (already normalised) start at sample offset
+ *    n_samples[0] + ... + n_samples[c-1].  n_samples: HOST int array [batch],
+ *    each in [400, max_samples].  1 <= batch <= min(max_batch, 64).
+ *  - logits_dev: float32 [T_0 + ... + T_{batch-1}][vocab], T_c =
+ *    w2v_num_frames(n_samples[c]); clip c's rows start at T_0 + ... + T_{c-1}.
+ *  - Each clip's conv feature encoder and positional conv run per clip; the
+ *    projection, encoder GEMMs and CTC head run once over all clips' frames
+ *    (packed on 128-row boundaries inside the model's workspace); attention
+ *    runs in one launch in which every query tile attends to its own clip's
+ *    keys only.  Results equal w2v_forward of each clip alone up to the GEMMs'
+ *    summation order.
+ *  - The first call whose packed frame count falls in a new bucket of 512
+ *    rows times the encoder GEMM tile candidates once (synchronous; make it
+ *    outside any stream capture); conv tiles come from a cost model, so a new
+ *    clip length never times anything.  Not recorded as a CUDA graph.
+ * Errors: W2V_EINVAL (null or misaligned pointer), W2V_ESHAPE (batch or a
+ * length out of range). */
+int w2v_forward_varlen(w2v_model* m, const float* pcm_dev, const int* n_samples, int batch, float* logits_dev,
+                       void* stream);
+
+/* Greedy CTC decode of packed clips of different lengths (the output of
+ * w2v_forward_varlen): logits_dev float32 [frames[0] + ... ][vocab], frames:
+ * HOST int array [batch] (frames decoded per clip, all of them).  tokens_dev:
+ * int32 [frames[0] + ...], clip c's tokens from offset frames[0] + ... +
+ * frames[c-1]; n_tokens_dev: int32 [batch].  Same decoding as
+ * w2v_ctc_greedy. */
+int w2v_ctc_greedy_varlen(w2v_model* m, const float* logits_dev, const int* frames, int batch, int32_t* tokens_dev,
+                          int32_t* n_tokens_dev, void* stream);
+
 /* Greedy CTC decode that allocates no memory and needs no model handle.  The
  * pages have no counterpart of this entry point: it exists for callers that
  * cannot allocate device memory when they decode — code driven from a

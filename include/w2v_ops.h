@@ -28,7 +28,11 @@ extern "C" {
  * `splits` CTAs whose partial sums are reduced in distributed shared memory;
  * splits -2 or -4 (bn >= 64) reduces 2 or 4 splits through an fp32 scratch in
  * L2 (TMA stores and loads; the call allocates and frees it on the stream),
- * summed in split order.  Invalid combinations return W2V_EINVAL. */
+ * summed in split order; splits 0 (bn >= 64) runs CTA pairs: clusters of two
+ * CTAs on 256-row tiles with the 2-CTA tensor-core instructions, each CTA
+ * loading its 128 rows of A and half of the tile's B columns (needs a
+ * 16-byte-aligned output row pitch: the direct TMA-store epilogue).  Invalid
+ * combinations return W2V_EINVAL. */
 int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, const float* bias, const void* residual,
                 int res_f32, void* out, int out_f32, int act, int bn, int splits, int* err_dev, void* stream);
 
@@ -60,7 +64,8 @@ int w2v_op_wait_probe(int* err_dev, uint64_t limit_ns, void* stream);
  *      polynomial path; argument clamped to [-15, 8], results below 2^-15
  *      flush to zero);
  *   2  tanh-GELU of a pair with the fp16x2 exponent (conv/FFN epilogues);
- *   3  tanh-GELU, fp32 sigmoid form;  4  exact GELU (erff);
+ *   3  tanh-GELU in fp32 with the hardware tanh (the GEMM epilogues);
+ *   4  exact GELU (erff);
  *   5  CUDA's exp2f(c x + b), the comparison point for 0 and 1.
  * Forms 0-2 take elements 2i and 2i+1 as one pair: n must be even.  The
  * softmax is the LiteRT discussion's plain SDPA and the tanh-GELU its first GPU

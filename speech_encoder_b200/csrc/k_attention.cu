@@ -62,9 +62,14 @@ __device__ __forceinline__ void quarter_barrier(int q) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kSubs) : "memory");
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
-attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmVt, int T, int H, __half* __restrict__ out, int* err) {
+// One CTA's work: query tile qt (local rows qt*128 ..) of one clip of T frames
+// and head h.  The clip's queries start at row qrow of the Q map (batch
+// coordinate bz), its keys at row krow0 of the K map and column krow0 of the V^T
+// map (V^T row block vrow .. vrow+63 for this head), its outputs at row
+// out_row0 of `out`.
+__device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt,
+                                               int T, int H, __half* __restrict__ out, int* err, int qt, int h,
+                                               int qrow, int krow0, int bz, int vrow, int64_t out_row0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red_max = reinterpret_cast<float*>(smem + AttnSmem::RED);  // [slot][sub][row]
@@ -78,7 +83,6 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int nkv = (T + 127) / 128;
 
   if (threadIdx.x == 0) {
@@ -123,8 +127,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (lane == 0) {
       pdl_wait();
       mbar_arrive_expect_tx(q_full, 16384);
-      tma_load_3d(smem + AttnSmem::Q, &tmQ, q_full, h * 64, qt * 128, b);
-      const int vrow = (b * H + h) * 64;
+      tma_load_3d(smem + AttnSmem::Q, &tmQ, q_full, h * 64, qrow, bz);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
@@ -136,9 +139,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         mbar_arrive_expect_tx(&kv_full[st], 32768);
         uint8_t* vs = smem + AttnSmem::V0 + st * 2 * AttnSmem::kVHalf;
-        tma_load_3d(smem + AttnSmem::K0 + st * 16384, &tmK, &kv_full[st], h * 64, j * 128, b);
-        tma_load_2d(vs, &tmVt, &kv_full[st], j * 128, vrow);
-        tma_load_2d(vs + AttnSmem::kVHalf, &tmVt, &kv_full[st], j * 128 + 64, vrow);
+        tma_load_3d(smem + AttnSmem::K0 + st * 16384, &tmK, &kv_full[st], h * 64, krow0 + j * 128, bz);
+        tma_load_2d(vs, &tmVt, &kv_full[st], krow0 + j * 128, vrow);
+        tma_load_2d(vs + AttnSmem::kVHalf, &tmVt, &kv_full[st], krow0 + j * 128 + 64, vrow);
         issued = j + 1;
       }
       if (!ok) {
@@ -303,7 +306,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const float l = tmem_ld1(tO + lane_base + 64);
       if (t < T) {
         const float inv = 1.0f / l;
-        __half* dst = out + (static_cast<int64_t>(b) * T + t) * (H * 64) + h * 64 + sub * kOCols;
+        __half* dst = out + (out_row0 + t) * (H * 64) + h * 64 + sub * kOCols;
 #pragma unroll
         for (int i = 0; i < kOCols; i += 8) {
           __half2 h0 = __floats2half2_rn(o[i] * inv, o[i + 1] * inv);
@@ -328,8 +331,34 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
 }
 
+__global__ void __launch_bounds__(kAttnThreads, 1)
+attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmVt, int T, int H, __half* __restrict__ out, int* err) {
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  attention_body(tmQ, tmK, tmVt, T, H, out, err, qt, h, qt * 128, 0, b, (b * H + h) * 64,
+                 static_cast<int64_t>(b) * T);
+}
+
+// Clips of different lengths packed along the rows of one [rows][H*64]
+// Q/K/output matrix (V^T [H*64][rows]), each clip's rows starting on a
+// 128-row boundary, so that no query or key tile holds two clips.  Query
+// tiles are numbered clip after clip; each attends to its own clip's keys.
+__global__ void __launch_bounds__(kAttnThreads, 1)
+attention_varlen_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmVt, int H, __half* __restrict__ out, int* err,
+                        const AttnClips clips) {
+  int c = 0;
+  while (c + 1 < clips.n && clips.qt0[c + 1] <= static_cast<int>(blockIdx.x)) ++c;
+  const int qt = static_cast<int>(blockIdx.x) - clips.qt0[c], h = blockIdx.y;
+  const int row0 = clips.row0[c];
+  attention_body(tmQ, tmK, tmVt, clips.len[c], H, out, err, qt, h, row0 + qt * 128, row0, 0, h * 64, row0);
+}
+
 cudaError_t attention_prepare() {
-  return cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::TOTAL);
+  cudaError_t r = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::TOTAL);
+  if (r == cudaSuccess)
+    r = cudaFuncSetAttribute(attention_varlen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::TOTAL);
+  return r;
 }
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt, int T,
@@ -337,6 +366,17 @@ cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, con
   if (T <= 0 || batch <= 0) return cudaSuccess;
   dim3 grid((T + 127) / 128, H, batch);
   return launch_pdl(attention_kernel, grid, dim3(kAttnThreads), AttnSmem::TOTAL, st, tmQ, tmK, tmVt, T, H, out, err);
+}
+
+cudaError_t launch_attention_varlen(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt,
+                                    const AttnClips& clips, int H, __half* out, int* err, cudaStream_t st) {
+  if (clips.n <= 0 || clips.n > kMaxVarlenClips) return cudaErrorInvalidValue;
+  for (int c = 0; c < clips.n; ++c)
+    if (clips.row0[c] % 128 != 0 || clips.len[c] <= 0 || clips.qt0[c + 1] - clips.qt0[c] != (clips.len[c] + 127) / 128)
+      return cudaErrorInvalidValue;
+  dim3 grid(clips.qt0[clips.n], H, 1);
+  return launch_pdl(attention_varlen_kernel, grid, dim3(kAttnThreads), AttnSmem::TOTAL, st, tmQ, tmK, tmVt, H, out,
+                    err, clips);
 }
 
 }  // namespace w2v

@@ -306,7 +306,9 @@ conv0_tc_kernel(const __grid_constant__ CUtensorMap tmOut, const float* pcm, int
       }
       if (lane == 0) bulk_commit_group();
     }
-    if (lane == 0) bulk_wait_all();
+    // the staging boxes must outlive the stores' reads of them; the grid
+    // boundary makes the global writes visible to the next kernel
+    if (lane == 0) bulk_wait_read_all();
   }
   tc_fence_before();
   __syncthreads();

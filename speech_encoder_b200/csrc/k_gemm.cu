@@ -38,12 +38,14 @@
 
 namespace w2v {
 
-template <int BN>
+// PAIR: a CTA pair computes a 256 x BN tile (cta_group::2), each CTA holding
+// 128 rows of A and BN/2 rows of B per stage.
+template <int BN, bool PAIR = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BK = 64;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int RING_MAX = 200 * 1024;
   static constexpr int STAGES = (RING_MAX / STAGE) > 8 ? 8 : (RING_MAX / STAGE);
@@ -75,15 +77,41 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The residual of 4 consecutive columns [col, col+4) of row grow, as stored
+// (before any LayerNorm), zeros where there is none.  `vec` selects 16-/8-byte
+// loads (row starts and pointers 16-byte aligned, full 4-vector in range).
+// Split from the arithmetic so that an epilogue can issue these loads long
+// before the accumulator is ready.
+__device__ __forceinline__ float4 load_res4(const GemmEpiArgs& e, int bzb, int grow, int col, int nv, bool vec) {
+  float rv[4] = {0.f, 0.f, 0.f, 0.f};
+  if (e.residual) {
+    const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+    if (e.res_f32) {
+      const float* rp = static_cast<const float*>(e.residual) + roff;
+      if (vec && nv == 4) return *reinterpret_cast<const float4*>(rp);
+      for (int i = 0; i < nv; ++i) rv[i] = rp[i];
+    } else {
+      const __half* rp = static_cast<const __half*>(e.residual) + roff;
+      if (vec && nv == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(rp);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        return make_float4(a.x, a.y, b.x, b.y);
+      }
+      for (int i = 0; i < nv; ++i) rv[i] = __half2float(rp[i]);
+    }
+  }
+  return make_float4(rv[0], rv[1], rv[2], rv[3]);
+}
+
 // Final epilogue for 4 consecutive columns [col, col+4) of row grow: bias
-// (from shared memory), GELU, residual, store.  `vec` selects 16-/8-byte
-// accesses (row starts and pointers 16-byte aligned, full 4-vector in range).
+// (from shared memory), GELU, the residual `res` (from load_res4), store.
 // lnr: the row's LayerNorm factors (rstd, -mean * rstd) when e.ln_mode != 0;
 // vec_s: the LN column vectors of this tile (ln_mode 1: column sums; 2: gamma,
 // then beta at vec_s + BN).
-__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, const float* vec_s, int bn, float2 lnr,
-                                        int lcol, int grow, int col, int nv, int bzb, const GemmEpiArgs& e,
-                                        void* outp, int ocol0, bool vec) {
+__device__ __forceinline__ void finish4r(float (&x)[4], float4 res, const float* bias_s, const float* vec_s, int bn,
+                                         float2 lnr, int lcol, int grow, int col, int nv, int bzb,
+                                         const GemmEpiArgs& e, void* outp, int ocol0, bool vec) {
   const int ln_mode = e.ln_cfg & 255;
   if (ln_mode == 1) {
 #pragma unroll
@@ -92,27 +120,7 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, cons
 #pragma unroll
   for (int i = 0; i < 4; ++i) x[i] = apply_act(x[i] + bias_s[lcol + i], e.act);
   if (e.residual) {
-    const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
-    float rv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (e.res_f32) {
-      const float* rp = static_cast<const float*>(e.residual) + roff;
-      if (vec && nv == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(rp);
-        rv[0] = t.x; rv[1] = t.y; rv[2] = t.z; rv[3] = t.w;
-      } else {
-        for (int i = 0; i < nv; ++i) rv[i] = rp[i];
-      }
-    } else {
-      const __half* rp = static_cast<const __half*>(e.residual) + roff;
-      if (vec && nv == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(rp);
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-        rv[0] = a.x; rv[1] = a.y; rv[2] = b.x; rv[3] = b.y;
-      } else {
-        for (int i = 0; i < nv; ++i) rv[i] = __half2float(rp[i]);
-      }
-    }
+    float rv[4] = {res.x, res.y, res.z, res.w};
     if (ln_mode == 2) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) rv[i] = fmaf(fmaf(rv[i], lnr.x, lnr.y), vec_s[lcol + i], vec_s[bn + lcol + i]);
@@ -136,16 +144,29 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, cons
   }
 }
 
+__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, const float* vec_s, int bn, float2 lnr,
+                                        int lcol, int grow, int col, int nv, int bzb, const GemmEpiArgs& e,
+                                        void* outp, int ocol0, bool vec) {
+  finish4r(x, load_res4(e, bzb, grow, col, nv, vec), bias_s, vec_s, bn, lnr, lcol, grow, col, nv, bzb, e, outp,
+           ocol0, vec);
+}
+
 // mode: 0 generic, 1 direct (TMA store), 2 split-K through distributed shared
 // memory, 3 split-K through an L2 scratch (with the direct stores)
 // SPLIT: the instantiation for split-K launches (modes 2 and 3); the other one
 // runs modes 0 and 1 only.
-template <int BN, bool SPLIT>
+// PAIR: CTA pairs (clusters of 2 along M) on 256-row tiles with the 2-CTA
+// tensor-core instructions, mode 1 only.  The pair halves the B operand bytes
+// each SM takes in per output, which bounds the mainloop (an SM receives
+// about 72 bytes per clock from L2).  Each CTA still owns 128 accumulator rows
+// (m0 = blockIdx.x * 128) and runs the same epilogue on them.
+template <int BN, bool SPLIT, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                const __grid_constant__ CUtensorMap tmV, GemmDims s, GemmEpiArgs e, int vec_ok, int mode, int* err) {
-  using C = GemmCfg<BN>;
+  static_assert(!(SPLIT && PAIR), "pairs do not split K");
+  using C = GemmCfg<BN, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + C::BIAS_OFF);
@@ -168,6 +189,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int kb0 = split * nk / S;
   const int nkl = (split + 1) * nk / S - kb0;  // K blocks of this CTA (>= 1)
   const int pre = nkl < C::STAGES ? nkl : C::STAGES;
+  // pair rank (0: the CTA that issues the MMAs), cluster rank of that CTA,
+  // the first B row this CTA loads, and the pair's CTA mask
+  const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+  const uint32_t prank = crank & 1u;
+  const uint32_t lead = crank & ~1u;
+  const int nb0 = PAIR ? n0 + static_cast<int>(prank) * (BN / 2) : n0;
+  const uint16_t pmask = static_cast<uint16_t>(3u << lead);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
@@ -180,22 +208,99 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     pdl_launch_dependents();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    // Weights do not depend on the previous kernel: start them right away.
-    for (int i = 0; i < pre; ++i) {
-      mbar_arrive_expect_tx(&full[i], C::STAGE);
-      tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, &full[i], (kb0 + i) * C::BK, n0);
+    // Weights do not depend on the previous kernel: start them right away
+    // (pairs: after the cluster barrier below, since they complete on the
+    // other CTA's barriers).
+    if (!PAIR) {
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], C::STAGE);
+        tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, &full[i], (kb0 + i) * C::BK, n0);
+      }
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // pairs: both CTAs' barriers are initialised before either signals the other
+  if (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (PAIR && warp == 0) {
+    if (lane == 0) {
+      // Both CTAs load their own A rows and B half; every copy completes on
+      // the even CTA's full barrier, which expects the bytes of both.
+      auto fbar = [&](int st) { return mapa_shared(smem_u32(&full[st]), lead); };
+      for (int i = 0; i < pre; ++i) {
+        if (prank == 0) mbar_arrive_expect_tx(&full[i], 2 * C::STAGE);
+        tma_load_2d_pair(smem + i * C::STAGE + C::A_BYTES, &tmB, fbar(i), (kb0 + i) * C::BK, nb0);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) {
+        const int k = (kb0 + i) * C::BK;
+        tma_load_3d_pair(smem + i * C::STAGE, &tmA, fbar(i), k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
+      }
+      bool ok = true;
+      for (int i = pre; i < nkl; ++i) {
+        const int st = i % C::STAGES;
+        if (!mbar_wait(&empty[st], ((i / C::STAGES) & 1) ^ 1)) {
+          atomicOr(err, kErrWaitProducer);
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + st * C::STAGE;
+        if (prank == 0) mbar_arrive_expect_tx(&full[st], 2 * C::STAGE);
+        const int k = (kb0 + i) * C::BK;
+        tma_load_3d_pair(sa, &tmA, fbar(st), k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
+        tma_load_2d_pair(sa + C::A_BYTES, &tmB, fbar(st), k, nb0);
+      }
+      // Wait until the last stages have been consumed: every copy into this
+      // CTA has landed and every release the MMA issuer sent here has
+      // arrived, before this CTA may leave.
+      if (ok) {
+        for (int i = (nkl > C::STAGES ? nkl - C::STAGES : 0); i < nkl; ++i)
+          if (!mbar_wait(&empty[i % C::STAGES], (i / C::STAGES) & 1)) {
+            atomicOr(err, kErrWaitProducer);
+            break;
+          }
+      }
+    }
+  } else if (PAIR && warp == 1) {
+    if (lane == 0 && prank == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(256, BN);
+      const uint64_t dA0 = desc_sw128(smem_u32(smem));
+      const uint64_t dB0 = desc_sw128(smem_u32(smem) + C::A_BYTES);
+      bool ok = true;
+      int st = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nkl; ++i) {
+        if (!mbar_wait(&full[st], ph)) {
+          atomicOr(err, kErrWaitMma);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t off = static_cast<uint64_t>(st * (C::STAGE >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16_pair(tmem, dA0 + off + 2 * kk, dB0 + off + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+        umma_commit_pair(&empty[st], pmask);
+        if (++st == C::STAGES) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      if (ok) umma_commit_pair(accf, pmask);
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       pdl_wait();
       for (int i = 0; i < pre; ++i) {
@@ -267,6 +372,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int region = e.qkv_d > 0 ? n0 / e.qkv_d : -1;
   const bool vec = vec_ok != 0;
   const int ln_mode = e.ln_cfg & 255;
+  // Owner rows per CTA in the distributed-shared-memory split form are at
+  // most 64 (S >= 2); for tiles up to 128 wide every thread finishes at most
+  // kIter2 4-column chunks of them, few enough to prefetch into registers.
+  constexpr int kIter2 = (64 * C::ROW_CHUNKS + kEpiThreads - 1) / kEpiThreads;
+  constexpr bool kPre2 = kIter2 <= 8;
+  float4 resv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) resv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   bool ok = true;
   if (epi) {
     for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (e.bias && n0 + i < s.N) ? e.bias[n0 + i] : 0.f;
@@ -309,6 +422,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           f = make_float2(rstd, -mean * rstd);
         }
         rowln_s[et] = f;
+      }
+    }
+    // Residual values this thread adds, loaded now while the mainloop runs
+    // (they come from earlier kernels): in the direct form the first 32-column
+    // chunk of its row, in the distributed-shared-memory split form every
+    // 4-column chunk of the rows its CTA finishes.
+    if (e.residual && region <= 0) {
+      pdl_wait();
+      if (mode == 1 || (SPLIT && mode == 3 && (q * S) / 4 == split)) {
+        const int grow = m0 + r;
+        const int col0 = n0 + half * (BN / 2);
+        if (grow < s.M) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) resv[i] = load_res4(e, bzb, grow, col0 + 4 * i, min(4, s.N - col0 - 4 * i), vec);
+        }
+      } else if (SPLIT && mode == 2 && kPre2) {
+        const int rank = static_cast<int>(cluster_ctarank());
+        const int r0 = rank * C::BM / S;
+        const int nrows = (rank + 1) * C::BM / S - r0;
+#pragma unroll
+        for (int it = 0; it < kIter2; ++it) {
+          const int idx = et + kEpiThreads * it;
+          const int lr = idx / C::ROW_CHUNKS, j = idx % C::ROW_CHUNKS;
+          const int grow = m0 + r0 + lr, col = n0 + 4 * j;
+          if (lr < nrows && grow < s.M && col < s.N) resv[it] = load_res4(e, bzb, grow, col, min(4, s.N - col), vec);
+        }
       }
     }
     ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
@@ -419,9 +558,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int i = 0; i < 32; ++i) dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(v[i]);
         }
       }
+      // The staging boxes must stay valid until the stores have read them;
+      // the grid boundary makes the global writes visible to the next kernel.
       if (lane == 0) {
         bulk_commit_group();
-        bulk_wait_all();
+        bulk_wait_read_all();
       }
     }
     tc_fence_before();
@@ -536,51 +677,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         const int col = n0 + c;
         if (e.residual && grow < s.M) {
-          const int64_t roff =
-              static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
-          const int nv = min(32, s.N - col);
-          if (e.res_f32) {
-            const float* rp = static_cast<const float*>(e.residual) + roff;
-            if (nv == 32) {
+          // the first chunk's residual was loaded during the mainloop
+          float4 rq[8];
+          if (c == half * (BN / 2)) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 rv = *reinterpret_cast<const float4*>(rp + i);
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + rv.x;
-                v[i + 1] = apply_act(v[i + 1] + bias_s[c + i + 1], e.act) + rv.y;
-                v[i + 2] = apply_act(v[i + 2] + bias_s[c + i + 2], e.act) + rv.z;
-                v[i + 3] = apply_act(v[i + 3] + bias_s[c + i + 3], e.act) + rv.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + (i < nv ? rp[i] : 0.f);
-            }
+            for (int i = 0; i < 8; ++i) rq[i] = resv[i];
           } else {
-            const __half* rp = static_cast<const __half*>(e.residual) + roff;
-            if (nv == 32) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 8) {
-                const uint4 u = *reinterpret_cast<const uint4*>(rp + i);
-                const __half2* h = reinterpret_cast<const __half2*>(&u);
+            for (int i = 0; i < 8; ++i) rq[i] = load_res4(e, bzb, grow, col + 4 * i, min(4, s.N - col - 4 * i), vec);
+          }
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  float2 f = __half22float2(h[k]);
-                  if (ln_mode == 2) {
-                    const int cc = c + i + 2 * k;
-                    f.x = fmaf(fmaf(f.x, lnr.x, lnr.y), vec_s[cc], vec_s[BN + cc]);
-                    f.y = fmaf(fmaf(f.y, lnr.x, lnr.y), vec_s[cc + 1], vec_s[BN + cc + 1]);
-                  }
-                  v[i + 2 * k] = apply_act(v[i + 2 * k] + bias_s[c + i + 2 * k], e.act) + f.x;
-                  v[i + 2 * k + 1] = apply_act(v[i + 2 * k + 1] + bias_s[c + i + 2 * k + 1], e.act) + f.y;
-                }
-              }
-            } else {
+          for (int i = 0; i < 8; ++i) {
+            float f[4] = {rq[i].x, rq[i].y, rq[i].z, rq[i].w};
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float f = i < nv ? __half2float(rp[i]) : 0.f;
-                if (ln_mode == 2) f = fmaf(fmaf(f, lnr.x, lnr.y), vec_s[c + i], vec_s[BN + c + i]);
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + f;
-              }
+            for (int k = 0; k < 4; ++k) {
+              const int cc = c + 4 * i + k;
+              if (ln_mode == 2) f[k] = fmaf(fmaf(f[k], lnr.x, lnr.y), vec_s[cc], vec_s[BN + cc]);
+              v[4 * i + k] = apply_act(v[4 * i + k] + bias_s[cc], e.act) + f[k];
             }
           }
         } else {
@@ -618,9 +731,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       if (e.ln_out && ok && grow < s.M)
         e.ln_out[static_cast<int64_t>(2 * blockIdx.y + half) * s.M + grow] = make_float2(st1, st2);
-      if (lane == 0) {
+      if (lane == 0) {  // as above: wait until the boxes have been read
         bulk_commit_group();
-        bulk_wait_all();
+        bulk_wait_read_all();
       }
       (void)outp;
     }
@@ -685,6 +798,50 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(apply_act(x[i] + bias_s[4 * j + i], e.act));
+        }
+      } else if (kPre2) {
+        // Chunk idx = et + 256 it of the owner rows (row idx / RC, chunk
+        // idx % RC): all residual loads were issued during the mainloop.  With
+        // row sums to store, the RC consecutive lanes of a row (a whole warp
+        // for 128-wide tiles) add up its two half-tile sums in a fixed order.
+        void* outp = region == 1 ? e.out_k : e.out;
+        const int ocol0 = region > 0 ? region * e.qkv_d : 0;
+        constexpr int RC = C::ROW_CHUNKS;
+        constexpr int GROUP = RC >= 32 ? 32 : RC;
+#pragma unroll
+        for (int it = 0; it < kIter2; ++it) {
+          const int idx = et + kEpiThreads * it;
+          const int lr = idx / RC, j = idx % RC;
+          const int grow = m0 + r0 + lr, col = n0 + 4 * j;
+          const bool row_live = lr < nrows && grow < s.M;
+          const bool live = row_live && col < s.N;
+          float p1 = 0.f, p2 = 0.f;
+          if (live) {
+            const int nv = min(4, s.N - col);
+            const float4 v = fetch(lr, j);
+            float x[4] = {v.x, v.y, v.z, v.w};
+            finish4r(x, resv[it], bias_s, vec_s, BN, row_lnr(r0 + lr), 4 * j, grow, col, nv, bzb, e, outp, ocol0,
+                     vec);
+            for (int i = 0; i < nv; ++i) {
+              p1 += x[i];
+              p2 = fmaf(x[i], x[i], p2);
+            }
+          }
+          if (e.ln_out) {
+            const bool lo = 4 * j < BN / 2;
+            float a1 = lo ? p1 : 0.f, a2 = lo ? p2 : 0.f, b1 = lo ? 0.f : p1, b2 = lo ? 0.f : p2;
+#pragma unroll
+            for (int o = GROUP / 2; o > 0; o >>= 1) {
+              a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+              a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+              b1 += __shfl_xor_sync(0xffffffffu, b1, o);
+              b2 += __shfl_xor_sync(0xffffffffu, b2, o);
+            }
+            if (row_live && j == 0) {
+              e.ln_out[static_cast<int64_t>(2 * blockIdx.y) * s.M + grow] = make_float2(a1, a2);
+              e.ln_out[static_cast<int64_t>(2 * blockIdx.y + 1) * s.M + grow] = make_float2(b1, b2);
+            }
+          }
         }
       } else {
         void* outp = region == 1 ? e.out_k : e.out;
@@ -780,9 +937,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     __syncthreads();
   }
 
+  if (PAIR) {
+    // neither CTA of the pair leaves (or frees the pair's TMEM) while the
+    // other may still touch its shared memory, barriers or TMEM
+    tc_fence_before();
+    cluster_sync();
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -833,10 +999,14 @@ int gemm_pick(GemmShape* s, int bn_divides) {
 
 template <int BN>
 static cudaError_t prepare_bn() {
-  cudaError_t r =
-      cudaFuncSetAttribute(gemm_tc_kernel<BN, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM);
+  cudaError_t r = cudaFuncSetAttribute(gemm_tc_kernel<BN, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       GemmCfg<BN>::SMEM);
   if (r == cudaSuccess)
-    r = cudaFuncSetAttribute(gemm_tc_kernel<BN, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM);
+    r = cudaFuncSetAttribute(gemm_tc_kernel<BN, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<BN>::SMEM);
+  if (r == cudaSuccess && BN >= 64)
+    r = cudaFuncSetAttribute(gemm_tc_kernel<BN, false, (BN >= 64)>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<BN, (BN >= 64)>::SMEM);
   return r;
 }
 
@@ -856,27 +1026,35 @@ template <int BN>
 static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmO,
                              const CUtensorMap& tmO2, const CUtensorMap& tmV, const GemmShape& s,
                              const GemmEpilogue& e, int vec_ok, int mode, int* err, cudaStream_t st) {
-  using C = GemmCfg<BN>;
   const int S = s.splits;
-  dim3 grid((s.M + 127) / 128, (s.N + BN - 1) / BN, S > 1 ? S : s.batch);  // modes 2 and 3: S > 1
+  const bool pair = s.pair;
+  // pairs: 2 CTAs per 256-row tile (grid x even), one cluster per pair
+  dim3 grid(pair ? 2 * ((s.M + 255) / 256) : (s.M + 127) / 128, (s.N + BN - 1) / BN, S > 1 ? S : s.batch);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.dynamicSmemBytes = pair ? GemmCfg<BN, (BN >= 64)>::SMEM : GemmCfg<BN>::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.x = pair ? 2 : 1;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = S > 1 ? S : 1;  // modes 2 and 3
   cfg.attrs = attr;
-  cfg.numAttrs = S > 1 ? 2 : 1;
+  cfg.numAttrs = (S > 1 || pair) ? 2 : 1;
   const GemmDims sd = s;      // the kernel's parameter block holds only
   const GemmEpiArgs ea = e;   // what it reads
-  return S > 1 ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, true>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok, mode, err)
-               : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok, mode, err);
+  if (pair) {
+    if (BN < 64 || S > 1 || mode != 1) return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, (BN >= 64)>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
+                              mode, err);
+  }
+  return S > 1 ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, true, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
+                                    mode, err)
+               : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
+                                    mode, err);
 }
 
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
@@ -885,6 +1063,8 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   if (s.K <= 0 || s.K % 64 != 0 || s.a_kwrap <= 0 || s.a_kwrap % 64 != 0) return cudaErrorInvalidValue;
   if (s.splits < 1 || s.splits > 8 || s.splits > s.K / 64 || (s.splits > 1 && s.batch != 1))
     return cudaErrorInvalidValue;
+  // pairs: no split, tiles at least 64 wide, the direct (TMA-store) epilogue
+  if (s.pair && (s.splits != 1 || s.split_l2 || bn < 64)) return cudaErrorInvalidValue;
   if (e.qkv_d > 0 && (e.qkv_d % bn != 0 || s.N != 3 * e.qkv_d || e.t_len <= 0)) return cudaErrorInvalidValue;
   // Folded LayerNorm: row statistics come as partial sums indexed by row
   // (one clip batch); the normalised residual must be fp16.
@@ -945,6 +1125,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
     if (built) mode = l2split ? 3 : 1;
   }
   if (l2split && mode != 3) return cudaErrorInvalidValue;
+  if (s.pair && mode != 1) return cudaErrorInvalidValue;
   switch (bn) {
     case 32: return launch_bn<32>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
     case 64: return launch_bn<64>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);

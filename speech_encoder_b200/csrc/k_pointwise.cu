@@ -5,7 +5,7 @@
 //   fn 0  exp2_affine_f16x2:      2^(c x + b) as fp16, exponent unit (f16x2)
 //   fn 1  exp2_affine_poly_f16x2: the same on the FMA/ALU pipes (cubic)
 //   fn 2  gelu_tanh2:             tanh-GELU of a pair, fp16x2 exponent
-//   fn 3  gelu_tanh:              tanh-GELU, fp32 sigmoid form
+//   fn 3  gelu_tanh:              tanh-GELU, fp32 with the hardware tanh
 //   fn 4  gelu_erf:               exact GELU through erff
 //   fn 5  exp2f(c x + b):         CUDA's own exp2f, for comparison
 // The pair forms take elements 2i and 2i+1 together (n must be even).

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -29,6 +30,8 @@ constexpr int kKern[7] = {10, 3, 3, 3, 3, 2, 2};
 constexpr int kStride[7] = {5, 2, 2, 2, 2, 2, 2};
 constexpr int kPosK = 128;
 constexpr int kPosG = 16;
+constexpr size_t kMaxPlans = 16;   // launch plans kept per model
+constexpr size_t kMaxGraphs = 8;   // instantiated forward graphs kept per model
 
 int conv_len(int n, int k, int s) { return n >= k ? (n - k) / s + 1 : 0; }
 
@@ -198,6 +201,13 @@ struct w2v_model {
   float* r = nullptr;
   __half* ra = nullptr;
   float2 *stats_a = nullptr, *stats_f = nullptr;
+  // Varlen form: the conv encoder output of every clip packed at 128-row
+  // aligned offsets, [varlen_rows_max][512] fp16.
+  __half* cpk = nullptr;
+  int varlen_rows_max = 0;
+  // Tile choices (bn, splits) of the encoder GEMM roles (projection, QKV,
+  // out, FFN1, FFN2, lm_head) per bucket of 512 packed rows, timed once.
+  std::map<int, std::array<std::array<int, 2>, 6>> varlen_choices;
   double* gn_partial = nullptr;   // [max_batch][<=296][65] per-block window moments
   unsigned* gn_ticket = nullptr;  // [max_batch] last-block tickets (zero between calls)
   float2* gn_ss = nullptr;        // [max_batch][512] GroupNorm scale/shift
@@ -211,9 +221,22 @@ struct w2v_model {
   float* part_ws = nullptr;      // split-K through L2: fp32 [4][ws_rows][ws_ld]
   int64_t ws_rows = 0, ws_ld = 0;
   int max_rows = 0;
-  std::map<std::pair<int, int>, std::unique_ptr<Plan>> plans;
-  std::map<std::tuple<int, int, const void*, void*>, cudaGraphExec_t> graphs;
-  std::map<std::tuple<int, int, const void*, void*>, int> graph_launches;
+  // Launch plans per (n_samples, batch) and instantiated graphs per
+  // (n_samples, batch, pcm, logits), both least-recently-used caches of a
+  // fixed size, so callers that vary lengths or hand over fresh buffers on
+  // every call do not grow them without bound.
+  struct PlanEntry {
+    std::unique_ptr<Plan> plan;
+    uint64_t used = 0;
+  };
+  struct GraphEntry {
+    cudaGraphExec_t exec = nullptr;
+    int launches = 0;
+    uint64_t used = 0;
+  };
+  std::map<std::pair<int, int>, PlanEntry> plans;
+  std::map<std::tuple<int, int, const void*, void*>, GraphEntry> graphs;
+  uint64_t use_tick = 0;
   cudaStream_t cap_stream = nullptr;
   const Plan* last_plan = nullptr;
   int last_launches = 0;
@@ -394,6 +417,23 @@ bool l2_split_ok(const w2v_model* m, const GemmShape& s, int N, int bn, int sp) 
          s.K / 64 >= 2 * sp;
 }
 
+// A GEMM role's launch form as one integer (plan files, refinement): 0 = CTA
+// pairs on 256-row tiles, 1 = one CTA per 128-row tile, s > 1 = s K splits
+// reduced through distributed shared memory, -s = s K splits through L2.
+int form_code(const GemmShape& s) { return s.pair ? 0 : (s.split_l2 ? -s.splits : s.splits); }
+
+void set_form(GemmShape* s, int code) {
+  s->pair = code == 0;
+  s->splits = code == 0 ? 1 : (code < 0 ? -code : code);
+  s->split_l2 = code < 0;
+}
+
+// The B operand map of a GEMM with tile width bn in form `code` (pairs load
+// half of the tile's rows per CTA).
+cudaError_t map_b(CUtensorMap* t, const __half* W, int N, int K, int bn, int code) {
+  return map_matrix(t, W, N, K, code == 0 ? bn / 2 : bn);
+}
+
 int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* W, int N, int K,
               const GemmEpilogue& e, int bn_divides, int* bn_out) {
   const int nk = K / 64;
@@ -404,10 +444,10 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     const bool bn_ok = (bn == 32 || bn == 64 || bn == 128 || bn == 192 || bn == 256) &&
                        (bn_divides <= 0 || bn_divides % bn == 0);
     const bool sp_ok = sp == 1 || (sp > 1 && sp <= 8 && s->batch == 1 && sp <= nk) ||
-                       ((sp == -2 || sp == -4) && l2_split_ok(m, *s, N, bn, -sp));
+                       ((sp == -2 || sp == -4) && l2_split_ok(m, *s, N, bn, -sp)) || (sp == 0 && bn >= 64);
     if (!bn_ok || !sp_ok) return fail(m, W2V_EINVAL, "plan file: bn=%d splits=%d invalid for N=%d K=%d", bn, sp, N, K);
-    s->splits = splits;
-    s->split_l2 = sp < 0;
+    (void)splits;
+    set_form(s, sp);
     *bn_out = bn;
     return W2V_OK;
   }
@@ -425,19 +465,22 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
   for (int bn : {32, 64, 128, 192, 256}) {
     if (bn == 32 ? N > 32 : N <= bn / 2) continue;
     if (bn_divides > 0 && bn_divides % bn != 0) continue;
-    CUtensorMap tmB;
+    CUtensorMap tmB, tmBp;
     CUDA_OR(m, map_matrix(&tmB, W, N, K, bn));
+    if (bn >= 64) CUDA_OR(m, map_b(&tmBp, W, N, K, bn, 0));
     // sp > 1: K splits reduced through distributed shared memory; sp < 0:
-    // -sp splits reduced through the L2 scratch
-    for (int sp : {1, 2, 3, 4, 6, -2, -4}) {
+    // -sp splits reduced through the L2 scratch; sp 0: CTA pairs
+    for (int sp : {1, 2, 3, 4, 6, -2, -4, 0}) {
       if (sp > 1 && (s->batch != 1 || nk < 16 || sp > nk)) continue;
       if (sp < 0 && !l2_split_ok(m, *s, N, bn, -sp)) continue;
+      if (sp == 0 && bn < 64) continue;
       GemmShape c = *s;
-      c.splits = sp < 0 ? -sp : sp;
-      c.split_l2 = sp < 0;
-      CUDA_OR(m, launch_gemm(tmA, tmB, c, bn, e, m->err_word, st));
+      set_form(&c, sp);
+      const cudaError_t lr = launch_gemm(tmA, sp == 0 ? tmBp : tmB, c, bn, e, m->err_word, st);
+      if (sp == 0 && lr == cudaErrorInvalidValue) continue;  // pairs need the direct epilogue
+      CUDA_OR(m, lr);
       CUDA_OR(m, cudaEventRecord(e0, st));
-      for (int it = 0; it < 3; ++it) CUDA_OR(m, launch_gemm(tmA, tmB, c, bn, e, m->err_word, st));
+      for (int it = 0; it < 3; ++it) CUDA_OR(m, launch_gemm(tmA, sp == 0 ? tmBp : tmB, c, bn, e, m->err_word, st));
       CUDA_OR(m, cudaEventRecord(e1, st));
       CUDA_OR(m, cudaEventSynchronize(e1));
       float ms = 0.f;
@@ -452,15 +495,15 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
   if (!best_bn) return fail(m, W2V_ECUDA, "no GEMM configuration for N=%d K=%d", N, K);
-  s->splits = best_s < 0 ? -best_s : best_s;
-  s->split_l2 = best_s < 0;
+  set_form(s, best_s);
   *bn_out = best_bn;
   return W2V_OK;
 }
 
-int build_plan(w2v_model* m, int n, int batch, Plan* p) {
-  const w2v_config& c = m->cfg;
-  const int d = c.d_model, F = c.d_ffn, V = c.vocab, H = c.n_heads;
+// The conv feature encoder part of a plan: frame counts of every layer and
+// the conv GEMMs' tensor maps and tile choices, for `batch` clips of n samples.
+// analytic: tile choices from the cost model (no timing on the device).
+int build_frontend(w2v_model* m, int n, int batch, Plan* p, bool analytic) {
   p->n = n;
   p->batch = batch;
   p->T[0] = conv_len(n, kKern[0], kStride[0]);
@@ -471,7 +514,6 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   p->t_pad = (p->Tf + 7) & ~7;
   p->rows = batch * p->Tf;
   if (p->Tf < 1) return fail(m, W2V_ESHAPE, "n_samples=%d gives no frame", n);
-
   for (int i = 1; i < 7; ++i) {
     const __half* in = ((i - 1) % 2 == 0) ? m->act_a : m->act_b;
     const int K = kKern[i] * kC;
@@ -483,22 +525,49 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
     s.K = K;
     s.a_kwrap = 2 * kC;
     s.batch = batch;
-    {
+    if (analytic) {
+      p->convBN[i] = gemm_pick(&s, 0);
+    } else {
       const int rc = tune_gemm(m, &s, p->convA[i], m->cw[i], kC, K, epi_conv(m, *p, i), 0, &p->convBN[i]);
       if (rc != W2V_OK) return rc;
     }
     p->convS[i] = s;
-    CUDA_OR(m, map_matrix(&p->convB[i], m->cw[i], kC, K, p->convBN[i]));
+    CUDA_OR(m, map_b(&p->convB[i], m->cw[i], kC, K, p->convBN[i], form_code(s)));
   }
+  return W2V_OK;
+}
+
+// One GEMM role's tile choice: timed on the device, or given (bn > 0).
+int pick_role(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* W, int N, int K, const GemmEpilogue& e,
+              int bn_divides, int* bn_out, int given_bn, int given_sp) {
+  if (given_bn > 0) {
+    set_form(s, given_sp);
+    *bn_out = given_bn;
+    return W2V_OK;
+  }
+  return tune_gemm(m, s, tmA, W, N, K, e, bn_divides, bn_out);
+}
+
+// The part of a plan after the conv encoder, over p->rows packed rows of
+// clips of p->Tf frames (p->batch of them; one pseudo-clip of all rows for
+// the varlen form): projection, encoder GEMMs, attention maps, CTC head.
+// given: tile choices (bn, splits) of proj, QKV, out, FFN1, FFN2, lm_head, or
+// null to choose them (timing each GEMM role on the device).
+int build_encoder(w2v_model* m, Plan* p, const int (*given)[2]) {
+  const w2v_config& c = m->cfg;
+  const int d = c.d_model, F = c.d_ffn, V = c.vocab, H = c.n_heads;
+  const int batch = p->batch;
   const int rows = p->rows;
+  auto g_bn = [&](int i) { return given ? given[i][0] : 0; };
+  auto g_sp = [&](int i) { return given ? given[i][1] : 1; };
   {
     CUDA_OR(m, map_a(&p->projA, m->ln512, kC, rows, kC, 1, 0));
     GemmShape s;
     s.M = rows; s.N = d; s.K = kC; s.a_kwrap = kC; s.batch = 1;
-    const int rc = tune_gemm(m, &s, p->projA, m->wp, d, kC, epi_proj(m), 0, &p->projBN);
+    const int rc = pick_role(m, &s, p->projA, m->wp, d, kC, epi_proj(m), 0, &p->projBN, g_bn(0), g_sp(0));
     if (rc != W2V_OK) return rc;
     p->projS = s;
-    CUDA_OR(m, map_matrix(&p->projB, m->wp, d, kC, p->projBN));
+    CUDA_OR(m, map_b(&p->projB, m->wp, d, kC, p->projBN, form_code(s)));
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(p->Tf), static_cast<uint64_t>(batch)};
@@ -520,11 +589,14 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   p->f1S = shp(F, d);
   p->f2S = shp(d, F);
   if (c.n_layers > 0) {
-    int rc = tune_gemm(m, &p->qkvS, p->aH, m->L[0].wqkv, 3 * d, d, epi_qkv(m, *p, 0), d, &p->qkvBN);
-    if (rc == W2V_OK) rc = tune_gemm(m, &p->oS, p->aAO, m->L[0].wo, d, d, epi_resid(m, *p, 0, false), 0, &p->oBN);
+    int rc = pick_role(m, &p->qkvS, p->aH, m->L[0].wqkv, 3 * d, d, epi_qkv(m, *p, 0), d, &p->qkvBN, g_bn(1), g_sp(1));
     if (rc == W2V_OK)
-      rc = tune_gemm(m, &p->f1S, m->fold ? p->aRa : p->aH, m->L[0].w1, F, d, epi_ffn1(m, *p, 0), 0, &p->f1BN);
-    if (rc == W2V_OK) rc = tune_gemm(m, &p->f2S, p->aF, m->L[0].w2, d, F, epi_resid(m, *p, 0, true), 0, &p->f2BN);
+      rc = pick_role(m, &p->oS, p->aAO, m->L[0].wo, d, d, epi_resid(m, *p, 0, false), 0, &p->oBN, g_bn(2), g_sp(2));
+    if (rc == W2V_OK)
+      rc = pick_role(m, &p->f1S, m->fold ? p->aRa : p->aH, m->L[0].w1, F, d, epi_ffn1(m, *p, 0), 0, &p->f1BN, g_bn(3),
+                     g_sp(3));
+    if (rc == W2V_OK)
+      rc = pick_role(m, &p->f2S, p->aF, m->L[0].w2, d, F, epi_resid(m, *p, 0, true), 0, &p->f2BN, g_bn(4), g_sp(4));
     if (rc != W2V_OK) return rc;
   }
   p->qkvB.resize(c.n_layers);
@@ -532,10 +604,10 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   p->f1B.resize(c.n_layers);
   p->f2B.resize(c.n_layers);
   for (int l = 0; l < c.n_layers; ++l) {
-    CUDA_OR(m, map_matrix(&p->qkvB[l], m->L[l].wqkv, 3 * d, d, p->qkvBN));
-    CUDA_OR(m, map_matrix(&p->oB[l], m->L[l].wo, d, d, p->oBN));
-    CUDA_OR(m, map_matrix(&p->f1B[l], m->L[l].w1, F, d, p->f1BN));
-    CUDA_OR(m, map_matrix(&p->f2B[l], m->L[l].w2, d, F, p->f2BN));
+    CUDA_OR(m, map_b(&p->qkvB[l], m->L[l].wqkv, 3 * d, d, p->qkvBN, form_code(p->qkvS)));
+    CUDA_OR(m, map_b(&p->oB[l], m->L[l].wo, d, d, p->oBN, form_code(p->oS)));
+    CUDA_OR(m, map_b(&p->f1B[l], m->L[l].w1, F, d, p->f1BN, form_code(p->f1S)));
+    CUDA_OR(m, map_b(&p->f2B[l], m->L[l].w2, d, F, p->f2BN, form_code(p->f2S)));
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(p->Tf), static_cast<uint64_t>(batch)};
@@ -550,7 +622,8 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   }
   p->lmS = shp(V, d);
   {
-    const int rc = tune_gemm(m, &p->lmS, p->aH, m->wlm, V, d, epi_lm(m, *p, m->tune_logits), 0, &p->lmBN);
+    const int rc = pick_role(m, &p->lmS, p->aH, m->wlm, V, d, epi_lm(m, *p, m->tune_logits), 0, &p->lmBN, g_bn(5),
+                             g_sp(5));
     if (rc != W2V_OK) return rc;
   }
   // Tuning wrote garbage into the activation buffers: nothing reads them before
@@ -559,8 +632,14 @@ int build_plan(w2v_model* m, int n, int batch, Plan* p) {
   int werr = 0;
   CUDA_OR(m, cudaMemcpy(&werr, m->err_word, sizeof(int), cudaMemcpyDeviceToHost));
   if (werr) return fail(m, W2V_ETIMEOUT, "a kernel's bounded wait gave up while tuning (code 0x%x)", werr);
-  CUDA_OR(m, map_matrix(&p->lmB, m->wlm, V, d, p->lmBN));
+  CUDA_OR(m, map_b(&p->lmB, m->wlm, V, d, p->lmBN, form_code(p->lmS)));
   return W2V_OK;
+}
+
+int build_plan(w2v_model* m, int n, int batch, Plan* p) {
+  int rc = build_frontend(m, n, batch, p, false);
+  if (rc != W2V_OK) return rc;
+  return build_encoder(m, p, nullptr);
 }
 
 int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits);
@@ -601,7 +680,7 @@ void plan_file_read(const char* path, const std::string& key, std::vector<std::p
 void plan_file_append(const char* path, const std::string& key, const Plan& p, bool layers) {
   FILE* f = std::fopen(path, "a");
   if (!f) return;
-  auto put = [&](int bn, const GemmShape& s) { std::fprintf(f, " %d:%d", bn, s.split_l2 ? -s.splits : s.splits); };
+  auto put = [&](int bn, const GemmShape& s) { std::fprintf(f, " %d:%d", bn, form_code(s)); };
   std::fputs(key.c_str(), f);
   for (int i = 1; i < 7; ++i) put(p.convBN[i], p.convS[i]);
   put(p.projBN, p.projS);
@@ -616,13 +695,18 @@ void plan_file_append(const char* path, const std::string& key, const Plan& p, b
   std::fclose(f);
 }
 
-int get_plan(w2v_model* m, int n, int batch, const Plan** out, const float* pcm, float* logits) {
+int get_plan(w2v_model* m, int n, int batch, const Plan** out, const float* pcm, float* logits,
+             cudaStream_t user_stream) {
   auto key = std::make_pair(n, batch);
   auto it = m->plans.find(key);
   if (it != m->plans.end()) {
-    *out = it->second.get();
+    it->second.used = ++m->use_tick;
+    *out = it->second.plan.get();
     return W2V_OK;
   }
+  // Building a plan times GEMM candidates on the model's own buffers: let any
+  // forward pass still queued on the caller's stream finish first.
+  CUDA_OR(m, cudaStreamSynchronize(user_stream));
   std::unique_ptr<Plan> p(new Plan());
   const char* pf = std::getenv("W2V_PLAN_FILE");
   const std::string pkey = plan_file_key(m, n, batch);
@@ -638,8 +722,18 @@ int get_plan(w2v_model* m, int n, int batch, const Plan** out, const float* pcm,
   if (rc == W2V_OK && !pinned) rc = refine_plan(m, p.get(), pcm, logits);
   if (rc != W2V_OK) return rc;
   if (pf && *pf && !pinned) plan_file_append(pf, pkey, *p, m->cfg.n_layers > 0);
+  // Bounded cache: drop the least recently used plan (graphs hold their own
+  // copies of every launch parameter, so none of them refers to a plan).
+  if (m->plans.size() >= kMaxPlans) {
+    auto lru = m->plans.end();
+    for (auto i = m->plans.begin(); i != m->plans.end(); ++i)
+      if (i->second.plan.get() != m->last_plan && (lru == m->plans.end() || i->second.used < lru->second.used)) lru = i;
+    if (lru != m->plans.end()) m->plans.erase(lru);
+  }
   *out = p.get();
-  m->plans[key] = std::move(p);
+  w2v_model::PlanEntry& pe = m->plans[key];
+  pe.plan = std::move(p);
+  pe.used = ++m->use_tick;
   return W2V_OK;
 }
 
@@ -693,16 +787,21 @@ struct Prof {
     }                                                                        \
   } while (0)
 
-// Queues the whole forward pass on `st`.
-int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits, cudaStream_t st, Prof* prof) {
+// Clips of the varlen form: clip c's n[c] samples, its frames in the packed
+// encoder rows [att.row0[c], att.row0[c] + att.len[c]).
+struct VarlenClips {
+  AttnClips att;
+  int n[kMaxVarlenClips] = {};
+};
+
+// Queues the conv feature encoder of plan p (its batch of clips of p.n
+// samples) on `st`.  The last conv layer writes packed rows [batch * Tf][512]
+// to act_a, or to out6 when given.
+int enqueue_frontend(w2v_model* m, const Plan& p, const float* pcm, __half* out6, cudaStream_t st, Prof* prof) {
   const w2v_config& c = m->cfg;
-  const int d = c.d_model, F = c.d_ffn, V = c.vocab, H = c.n_heads, B = p.batch;
+  const int B = p.batch;
   const int act = c.gelu_tanh ? 2 : 1;
   const float eps = c.ln_eps;
-  const int rows = p.rows;
-  const double R = rows, D = d, FF = F, VV = V;
-
-  // --- conv feature encoder
   if (c.conv_norm == 0) {
     LAUNCH(W2V_K_GN_MOMENTS, 130.0 * p.T[0] * B, 4.0 * p.n * B,
            launch_gn_moments(pcm, p.n, B, p.T[0], m->c0w, m->c0g, m->c0beta, eps, m->gn_partial, m->gn_ticket,
@@ -712,7 +811,8 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
          launch_conv0_tc(pcm, p.n, B, p.T[0], p.Tpad[0], m->c0wp, m->c0b, m->c0g, m->c0beta, m->gn_ss, c.conv_norm,
                          eps, act, m->act_a, m->err_word, st));
   for (int i = 1; i < 7; ++i) {
-    const GemmEpilogue e = epi_conv(m, p, i);
+    GemmEpilogue e = epi_conv(m, p, i);
+    if (i == 6 && out6) e.out = out6;
     const double K = p.convS[i].K;
     LAUNCH(W2V_K_CONV_GEMM, 2.0 * p.T[i] * kC * K * B,
            2.0 * kC * (p.T[i - 1] + p.T[i]) * B + 2.0 * kC * K,
@@ -722,7 +822,20 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
              launch_layernorm(e.out, 0, static_cast<__half*>(e.out), B * p.Tpad[i], kC, m->cg[i], m->cbeta[i], eps,
                               act, st));
   }
-  const __half* conv_out = m->act_a;  // layer 6 (even) writes act_a, packed [B*Tf][512]
+  return W2V_OK;
+}
+
+// Queues everything after the conv encoder for the p.rows packed rows of
+// conv_out: feature LN + projection, positional conv (per clip in the varlen
+// form), encoder blocks, CTC head -> logits [rows][vocab].
+int enqueue_encoder(w2v_model* m, const Plan& p, const __half* conv_out, float* logits, cudaStream_t st, Prof* prof,
+                    const VarlenClips* vl) {
+  const w2v_config& c = m->cfg;
+  const int d = c.d_model, F = c.d_ffn, V = c.vocab, H = c.n_heads, B = p.batch;
+  const int act = c.gelu_tanh ? 2 : 1;
+  const float eps = c.ln_eps;
+  const int rows = p.rows;
+  const double R = rows, D = d, FF = F, VV = V;
 
   // --- feature projection: LN(512) then Linear 512 -> d
   LAUNCH(W2V_K_FP_LN, 0.0, 4.0 * kC * R, launch_layernorm(conv_out, 0, m->ln512, rows, kC, m->fpg, m->fpb, eps, 0, st));
@@ -731,15 +844,35 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
     LAUNCH(W2V_K_PROJ_GEMM, 2.0 * R * D * kC, 2.0 * R * kC + 2.0 * D * kC + 2.0 * R * D,
            launch_gemm(p.projA, p.projB, p.projS, p.projBN, e, m->err_word, st));
   }
-  // --- positional conv + residual -> r (fp32)
-  LAUNCH(W2V_K_POSCONV, 2.0 * R * D * (D / 16) * 128, 2.0 * R * D + 2.0 * D * (D / 16) * 128 + 4.0 * R * D,
-         launch_posconv(p.posX, m->x, m->wpos, m->bpos, p.Tf, B, d, act, m->r, m->err_word, st));
+  // --- positional conv + residual -> r (fp32); zero padding at each clip's ends
+  if (!vl) {
+    LAUNCH(W2V_K_POSCONV, 2.0 * R * D * (D / 16) * 128, 2.0 * R * D + 2.0 * D * (D / 16) * 128 + 4.0 * R * D,
+           launch_posconv(p.posX, m->x, m->wpos, m->bpos, p.Tf, B, d, act, m->r, m->err_word, st));
+  } else {
+    for (int ci = 0; ci < vl->att.n; ++ci) {
+      const int T = vl->att.len[ci];
+      const size_t off = static_cast<size_t>(vl->att.row0[ci]) * d;
+      CUtensorMap tmX;
+      const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(T), 1};
+      const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(T) * d * 2};
+      const uint32_t box[3] = {8, 256, 1};
+      CUDA_OR(m, make_tmap_f16(&tmX, m->x + off, 3, dims, str, box, false));
+      const double Rc = T;
+      LAUNCH(W2V_K_POSCONV, 2.0 * Rc * D * (D / 16) * 128, 2.0 * Rc * D + 2.0 * D * (D / 16) * 128 + 4.0 * Rc * D,
+             launch_posconv(tmX, m->x + off, m->wpos, m->bpos, T, 1, d, act, m->r + off, m->err_word, st));
+    }
+  }
 
   // --- encoder blocks
   const bool stable = c.stable_layer_norm != 0;
   const double ln_bytes = 6.0 * R * D;  // fp32 in, fp16 out
   if (!stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, m->encg, m->encb, eps, 0, st));
   const double res_bytes = (stable ? 4.0 : 2.0) * R * D;
+  double att_flops = 4.0 * B * double(p.Tf) * p.Tf * D;
+  if (vl) {
+    att_flops = 0.0;
+    for (int ci = 0; ci < vl->att.n; ++ci) att_flops += 4.0 * double(vl->att.len[ci]) * vl->att.len[ci] * D;
+  }
   for (int l = 0; l < c.n_layers; ++l) {
     const LayerDev& w = m->L[l];
     if (stable) LAUNCH(W2V_K_ENC_LN, 0.0, ln_bytes, launch_layernorm(m->r, 1, m->h, rows, d, w.ln1g, w.ln1b, eps, 0, st));
@@ -748,8 +881,13 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
       LAUNCH(W2V_K_QKV_GEMM, 2.0 * R * 3 * D * D, 2.0 * R * D + 6.0 * D * D + 6.0 * R * D,
              launch_gemm(p.aH, p.qkvB[l], p.qkvS, p.qkvBN, e, m->err_word, st));
     }
-    LAUNCH(W2V_K_ATTENTION, 4.0 * B * double(p.Tf) * p.Tf * D, 8.0 * R * D,
-           launch_attention(p.attQ, p.attK, p.attVt, p.Tf, B, H, m->ao, m->err_word, st));
+    if (!vl) {
+      LAUNCH(W2V_K_ATTENTION, att_flops, 8.0 * R * D,
+             launch_attention(p.attQ, p.attK, p.attVt, p.Tf, B, H, m->ao, m->err_word, st));
+    } else {
+      LAUNCH(W2V_K_ATTENTION, att_flops, 8.0 * R * D,
+             launch_attention_varlen(p.attQ, p.attK, p.attVt, vl->att, H, m->ao, m->err_word, st));
+    }
     {
       const GemmEpilogue e = epi_resid(m, p, l, false);
       LAUNCH(W2V_K_OUT_GEMM, 2.0 * R * D * D, 2.0 * R * D + 2.0 * D * D + res_bytes + 4.0 * R * D,
@@ -780,6 +918,14 @@ int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits
            launch_gemm(p.aH, p.lmB, p.lmS, p.lmBN, e, m->err_word, st));
   }
   return W2V_OK;
+}
+
+// Queues the whole forward pass on `st`.
+int enqueue_forward(w2v_model* m, const Plan& p, const float* pcm, float* logits, cudaStream_t st, Prof* prof) {
+  int rc = enqueue_frontend(m, p, pcm, nullptr, st, prof);
+  if (rc != W2V_OK) return rc;
+  // layer 6 (even) writes act_a, packed [B*Tf][512]
+  return enqueue_encoder(m, p, m->act_a, logits, st, prof, nullptr);
 }
 
 int enqueue_ctc(w2v_model* m, const float* logits, int batch, int T, int t_valid, int32_t* tokens, int32_t* n_tokens,
@@ -1058,8 +1204,9 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   const int t0max = conv_len(c.max_samples, kKern[0], kStride[0]);
   const size_t act_rows = static_cast<size_t>(B) * (t0max + 2) + 256;
   const int tf = frames_of(c.max_samples);
-  const size_t rows = static_cast<size_t>(B) * tf + 256;
-  const size_t tpad = (tf + 7) & ~7;
+  // per-row buffers hold B clips of up to tf frames each starting on a
+  // 128-row boundary (the varlen form), plus slack for tile overhang
+  const size_t rows = static_cast<size_t>(B) * (tf + 128) + 256;
   cursor = 0;
   std::vector<std::pair<size_t, void**>> wfix;
   auto wtake = [&](void** dst, size_t bytes) {
@@ -1074,7 +1221,8 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   wtake(reinterpret_cast<void**>(&m->h), rows * d * 2);
   wtake(reinterpret_cast<void**>(&m->q), rows * d * 2);
   wtake(reinterpret_cast<void**>(&m->k), rows * d * 2);
-  wtake(reinterpret_cast<void**>(&m->vt), static_cast<size_t>(B) * d * tpad * 2 + 4096);
+  wtake(reinterpret_cast<void**>(&m->vt), static_cast<size_t>(d) * ((rows + 7) & ~static_cast<size_t>(7)) * 2 + 4096);
+  wtake(reinterpret_cast<void**>(&m->cpk), rows * kC * 2);
   wtake(reinterpret_cast<void**>(&m->ao), rows * d * 2);
   wtake(reinterpret_cast<void**>(&m->f), rows * F * 2);
   wtake(reinterpret_cast<void**>(&m->r), rows * d * 4);
@@ -1107,6 +1255,7 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     return W2V_ECUDA;
   }
   m->max_rows = static_cast<int>(B) * tf;
+  m->varlen_rows_max = static_cast<int>(B) * ((tf + 127) / 128 * 128);
   if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
     cudaFree(m->ws);
     cudaFree(m->wmem);
@@ -1125,20 +1274,18 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
 // descent; the incumbent wins ties within 0.5 %).
 namespace {
 int apply_role(w2v_model* m, Plan* p, int role, int bn, int sp) {
-  const int splits = sp < 0 ? -sp : sp;
   const int d = m->cfg.d_model, F = m->cfg.d_ffn;
   std::vector<CUtensorMap>* maps[4] = {&p->qkvB, &p->oB, &p->f1B, &p->f2B};
   int* bns[4] = {&p->qkvBN, &p->oBN, &p->f1BN, &p->f2BN};
   GemmShape* shapes[4] = {&p->qkvS, &p->oS, &p->f1S, &p->f2S};
   *bns[role] = bn;
-  shapes[role]->splits = splits;
-  shapes[role]->split_l2 = sp < 0;
+  set_form(shapes[role], sp);
   for (int l = 0; l < m->cfg.n_layers; ++l) {
     const LayerDev& w = m->L[l];
     const __half* W = role == 0 ? w.wqkv : role == 1 ? w.wo : role == 2 ? w.w1 : w.w2;
     const int N = role == 0 ? 3 * d : role == 2 ? F : d;
     const int K = role == 3 ? F : d;
-    CUDA_OR(m, map_matrix(&(*maps[role])[l], W, N, K, bn));
+    CUDA_OR(m, map_b(&(*maps[role])[l], W, N, K, bn, sp));
   }
   return W2V_OK;
 }
@@ -1190,13 +1337,14 @@ int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
     const int nk = K / 64;
     GemmShape* sh = role == 0 ? &p->qkvS : role == 1 ? &p->oS : role == 2 ? &p->f1S : &p->f2S;
     int cur_bn = role == 0 ? p->qkvBN : role == 1 ? p->oBN : role == 2 ? p->f1BN : p->f2BN;
-    int cur_s = sh->split_l2 ? -sh->splits : sh->splits;
+    int cur_s = form_code(*sh);
     for (int bn : {32, 64, 128, 192, 256}) {
       if (bn == 32 ? N > 32 : N <= bn / 2) continue;
       if (role == 0 && d % bn != 0) continue;
-      for (int sp : {1, 2, 3, 4, 6, -2, -4}) {
+      for (int sp : {1, 2, 3, 4, 6, -2, -4, 0}) {
         if (sp > 1 && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
         if (sp < 0 && !l2_split_ok(m, *sh, N, bn, -sp)) continue;
+        if (sp == 0 && bn < 64) continue;
         if (bn == cur_bn && sp == cur_s) continue;
         int rc = apply_role(m, p, role, bn, sp);
         if (rc != W2V_OK) return rc;
@@ -1229,7 +1377,7 @@ extern "C" int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, in
   if (cudaSetDevice(m->device) != cudaSuccess) return fail(m, W2V_ECUDA, "cudaSetDevice failed");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Plan* p = nullptr;
-  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev);
+  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev, st);
   if (rc != W2V_OK) return rc;
   m->last_plan = p;
   if (!m->cfg.use_cuda_graph) {
@@ -1242,11 +1390,18 @@ extern "C" int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, in
   auto key = std::make_tuple(n_samples, batch, static_cast<const void*>(pcm_dev), static_cast<void*>(logits_dev));
   auto it = m->graphs.find(key);
   if (it == m->graphs.end()) {
+    if (m->graphs.size() >= kMaxGraphs) {
+      // An executable graph still running on a stream is freed once it completes.
+      auto lru = m->graphs.begin();
+      for (auto i = m->graphs.begin(); i != m->graphs.end(); ++i)
+        if (i->second.used < lru->second.used) lru = i;
+      cudaGraphExecDestroy(lru->second.exec);
+      m->graphs.erase(lru);
+    }
     cudaGraph_t g = nullptr;
     CUDA_OR(m, cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
     Prof counter;
     rc = enqueue_forward(m, *p, pcm_dev, logits_dev, m->cap_stream, &counter);
-    m->graph_launches[key] = counter.launches;
     cudaError_t e = cudaStreamEndCapture(m->cap_stream, &g);
     if (rc != W2V_OK) {
       if (g) cudaGraphDestroy(g);
@@ -1257,10 +1412,14 @@ extern "C" int w2v_forward(w2v_model* m, const float* pcm_dev, int n_samples, in
     e = cudaGraphInstantiate(&ex, g, 0);
     cudaGraphDestroy(g);
     if (e != cudaSuccess) return fail(m, W2V_ECUDA, "graph instantiate: %s", cudaGetErrorString(e));
-    it = m->graphs.emplace(key, ex).first;
+    w2v_model::GraphEntry ge;
+    ge.exec = ex;
+    ge.launches = counter.launches;
+    it = m->graphs.emplace(key, ge).first;
   }
-  CUDA_OR(m, cudaGraphLaunch(it->second, st));
-  m->last_launches = m->graph_launches[key];
+  it->second.used = ++m->use_tick;
+  CUDA_OR(m, cudaGraphLaunch(it->second.exec, st));
+  m->last_launches = it->second.launches;
   return W2V_OK;
 }
 
@@ -1276,6 +1435,165 @@ extern "C" int w2v_ctc_greedy(w2v_model* m, const float* logits_dev, int batch, 
   CUDA_OR(m, cudaSetDevice(m->device));
   return enqueue_ctc(m, logits_dev, batch, T, t_valid, tokens_dev, n_tokens_dev, static_cast<cudaStream_t>(stream),
                      nullptr);
+}
+
+// ----------------------------------------------------------- varlen form
+namespace {
+
+// Inserts a plan into the model's bounded plan cache (least recently used out).
+const Plan* cache_plan(w2v_model* m, std::pair<int, int> key, std::unique_ptr<Plan> p) {
+  if (m->plans.size() >= kMaxPlans) {
+    auto lru = m->plans.end();
+    for (auto i = m->plans.begin(); i != m->plans.end(); ++i)
+      if (i->second.plan.get() != m->last_plan && (lru == m->plans.end() || i->second.used < lru->second.used)) lru = i;
+    if (lru != m->plans.end()) m->plans.erase(lru);
+  }
+  w2v_model::PlanEntry& pe = m->plans[key];
+  pe.plan = std::move(p);
+  pe.used = ++m->use_tick;
+  return pe.plan.get();
+}
+
+const Plan* find_plan(w2v_model* m, std::pair<int, int> key) {
+  auto it = m->plans.find(key);
+  if (it == m->plans.end()) return nullptr;
+  it->second.used = ++m->use_tick;
+  return it->second.plan.get();
+}
+
+// Conv-encoder plan of one clip of n samples (tile choices from the cost
+// model, so a new length never times anything); cache key (n, 0).
+int varlen_frontend_plan(w2v_model* m, int n, const Plan** out) {
+  const auto key = std::make_pair(n, 0);
+  if ((*out = find_plan(m, key))) return W2V_OK;
+  std::unique_ptr<Plan> p(new Plan());
+  const int rc = build_frontend(m, n, 1, p.get(), true);
+  if (rc != W2V_OK) return rc;
+  *out = cache_plan(m, key, std::move(p));
+  return W2V_OK;
+}
+
+// Encoder plan over `rows` packed rows (one pseudo-clip of all of them); its
+// tile choices are timed once per bucket of 512 rows and reused for every row
+// count in the bucket.  Cache key (-rows, 0).
+int varlen_encoder_plan(w2v_model* m, int rows, cudaStream_t user_stream, const Plan** out) {
+  const auto key = std::make_pair(-rows, 0);
+  if ((*out = find_plan(m, key))) return W2V_OK;
+  std::unique_ptr<Plan> p(new Plan());
+  p->n = 0;
+  p->batch = 1;
+  p->Tf = rows;
+  p->rows = rows;
+  p->t_pad = (rows + 7) & ~7;
+  const int bucket = (rows + 511) / 512;
+  auto it = m->varlen_choices.find(bucket);
+  int rc;
+  if (it != m->varlen_choices.end()) {
+    int given[6][2];
+    for (int i = 0; i < 6; ++i) {
+      given[i][0] = it->second[i][0];
+      given[i][1] = it->second[i][1];
+    }
+    rc = build_encoder(m, p.get(), given);
+  } else {
+    // timing candidates uses the model's buffers: wait for queued work first
+    CUDA_OR(m, cudaStreamSynchronize(user_stream));
+    rc = build_encoder(m, p.get(), nullptr);
+    if (rc == W2V_OK) {
+      auto sp = [](const GemmShape& s) { return form_code(s); };
+      std::array<std::array<int, 2>, 6> ch = {{{p->projBN, sp(p->projS)}, {p->qkvBN, sp(p->qkvS)},
+                                               {p->oBN, sp(p->oS)}, {p->f1BN, sp(p->f1S)}, {p->f2BN, sp(p->f2S)},
+                                               {p->lmBN, sp(p->lmS)}}};
+      m->varlen_choices[bucket] = ch;
+    }
+  }
+  if (rc != W2V_OK) return rc;
+  *out = cache_plan(m, key, std::move(p));
+  return W2V_OK;
+}
+
+}  // namespace
+
+extern "C" int w2v_forward_varlen(w2v_model* m, const float* pcm_dev, const int* n_samples, int batch,
+                                  float* logits_dev, void* stream) {
+  if (!m) return W2V_EINVAL;
+  if (!pcm_dev || !logits_dev || !n_samples) return fail(m, W2V_EINVAL, "null pointer");
+  if (!aligned16(pcm_dev) || !aligned16(logits_dev)) return fail(m, W2V_EINVAL, "pointers must be 16-byte aligned");
+  const int max_clips = std::min(m->cfg.max_batch, kMaxVarlenClips);
+  if (batch < 1 || batch > max_clips) return fail(m, W2V_ESHAPE, "batch=%d outside [1, %d]", batch, max_clips);
+  VarlenClips vl;
+  vl.att.n = batch;
+  int rows = 0, qt = 0;
+  for (int c = 0; c < batch; ++c) {
+    const int n = n_samples[c];
+    if (n < 400 || n > m->cfg.max_samples)
+      return fail(m, W2V_ESHAPE, "n_samples[%d]=%d outside [400, %d]", c, n, m->cfg.max_samples);
+    const int T = frames_of(n);
+    vl.n[c] = n;
+    vl.att.row0[c] = rows;
+    vl.att.len[c] = T;
+    vl.att.qt0[c] = qt;
+    qt += (T + 127) / 128;
+    rows += (T + 127) / 128 * 128;
+  }
+  vl.att.qt0[batch] = qt;
+  if (rows > m->varlen_rows_max) return fail(m, W2V_ESHAPE, "packed rows %d > %d", rows, m->varlen_rows_max);
+  CUDA_OR(m, cudaSetDevice(m->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Plan* ep = nullptr;
+  int rc = varlen_encoder_plan(m, rows, st, &ep);
+  if (rc != W2V_OK) return rc;
+  std::vector<const Plan*> fps(batch);
+  for (int c = 0; c < batch; ++c) {
+    rc = varlen_frontend_plan(m, vl.n[c], &fps[c]);
+    if (rc != W2V_OK) return rc;
+  }
+  Prof counter;
+  int64_t off = 0;
+  for (int c = 0; c < batch; ++c) {
+    rc = enqueue_frontend(m, *fps[c], pcm_dev + off, m->cpk + static_cast<size_t>(vl.att.row0[c]) * kC, st, &counter);
+    if (rc != W2V_OK) return rc;
+    off += vl.n[c];
+  }
+  rc = enqueue_encoder(m, *ep, m->cpk, m->tune_logits, st, &counter, &vl);
+  if (rc != W2V_OK) return rc;
+  // clip c's logits rows [row0, row0 + T) -> rows [sum of earlier T, + T) of the output
+  const size_t V = m->cfg.vocab;
+  size_t dst = 0;
+  for (int c = 0; c < batch; ++c) {
+    const size_t T = vl.att.len[c];
+    CUDA_OR(m, cudaMemcpyAsync(logits_dev + dst * V, m->tune_logits + static_cast<size_t>(vl.att.row0[c]) * V,
+                               T * V * sizeof(float), cudaMemcpyDeviceToDevice, st));
+    dst += T;
+  }
+  m->last_plan = nullptr;  // intermediate buffers hold packed clips: nothing for w2v_debug_read
+  m->last_launches = counter.launches;
+  return W2V_OK;
+}
+
+extern "C" int w2v_ctc_greedy_varlen(w2v_model* m, const float* logits_dev, const int* frames, int batch,
+                                     int32_t* tokens_dev, int32_t* n_tokens_dev, void* stream) {
+  if (!m) return W2V_EINVAL;
+  if (!logits_dev || !frames || !tokens_dev || !n_tokens_dev) return fail(m, W2V_EINVAL, "null pointer");
+  if (!aligned16(logits_dev) || !aligned16(tokens_dev) || !aligned16(n_tokens_dev))
+    return fail(m, W2V_EINVAL, "pointers must be 16-byte aligned");
+  if (batch < 1 || batch > m->cfg.max_batch) return fail(m, W2V_ESHAPE, "batch=%d outside [1, %d]", batch, m->cfg.max_batch);
+  int64_t total = 0;
+  for (int c = 0; c < batch; ++c) {
+    if (frames[c] < 0) return fail(m, W2V_ESHAPE, "frames[%d]=%d < 0", c, frames[c]);
+    total += frames[c];
+  }
+  if (total > m->max_rows) return fail(m, W2V_ESHAPE, "%lld frames in all > %d", static_cast<long long>(total), m->max_rows);
+  CUDA_OR(m, cudaSetDevice(m->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUDA_OR(m, launch_argmax(logits_dev, static_cast<int>(total), m->cfg.vocab, m->ids, st));
+  int64_t off = 0;
+  for (int c = 0; c < batch; ++c) {
+    CUDA_OR(m, launch_ctc_collapse(m->ids + off, 1, frames[c], frames[c], m->cfg.blank_id, tokens_dev + off,
+                                   n_tokens_dev + c, st));
+    off += frames[c];
+  }
+  return W2V_OK;
 }
 
 extern "C" int w2v_sync(w2v_model* m, void* stream) {
@@ -1329,7 +1647,7 @@ extern "C" int w2v_last_error(w2v_model* m, char* buf, size_t len) {
 extern "C" void w2v_destroy(w2v_model* m) {
   if (!m) return;
   cudaSetDevice(m->device);
-  for (auto& g : m->graphs) cudaGraphExecDestroy(g.second);
+  for (auto& g : m->graphs) cudaGraphExecDestroy(g.second.exec);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   if (m->pcm_stage) cudaFree(m->pcm_stage);
   if (m->logits_stage) cudaFree(m->logits_stage);
@@ -1359,7 +1677,7 @@ extern "C" int w2v_profile_forward(w2v_model* m, const float* pcm_dev, int n_sam
   CUDA_OR(m, cudaSetDevice(m->device));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Plan* p = nullptr;
-  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev);
+  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev, st);
   if (rc != W2V_OK) return rc;
   m->last_plan = p;
   Prof prof;
@@ -1402,7 +1720,7 @@ extern "C" int w2v_time_class(w2v_model* m, const float* pcm_dev, int n_samples,
   CUDA_OR(m, cudaSetDevice(m->device));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Plan* p = nullptr;
-  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev);
+  int rc = get_plan(m, n_samples, batch, &p, pcm_dev, logits_dev, st);
   if (rc != W2V_OK) return rc;
   // Record `reps` passes of only this class's launches as one graph.
   Prof filt;
@@ -1505,6 +1823,8 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   s.M = M; s.N = N; s.K = K; s.a_kwrap = K; s.batch = 1;
   if (bn == 0) {
     bn = gemm_pick(&s, 0);
+  } else if (splits == 0) {
+    s.pair = true;
   } else {
     s.splits = splits < 0 ? -splits : splits;
     s.split_l2 = splits < 0;
@@ -1512,9 +1832,10 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   if (bn != 32 && bn != 64 && bn != 128 && bn != 192 && bn != 256) return W2V_EINVAL;
   if (s.splits < 1 || s.splits > 8 || s.splits > K / 64) return W2V_EINVAL;
   if (s.split_l2 && ((s.splits != 2 && s.splits != 4) || bn < 64)) return W2V_EINVAL;
+  if (s.pair && bn < 64) return W2V_EINVAL;
   CUtensorMap ta, tb;
   if (map_a(&ta, A, K, M, K, 1, 0) != cudaSuccess) return W2V_ECUDA;
-  if (map_matrix(&tb, B, N, K, bn) != cudaSuccess) return W2V_ECUDA;
+  if (map_matrix(&tb, B, N, K, s.pair ? bn / 2 : bn) != cudaSuccess) return W2V_ECUDA;
   GemmEpilogue e;
   e.bias = bias;
   e.residual = residual;

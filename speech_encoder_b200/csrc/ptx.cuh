@@ -182,6 +182,68 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// ------------------------------------------- CTA pairs (tcgen05 cta_group::2)
+// A pair of CTAs (ranks 2i and 2i+1 of a cluster) computes one M = 256 tile:
+// each CTA holds 128 rows of A and half of the N columns of B in its own
+// shared memory at the same offsets, and 128 rows of the accumulator in its
+// own TMEM at the same column address.  The even CTA issues the MMAs.
+
+// TMEM allocation, permit release and free for the pair: executed by the same
+// warp of both CTAs, with the same destination slot offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[256 rows: 128 per CTA] * B[N: N/2 per CTA]^T.
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives once on the mbarrier at the same offset in every CTA of cta_mask
+// when the pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// TMA tile loads of a pair member into its own shared memory, completing on
+// the mbarrier at shared::cluster address bar_cluster (the even CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int x, int y,
+                                                 int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Loads 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (one lane
 // per thread) and waits for the load to complete.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -395,21 +457,30 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // GELU, exact form x * Phi(x) through the CUDA erff, or the tanh form.
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
-// tanh-form GELU, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi) (x + 0.044715 x^3),
-// evaluated through the identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)):
-// one ex2.approx and one rcp.approx (relative errors ~2^-22), no cancellation
-// for negative x (unlike 1 + tanh(u) near -1).
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// tanh-form GELU, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi) (x + 0.044715 x^3),
+// with one hardware tanh (a single exponent-unit operation; the epilogues
+// that apply GELU to whole output tiles are bound by that unit, which the
+// sigmoid form 1 / (1 + exp(-2u)) needs twice).  The error is the tanh
+// approximation's, scaled by 0.5 |x|: for negative x the result is a small
+// difference 0.5 x + 0.5 x tanh(u), whose absolute error stays below
+// 0.5 |x| |tanh(u)| times tanh's relative error.
 __device__ __forceinline__ float gelu_tanh(float x) {
-  const float k2 = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2(e)
-  const float u = x * fmaf(0.044715f * x, x, 1.0f);
-  const float e = ex2_approx(k2 * u);  // exp(-2 sqrt(2/pi) (x + 0.044715 x^3))
-  return x * rcp_approx(1.0f + e);
+  const float k = 0.7978845608028654f;  // sqrt(2/pi)
+  const float u = x * fmaf(0.044715f * k, x * x, k);
+  const float hx = 0.5f * x;
+  return fmaf(hx, tanh_approx(u), hx);
 }
 
 // Packed fp32 pair arithmetic (one f32x2 instruction for two lanes of data).

@@ -116,6 +116,8 @@ struct GemmDims {
 struct GemmShape : GemmDims {
   bool split_l2 = false;  // or, with splits 2 or 4, through the L2 scratch of
                           // GemmEpilogue (TMA stores and loads of fp32 boxes)
+  bool pair = false;      // CTA pairs on 256-row tiles (2-CTA tensor-core
+                          // instructions); then tmB's box is {64, bn/2}, no split
 };
 
 // Chooses the N tile width (returned) and the split-K factor (s->splits) for
@@ -169,6 +171,19 @@ cudaError_t launch_posconv(const CUtensorMap& tmX, const __half* x, const __half
 // tmQ/tmK: {d, T, batch} box {64,128,1} SW128; tmVt: {T, batch*H*64} box {64,64} SW128.
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt, int T,
                              int batch, int H, __half* out, int* err, cudaStream_t st);
+// Clips of different lengths in one launch: clip c has len[c] frames at rows
+// row0[c] (a multiple of 128) of the packed Q/K/out matrices and columns
+// row0[c] of V^T; its query tiles are qt0[c] .. qt0[c+1]-1 of the grid.
+// tmQ/tmK: {d, rows, 1} box {64,128,1}; tmVt: {rows, H*64} box {64,64}.
+constexpr int kMaxVarlenClips = 64;
+struct AttnClips {
+  int n = 0;
+  int row0[kMaxVarlenClips] = {};
+  int len[kMaxVarlenClips] = {};
+  int qt0[kMaxVarlenClips + 1] = {};
+};
+cudaError_t launch_attention_varlen(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt,
+                                    const AttnClips& clips, int H, __half* out, int* err, cudaStream_t st);
 
 // ----------------------------------------------------------------------- CTC
 cudaError_t launch_argmax(const float* logits, int rows, int V, int32_t* ids, cudaStream_t st);

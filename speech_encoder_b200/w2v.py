@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         "w2v_forward": (I, [VP, VP, I, I, VP, VP]),
         "w2v_ctc_greedy": (I, [VP, VP, I, I, I, VP, VP, VP]),
         "w2v_sync": (I, [VP, VP]),
+        "w2v_forward_varlen": (I, [VP, VP, ctypes.POINTER(I), I, VP, VP]),
+        "w2v_ctc_greedy_varlen": (I, [VP, VP, ctypes.POINTER(I), I, VP, VP, VP]),
         "w2v_debug_read": (I, [VP, I, VP, SZ, ctypes.POINTER(SZ), VP]),
         "w2v_last_error": (I, [VP, ctypes.c_char_p, SZ]),
         "w2v_destroy": (None, [VP]),
@@ -201,6 +203,23 @@ def w2v_create(cfg: w2v_config, blob: np.ndarray) -> int:
 def w2v_forward(model: int, pcm, n_samples: int, batch: int, logits, stream=None) -> None:
     _check(lib().w2v_forward(model, _ptr(pcm), int(n_samples), int(batch), _ptr(logits), _stream(stream)), model,
            "w2v_forward")
+
+
+def _int_array(values):
+    vals = [int(v) for v in values]
+    return (ctypes.c_int * len(vals))(*vals), len(vals)
+
+
+def w2v_forward_varlen(model: int, pcm, n_samples, logits, stream=None) -> None:
+    arr, n = _int_array(n_samples)
+    _check(lib().w2v_forward_varlen(model, _ptr(pcm), arr, n, _ptr(logits), _stream(stream)), model,
+           "w2v_forward_varlen")
+
+
+def w2v_ctc_greedy_varlen(model: int, logits, frames, tokens, n_tokens, stream=None) -> None:
+    arr, n = _int_array(frames)
+    _check(lib().w2v_ctc_greedy_varlen(model, _ptr(logits), arr, n, _ptr(tokens), _ptr(n_tokens), _stream(stream)),
+           model, "w2v_ctc_greedy_varlen")
 
 
 def w2v_ctc_greedy(model: int, logits, batch: int, T: int, t_valid: int, tokens, n_tokens, stream=None) -> None:
@@ -351,6 +370,32 @@ class Model:
             n_tokens = torch.empty((batch,), dtype=torch.int32, device=logits.device)
         w2v_ctc_greedy(self.handle, logits, batch, T, t_valid, tokens, n_tokens, stream)
         return tokens, n_tokens
+
+    def forward_varlen(self, clips, logits=None, stream=None):
+        """clips: list of 1-D float32 CUDA tensors (one per clip, any lengths).
+        Returns (logits [sum T_c, vocab], frames [T_c])."""
+        import torch
+        lens = [int(c.numel()) for c in clips]
+        frames = [w2v_num_frames(n) for n in lens]
+        pcm = torch.cat([c.reshape(-1) for c in clips]).contiguous()
+        if logits is None:
+            logits = torch.empty((sum(frames), self.shape.vocab), dtype=torch.float32, device=pcm.device)
+        w2v_forward_varlen(self.handle, pcm, lens, logits, stream)
+        return logits, frames
+
+    def ctc_greedy_varlen(self, logits, frames, stream=None):
+        """Tokens of each clip of a packed forward_varlen output: a list of int32
+        CUDA tensors (one per clip), after a stream sync."""
+        import torch
+        tokens = torch.empty((max(sum(frames), 1),), dtype=torch.int32, device=logits.device)
+        n_tokens = torch.empty((len(frames),), dtype=torch.int32, device=logits.device)
+        w2v_ctc_greedy_varlen(self.handle, logits, frames, tokens, n_tokens, stream)
+        self.sync(stream)
+        out, off = [], 0
+        for c, T in enumerate(frames):
+            out.append(tokens[off:off + int(n_tokens[c])])
+            off += T
+        return out
 
     def sync(self, stream=None):
         w2v_sync(self.handle, stream)
