@@ -404,13 +404,19 @@ def measure_workload(name, steps, warmup, tc_peak, dev, flush, cpu_budget_s=10.0
            "tensor_frac_of_step": flops / (ms * 1e-3) / 1e12 / tc_peak}
     if name != "c4":
         # per-class kernel times, as for the headline workload
-        us_t, fl_t = 0.0, 0.0
+        us_t, fl_t, per = 0.0, 0.0, {}
         bsz, n = w.calls[0][0].shape
-        for cls in TENSOR_CLASSES:
+        for cls in B.KERNEL_CLASSES:
             us, nl, fl, _ = B.w2v_time_class(model.handle, pcm, n, bsz, logits, cls, reps=5, stream=stream)
-            us_t += us * nl
-            fl_t += fl * nl
+            if not nl:
+                continue
+            per[cls] = {"us_per_launch": round(us, 2), "launches_per_step": nl, "ms_per_step": round(us * nl / 1000, 4)}
+            if cls in TENSOR_CLASSES:
+                us_t += us * nl
+                fl_t += fl * nl
+                per[cls]["frac_tensor"] = round(fl / (us * 1e-6) / 1e12 / tc_peak, 4)
         out["tensor_frac_all_contractions"] = fl_t / (us_t * 1e-6) / 1e12 / tc_peak
+        out["kernels"] = dict(sorted(per.items(), key=lambda kv: -kv[1]["ms_per_step"]))
     model.close()
     # the oracle on a bounded sample of the same workload (host cores)
     from oracle import w2v_oracle as O

@@ -77,41 +77,15 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// The residual of 4 consecutive columns [col, col+4) of row grow, as stored
-// (before any LayerNorm), zeros where there is none.  `vec` selects 16-/8-byte
-// loads (row starts and pointers 16-byte aligned, full 4-vector in range).
-// Split from the arithmetic so that an epilogue can issue these loads long
-// before the accumulator is ready.
-__device__ __forceinline__ float4 load_res4(const GemmEpiArgs& e, int bzb, int grow, int col, int nv, bool vec) {
-  float rv[4] = {0.f, 0.f, 0.f, 0.f};
-  if (e.residual) {
-    const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
-    if (e.res_f32) {
-      const float* rp = static_cast<const float*>(e.residual) + roff;
-      if (vec && nv == 4) return *reinterpret_cast<const float4*>(rp);
-      for (int i = 0; i < nv; ++i) rv[i] = rp[i];
-    } else {
-      const __half* rp = static_cast<const __half*>(e.residual) + roff;
-      if (vec && nv == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(rp);
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-        return make_float4(a.x, a.y, b.x, b.y);
-      }
-      for (int i = 0; i < nv; ++i) rv[i] = __half2float(rp[i]);
-    }
-  }
-  return make_float4(rv[0], rv[1], rv[2], rv[3]);
-}
-
 // Final epilogue for 4 consecutive columns [col, col+4) of row grow: bias
-// (from shared memory), GELU, the residual `res` (from load_res4), store.
+// (from shared memory), GELU, residual, store.  `vec` selects 16-/8-byte
+// accesses (row starts and pointers 16-byte aligned, full 4-vector in range).
 // lnr: the row's LayerNorm factors (rstd, -mean * rstd) when e.ln_mode != 0;
 // vec_s: the LN column vectors of this tile (ln_mode 1: column sums; 2: gamma,
 // then beta at vec_s + BN).
-__device__ __forceinline__ void finish4r(float (&x)[4], float4 res, const float* bias_s, const float* vec_s, int bn,
-                                         float2 lnr, int lcol, int grow, int col, int nv, int bzb,
-                                         const GemmEpiArgs& e, void* outp, int ocol0, bool vec) {
+__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, const float* vec_s, int bn, float2 lnr,
+                                        int lcol, int grow, int col, int nv, int bzb, const GemmEpiArgs& e,
+                                        void* outp, int ocol0, bool vec) {
   const int ln_mode = e.ln_cfg & 255;
   if (ln_mode == 1) {
 #pragma unroll
@@ -120,7 +94,27 @@ __device__ __forceinline__ void finish4r(float (&x)[4], float4 res, const float*
 #pragma unroll
   for (int i = 0; i < 4; ++i) x[i] = apply_act(x[i] + bias_s[lcol + i], e.act);
   if (e.residual) {
-    float rv[4] = {res.x, res.y, res.z, res.w};
+    const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+    float rv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (e.res_f32) {
+      const float* rp = static_cast<const float*>(e.residual) + roff;
+      if (vec && nv == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(rp);
+        rv[0] = t.x; rv[1] = t.y; rv[2] = t.z; rv[3] = t.w;
+      } else {
+        for (int i = 0; i < nv; ++i) rv[i] = rp[i];
+      }
+    } else {
+      const __half* rp = static_cast<const __half*>(e.residual) + roff;
+      if (vec && nv == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(rp);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        rv[0] = a.x; rv[1] = a.y; rv[2] = b.x; rv[3] = b.y;
+      } else {
+        for (int i = 0; i < nv; ++i) rv[i] = __half2float(rp[i]);
+      }
+    }
     if (ln_mode == 2) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) rv[i] = fmaf(fmaf(rv[i], lnr.x, lnr.y), vec_s[lcol + i], vec_s[bn + lcol + i]);
@@ -142,13 +136,6 @@ __device__ __forceinline__ void finish4r(float (&x)[4], float4 res, const float*
     else
       for (int i = 0; i < nv; ++i) op[i] = __float2half_rn(x[i]);
   }
-}
-
-__device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, const float* vec_s, int bn, float2 lnr,
-                                        int lcol, int grow, int col, int nv, int bzb, const GemmEpiArgs& e,
-                                        void* outp, int ocol0, bool vec) {
-  finish4r(x, load_res4(e, bzb, grow, col, nv, vec), bias_s, vec_s, bn, lnr, lcol, grow, col, nv, bzb, e, outp,
-           ocol0, vec);
 }
 
 // mode: 0 generic, 1 direct (TMA store), 2 split-K through distributed shared
@@ -372,14 +359,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int region = e.qkv_d > 0 ? n0 / e.qkv_d : -1;
   const bool vec = vec_ok != 0;
   const int ln_mode = e.ln_cfg & 255;
-  // Owner rows per CTA in the distributed-shared-memory split form are at
-  // most 64 (S >= 2); for tiles up to 128 wide every thread finishes at most
-  // kIter2 4-column chunks of them, few enough to prefetch into registers.
-  constexpr int kIter2 = (64 * C::ROW_CHUNKS + kEpiThreads - 1) / kEpiThreads;
-  constexpr bool kPre2 = kIter2 <= 8;
-  float4 resv[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) resv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   bool ok = true;
   if (epi) {
     for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (e.bias && n0 + i < s.N) ? e.bias[n0 + i] : 0.f;
@@ -422,32 +401,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           f = make_float2(rstd, -mean * rstd);
         }
         rowln_s[et] = f;
-      }
-    }
-    // Residual values this thread adds, loaded now while the mainloop runs
-    // (they come from earlier kernels): in the direct form the first 32-column
-    // chunk of its row, in the distributed-shared-memory split form every
-    // 4-column chunk of the rows its CTA finishes.
-    if (e.residual && region <= 0) {
-      pdl_wait();
-      if (mode == 1 || (SPLIT && mode == 3 && (q * S) / 4 == split)) {
-        const int grow = m0 + r;
-        const int col0 = n0 + half * (BN / 2);
-        if (grow < s.M) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) resv[i] = load_res4(e, bzb, grow, col0 + 4 * i, min(4, s.N - col0 - 4 * i), vec);
-        }
-      } else if (SPLIT && mode == 2 && kPre2) {
-        const int rank = static_cast<int>(cluster_ctarank());
-        const int r0 = rank * C::BM / S;
-        const int nrows = (rank + 1) * C::BM / S - r0;
-#pragma unroll
-        for (int it = 0; it < kIter2; ++it) {
-          const int idx = et + kEpiThreads * it;
-          const int lr = idx / C::ROW_CHUNKS, j = idx % C::ROW_CHUNKS;
-          const int grow = m0 + r0 + lr, col = n0 + 4 * j;
-          if (lr < nrows && grow < s.M && col < s.N) resv[it] = load_res4(e, bzb, grow, col, min(4, s.N - col), vec);
-        }
       }
     }
     ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
@@ -677,23 +630,51 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         const int col = n0 + c;
         if (e.residual && grow < s.M) {
-          // the first chunk's residual was loaded during the mainloop
-          float4 rq[8];
-          if (c == half * (BN / 2)) {
+          const int64_t roff =
+              static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+          const int nv = min(32, s.N - col);
+          if (e.res_f32) {
+            const float* rp = static_cast<const float*>(e.residual) + roff;
+            if (nv == 32) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) rq[i] = resv[i];
+              for (int i = 0; i < 32; i += 4) {
+                const float4 rv = *reinterpret_cast<const float4*>(rp + i);
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + rv.x;
+                v[i + 1] = apply_act(v[i + 1] + bias_s[c + i + 1], e.act) + rv.y;
+                v[i + 2] = apply_act(v[i + 2] + bias_s[c + i + 2], e.act) + rv.z;
+                v[i + 3] = apply_act(v[i + 3] + bias_s[c + i + 3], e.act) + rv.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + (i < nv ? rp[i] : 0.f);
+            }
           } else {
+            const __half* rp = static_cast<const __half*>(e.residual) + roff;
+            if (nv == 32) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) rq[i] = load_res4(e, bzb, grow, col + 4 * i, min(4, s.N - col - 4 * i), vec);
-          }
+              for (int i = 0; i < 32; i += 8) {
+                const uint4 u = *reinterpret_cast<const uint4*>(rp + i);
+                const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float f[4] = {rq[i].x, rq[i].y, rq[i].z, rq[i].w};
+                for (int k = 0; k < 4; ++k) {
+                  float2 f = __half22float2(h[k]);
+                  if (ln_mode == 2) {
+                    const int cc = c + i + 2 * k;
+                    f.x = fmaf(fmaf(f.x, lnr.x, lnr.y), vec_s[cc], vec_s[BN + cc]);
+                    f.y = fmaf(fmaf(f.y, lnr.x, lnr.y), vec_s[cc + 1], vec_s[BN + cc + 1]);
+                  }
+                  v[i + 2 * k] = apply_act(v[i + 2 * k] + bias_s[c + i + 2 * k], e.act) + f.x;
+                  v[i + 2 * k + 1] = apply_act(v[i + 2 * k + 1] + bias_s[c + i + 2 * k + 1], e.act) + f.y;
+                }
+              }
+            } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int cc = c + 4 * i + k;
-              if (ln_mode == 2) f[k] = fmaf(fmaf(f[k], lnr.x, lnr.y), vec_s[cc], vec_s[BN + cc]);
-              v[4 * i + k] = apply_act(v[4 * i + k] + bias_s[cc], e.act) + f[k];
+              for (int i = 0; i < 32; ++i) {
+                float f = i < nv ? __half2float(rp[i]) : 0.f;
+                if (ln_mode == 2) f = fmaf(fmaf(f, lnr.x, lnr.y), vec_s[c + i], vec_s[BN + c + i]);
+                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + f;
+              }
             }
           }
         } else {
@@ -798,50 +779,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(apply_act(x[i] + bias_s[4 * j + i], e.act));
-        }
-      } else if (kPre2) {
-        // Chunk idx = et + 256 it of the owner rows (row idx / RC, chunk
-        // idx % RC): all residual loads were issued during the mainloop.  With
-        // row sums to store, the RC consecutive lanes of a row (a whole warp
-        // for 128-wide tiles) add up its two half-tile sums in a fixed order.
-        void* outp = region == 1 ? e.out_k : e.out;
-        const int ocol0 = region > 0 ? region * e.qkv_d : 0;
-        constexpr int RC = C::ROW_CHUNKS;
-        constexpr int GROUP = RC >= 32 ? 32 : RC;
-#pragma unroll
-        for (int it = 0; it < kIter2; ++it) {
-          const int idx = et + kEpiThreads * it;
-          const int lr = idx / RC, j = idx % RC;
-          const int grow = m0 + r0 + lr, col = n0 + 4 * j;
-          const bool row_live = lr < nrows && grow < s.M;
-          const bool live = row_live && col < s.N;
-          float p1 = 0.f, p2 = 0.f;
-          if (live) {
-            const int nv = min(4, s.N - col);
-            const float4 v = fetch(lr, j);
-            float x[4] = {v.x, v.y, v.z, v.w};
-            finish4r(x, resv[it], bias_s, vec_s, BN, row_lnr(r0 + lr), 4 * j, grow, col, nv, bzb, e, outp, ocol0,
-                     vec);
-            for (int i = 0; i < nv; ++i) {
-              p1 += x[i];
-              p2 = fmaf(x[i], x[i], p2);
-            }
-          }
-          if (e.ln_out) {
-            const bool lo = 4 * j < BN / 2;
-            float a1 = lo ? p1 : 0.f, a2 = lo ? p2 : 0.f, b1 = lo ? 0.f : p1, b2 = lo ? 0.f : p2;
-#pragma unroll
-            for (int o = GROUP / 2; o > 0; o >>= 1) {
-              a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-              a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-              b1 += __shfl_xor_sync(0xffffffffu, b1, o);
-              b2 += __shfl_xor_sync(0xffffffffu, b2, o);
-            }
-            if (row_live && j == 0) {
-              e.ln_out[static_cast<int64_t>(2 * blockIdx.y) * s.M + grow] = make_float2(a1, a2);
-              e.ln_out[static_cast<int64_t>(2 * blockIdx.y + 1) * s.M + grow] = make_float2(b1, b2);
-            }
-          }
         }
       } else {
         void* outp = region == 1 ? e.out_k : e.out;
@@ -957,10 +894,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 //  * MMA time per CTA: per 64-deep K block the larger of the MMA time
 //    (2*BN cycles for M=128) and the shared-memory operand reads
 //    ((16 KB + BN*128 B) at 128 B/cycle), times waves of CTAs;
-//  * operand delivery: every CTA streams its A and B blocks from L2; the
-//    measured aggregate L2->SM throughput of these kernels is ~4.6 KB/cycle
-//    (~8.8 TB/s) and one SM takes in at most ~110 B/cycle, so both the total
-//    and the per-CTA operand bytes give floors;
+//  * operand delivery: every CTA streams its A and B blocks from L2, and one
+//    SM takes in about 72 B/cycle of TMA traffic whatever the number of SMs
+//    streaming (measured on this B200 with a copy-only kernel: 148 SMs
+//    together reach ~21 TB/s from L2), so the per-CTA operand bytes give the
+//    floor;
 //  * fixed costs: set-up, the epilogue (split S ways), the cluster reduction.
 int gemm_pick(GemmShape* s, int bn_divides) {
   const int cands[] = {32, 64, 128, 192, 256};
@@ -980,10 +918,8 @@ int gemm_pick(GemmShape* s, int bn_divides) {
       const long nkl = (nk + sp - 1) / sp;
       const double per_k = (2.0 * bn > 128.0 + bn) ? 2.0 * bn : 128.0 + bn;
       const double t_mma = waves * nkl * per_k;
-      const double t_l2 = static_cast<double>(ctas) * nkl * (128.0 + bn) * 128.0 / 4600.0;
-      const double t_sm = waves * nkl * (128.0 + bn) * 128.0 / 110.0;
-      double t_max = t_mma > t_l2 ? t_mma : t_l2;
-      if (t_sm > t_max) t_max = t_sm;
+      const double t_sm = waves * nkl * (128.0 + bn) * 128.0 / 72.0;
+      const double t_max = t_mma > t_sm ? t_mma : t_sm;
       const double t = t_max + 2000.0 + waves * (600.0 + 6.0 * bn / sp) +
                        (sp > 1 ? 800.0 + 150.0 * sp : 0.0);
       if (t < best_t - 1e-9) {

@@ -1223,10 +1223,6 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   wtake(reinterpret_cast<void**>(&m->k), rows * d * 2);
   wtake(reinterpret_cast<void**>(&m->vt), static_cast<size_t>(d) * ((rows + 7) & ~static_cast<size_t>(7)) * 2 + 4096);
   wtake(reinterpret_cast<void**>(&m->cpk), rows * kC * 2);
-  wtake(reinterpret_cast<void**>(&m->ao), rows * d * 2);
-  wtake(reinterpret_cast<void**>(&m->f), rows * F * 2);
-  wtake(reinterpret_cast<void**>(&m->r), rows * d * 4);
-  wtake(reinterpret_cast<void**>(&m->ra), rows * d * 2);
   // partial row sums of the folded LayerNorms: up to 2 per 32 columns
   const size_t ln_parts_max = 2 * static_cast<size_t>((d + 31) / 32);
   wtake(reinterpret_cast<void**>(&m->stats_a), ln_parts_max * rows * 8);

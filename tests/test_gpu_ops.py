@@ -136,12 +136,14 @@ def _attn_ref(q, k, v, H):
 
 @pytest.mark.parametrize("batch,T,H,growth", [(1, 1, 1, 0), (1, 7, 2, 0), (1, 128, 1, 0), (2, 129, 2, 0),
                                               (1, 799, 12, 0), (2, 499, 3, 0), (1, 1000, 2, 0), (1, 256, 16, 0),
-                                              (1, 799, 2, 1), (2, 640, 2, 2)])
+                                              (1, 799, 2, 1), (2, 640, 2, 2), (1, 799, 12, 1), (1, 799, 12, 2),
+                                              (1, 799, 16, 0), (3, 300, 4, 2)])
 def test_attention_matches_oracle(batch, T, H, growth):
     """growth > 0 makes later key tiles score much higher than the first ones
     (growth 1: key t scaled by 1 + 4 t / T and the queries by 2; growth 2: every
     128-key block scaled by twice the previous one), so a row's running maximum
-    rises by more than 2^8 across tiles and the accumulator rescale runs."""
+    rises by more than 2^8 across tiles and the accumulator rescale runs
+    (also with the 16 s window's 12 heads, and with several clips)."""
     g = torch.Generator().manual_seed(T * 31 + H + 7 * growth)
     d = 64 * H
     q = torch.randn(batch, T, d, generator=g)
