@@ -26,10 +26,13 @@ extern "C" {
  * tile width and split-K factor; otherwise bn (32/64/128/192/256) and splits
  * are forced: splits 1..8 (<= K/64) divides the K blocks among a cluster of
  * `splits` CTAs whose partial sums are reduced in distributed shared memory;
- * splits -2 or -4 (bn >= 64) reduces 2 or 4 splits through an fp32 scratch in
- * L2 (TMA stores and loads; the call allocates and frees it on the stream),
- * summed in split order; splits 0 (bn >= 64) runs CTA pairs: clusters of two
- * CTAs on 256-row tiles with the 2-CTA tensor-core instructions, each CTA
+ * splits -2, -3 or -4 (bn >= 64, as far as the last arrival's staging fits:
+ * bn 64 up to 4 splits, 128 up to 3, 192 up to 2) reduces the splits through
+ * an fp32 scratch in L2 without a cluster: each split TMA-stores its partial,
+ * takes a ticket, and the last to arrive loads the others and finishes the
+ * tile, adding the partials in split order (the call allocates and frees
+ * the scratch on the stream); splits 0 (bn >= 64) runs CTA pairs: clusters of
+ * two CTAs on 256-row tiles with the 2-CTA tensor-core instructions, each CTA
  * loading its 128 rows of A and half of the tile's B columns (needs a
  * 16-byte-aligned output row pitch: the direct TMA-store epilogue).  Invalid
  * combinations return W2V_EINVAL. */

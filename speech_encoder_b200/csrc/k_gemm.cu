@@ -522,27 +522,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     __syncthreads();
   } else if (mode == 1 || (SPLIT && mode == 3)) {
     // ------------------------------------------------------------- direct
-    // mode 3 = split-K through L2: the S = 2 or 4 CTAs of a tile (a cluster
-    // along z) split K; split k owns the 32-row quarters q with q S / 4 = k.
-    // Warps whose quarter another split owns TMA-store their fp32 partial
-    // boxes to that split's plane of the scratch (map in tmV's slot); after a
-    // cluster barrier the owning warps TMA-load the other splits' boxes of
-    // their rows (into the drained staging of the non-owning warps), add them
-    // in split order (deterministic) and finish as in the direct form.
+    // mode 3 = split-K through L2, finished by the last arrival: the S CTAs
+    // of a tile (grid z, no cluster) each TMA-store their fp32 partial boxes
+    // to their plane of the scratch (map in tmV's slot), then take a ticket
+    // (one counter per tile, at e.out_k); the CTA that arrives last TMA-loads
+    // the other planes' boxes of its rows (into the drained operand ring), adds
+    // the partials in split order 0..S-1 (deterministic: its own from TMEM in
+    // its place) and finishes as in the direct form; it resets the counter.
+    // No CTA waits for another: the others are done once their partial and
+    // ticket are out.
     constexpr int kChunks = BN / 2 / 32;  // 32-column boxes per warp
     const bool m3 = SPLIT && mode == 3;
-    const bool owner = !m3 || (q * S) / 4 == split;
-    // Staging region of the non-owner warp that holds peer pi's boxes for the
-    // owner warp (q, half): the same half, quarter q ^ 2 (S = 2) or the pi-th
-    // quarter other than q (S = 4); epilogue warp w has quarter (w + 2) & 3
-    // and half w >> 2.
+    bool owner = true;
+    // Staging of the boxes of the other splits for warp w (0..7), split slot
+    // pi (0..S-2): after the eight warps' own output staging.
     auto peer_region = [&](int pi) -> uint8_t* {
-      const int q2 = S == 2 ? (q ^ 2) : (pi < q ? pi : pi + 1);
-      const int w = half * 4 + ((q2 - 2) & 3);
-      return smem + w * kChunks * 4096;
+      return smem + (8 * kChunks + ((warp - 2) * (S - 1) + pi) * kChunks) * 4096;
     };
     if (m3) {
-      if (epi && !owner && ok) {
+      int* tickets = static_cast<int*>(e.out_k);
+      const int tile = static_cast<int>(blockIdx.y) * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
+      int* last_s = reinterpret_cast<int*>(tmem_slot + 1);
+      if (epi && ok) {
         uint8_t* stg = smem + (warp - 2) * kChunks * 4096;
 #pragma unroll 1
         for (int cb = 0; cb < kChunks; ++cb) {
@@ -560,17 +561,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         if (lane == 0) {
           bulk_commit_group();
-          bulk_wait_all();
+          bulk_wait_all();  // the partial is in global memory
+          asm volatile("fence.proxy.async.global;" ::: "memory");
         }
       }
-      __threadfence();
-      tc_fence_before();
-      __syncwarp();
-      cluster_sync();  // every partial box of the cluster is in the scratch
-      tc_fence_after();
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      if (epi && owner && ok) {
-        if (lane == 0) {
+      if (epi) {
+        __threadfence();
+        named_barrier_sync(2, kEpiThreads);  // every box of this CTA is out
+        if (et == 0) *last_s = atomicAdd(&tickets[tile], 1) == S - 1 ? 1 : 0;
+        named_barrier_sync(2, kEpiThreads);
+        owner = *last_s != 0;
+      }
+      if (epi && owner) {
+        // the other splits' partials are complete: load this warp's boxes of them
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        if (ok && lane == 0) {
           mbar_arrive_expect_tx(&peer_bar[warp - 2], static_cast<uint32_t>((S - 1) * kChunks * 4096));
           int pi = 0;
           for (int k = 0; k < S; ++k) {
@@ -581,12 +587,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             ++pi;
           }
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(&peer_bar[warp - 2], 0));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&peer_bar[warp - 2], 0));
         if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+        if (et == 0) tickets[tile] = 0;  // ready for the next launch
       }
     }
     if (epi && owner) {
-      if (mode == 1) named_barrier_sync(1, kEpiThreads);  // bias staged (mode 3: the cluster barrier)
+      if (mode == 1) named_barrier_sync(1, kEpiThreads);  // bias staged (mode 3: the ticket barriers)
       const int grow = m0 + r;
       void* outp = region == 1 ? e.out_k : e.out;
       const int ocol0 = region > 0 ? region * e.qkv_d : 0;
@@ -933,6 +940,21 @@ int gemm_pick(GemmShape* s, int bn_divides) {
   return best_bn;
 }
 
+// The L2 split form's last arrival keeps its own output staging plus the
+// other S-1 splits' boxes of its rows in the drained operand ring.
+bool gemm_l2_split_fits(int bn, int splits) {
+  const int chunks = bn / 2 / 32;
+  int ring = 0;
+  switch (bn) {
+    case 64: ring = GemmCfg<64>::RING; break;
+    case 128: ring = GemmCfg<128>::RING; break;
+    case 192: ring = GemmCfg<192>::RING; break;
+    case 256: ring = GemmCfg<256>::RING; break;
+    default: return false;
+  }
+  return chunks >= 1 && splits >= 2 && 8 * splits * chunks * 4096 <= ring;
+}
+
 template <int BN>
 static cudaError_t prepare_bn() {
   cudaError_t r = cudaFuncSetAttribute(gemm_tc_kernel<BN, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -977,11 +999,13 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = pair ? 2 : 1;
   attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = S > 1 ? S : 1;  // modes 2 and 3
+  const bool cluster_split = S > 1 && mode == 2;  // the L2 form (mode 3) needs no cluster
+  attr[1].val.clusterDim.z = cluster_split ? S : 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (S > 1 || pair) ? 2 : 1;
+  cfg.numAttrs = (cluster_split || pair) ? 2 : 1;
   const GemmDims sd = s;      // the kernel's parameter block holds only
-  const GemmEpiArgs ea = e;   // what it reads
+  GemmEpiArgs ea = e;         // what it reads
+  if (mode == 3) ea.out_k = e.split_tickets;  // the L2 form's tickets (out_k is a QKV-only field)
   if (pair) {
     if (BN < 64 || S > 1 || mode != 1) return cudaErrorInvalidValue;
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, (BN >= 64)>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
@@ -1025,8 +1049,11 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   std::memset(&tmO2, 0, sizeof tmO2);
   std::memset(&tmV, 0, sizeof tmV);
   int mode = s.splits > 1 ? 2 : 0;
-  // split-K through L2 (mode 3): S = 2 or 4, the scratch, and a TMA-storable output
-  const bool l2split = s.split_l2 && (s.splits == 2 || s.splits == 4) && e.part_ws && e.qkv_d == 0 &&
+  // split-K through L2 (mode 3): S = 2..4, the scratch, a ticket per tile, the
+  // last arrival's staging in shared memory, and a TMA-storable output
+  const int64_t n_tiles = static_cast<int64_t>((s.M + 127) / 128) * ((s.N + bn - 1) / bn);
+  const bool l2split = s.split_l2 && s.splits >= 2 && s.splits <= 4 && gemm_l2_split_fits(bn, s.splits) &&
+                       e.part_ws && e.split_tickets && n_tiles <= e.ticket_cap && e.qkv_d == 0 &&
                        s.N <= e.ws_ld && e.ws_ld % 4 == 0 && e.ws_rows >= 128L * ((s.M + 127) / 128) &&
                        (reinterpret_cast<uintptr_t>(e.part_ws) % 16) == 0;
   if (s.split_l2 && !l2split) return cudaErrorInvalidValue;

@@ -220,6 +220,8 @@ struct w2v_model {
   size_t forced_i = 0;
   float* part_ws = nullptr;      // split-K through L2: fp32 [4][ws_rows][ws_ld]
   int64_t ws_rows = 0, ws_ld = 0;
+  int* split_tickets = nullptr;  // and its arrival counters, one per output tile
+  static constexpr int64_t kTicketCap = 4096;
   int max_rows = 0;
   // Launch plans per (n_samples, batch) and instantiated graphs per
   // (n_samples, batch, pcm, logits), both least-recently-used caches of a
@@ -295,6 +297,8 @@ GemmEpilogue epi_base(const w2v_model* m) {
   e.part_ws = m->part_ws;
   e.ws_rows = m->ws_rows;
   e.ws_ld = m->ws_ld;
+  e.split_tickets = m->split_tickets;
+  e.ticket_cap = w2v_model::kTicketCap;
   return e;
 }
 
@@ -414,7 +418,8 @@ GemmEpilogue epi_lm(const w2v_model* m, const Plan& p, float* logits) {
 // Whether a GEMM may split K by `sp` (2 or 4) through the L2 scratch.
 bool l2_split_ok(const w2v_model* m, const GemmShape& s, int N, int bn, int sp) {
   return s.batch == 1 && bn >= 64 && N <= m->ws_ld && 128L * ((s.M + 127) / 128) <= m->ws_rows &&
-         s.K / 64 >= 2 * sp;
+         s.K / 64 >= 2 * sp && gemm_l2_split_fits(bn, sp) &&
+         static_cast<int64_t>((s.M + 127) / 128) * ((N + bn - 1) / bn) <= w2v_model::kTicketCap;
 }
 
 // A GEMM role's launch form as one integer (plan files, refinement): 0 = CTA
@@ -444,7 +449,7 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     const bool bn_ok = (bn == 32 || bn == 64 || bn == 128 || bn == 192 || bn == 256) &&
                        (bn_divides <= 0 || bn_divides % bn == 0);
     const bool sp_ok = sp == 1 || (sp > 1 && sp <= 8 && s->batch == 1 && sp <= nk) ||
-                       ((sp == -2 || sp == -4) && l2_split_ok(m, *s, N, bn, -sp)) || (sp == 0 && bn >= 64);
+                       ((sp >= -4 && sp <= -2) && l2_split_ok(m, *s, N, bn, -sp)) || (sp == 0 && bn >= 64);
     if (!bn_ok || !sp_ok) return fail(m, W2V_EINVAL, "plan file: bn=%d splits=%d invalid for N=%d K=%d", bn, sp, N, K);
     (void)splits;
     set_form(s, sp);
@@ -470,7 +475,7 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     if (bn >= 64) CUDA_OR(m, map_b(&tmBp, W, N, K, bn, 0));
     // sp > 1: K splits reduced through distributed shared memory; sp < 0:
     // -sp splits reduced through the L2 scratch; sp 0: CTA pairs
-    for (int sp : {1, 2, 3, 4, 6, -2, -4, 0}) {
+    for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0}) {
       if (sp > 1 && (s->batch != 1 || nk < 16 || sp > nk)) continue;
       if (sp < 0 && !l2_split_ok(m, *s, N, bn, -sp)) continue;
       if (sp == 0 && bn < 64) continue;
@@ -1223,6 +1228,10 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   wtake(reinterpret_cast<void**>(&m->k), rows * d * 2);
   wtake(reinterpret_cast<void**>(&m->vt), static_cast<size_t>(d) * ((rows + 7) & ~static_cast<size_t>(7)) * 2 + 4096);
   wtake(reinterpret_cast<void**>(&m->cpk), rows * kC * 2);
+  wtake(reinterpret_cast<void**>(&m->ao), rows * d * 2);
+  wtake(reinterpret_cast<void**>(&m->f), rows * F * 2);
+  wtake(reinterpret_cast<void**>(&m->r), rows * d * 4);
+  wtake(reinterpret_cast<void**>(&m->ra), rows * d * 2);
   // partial row sums of the folded LayerNorms: up to 2 per 32 columns
   const size_t ln_parts_max = 2 * static_cast<size_t>((d + 31) / 32);
   wtake(reinterpret_cast<void**>(&m->stats_a), ln_parts_max * rows * 8);
@@ -1238,6 +1247,7 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   m->ws_rows = std::min<int64_t>((static_cast<int64_t>(B) * tf + 127) / 128 * 128, 2048);
   m->ws_ld = std::max(d, kC);
   wtake(reinterpret_cast<void**>(&m->part_ws), static_cast<size_t>(4) * m->ws_rows * m->ws_ld * 4);
+  wtake(reinterpret_cast<void**>(&m->split_tickets), static_cast<size_t>(w2v_model::kTicketCap) * 4);
   const size_t wsbytes = round_up(cursor, 1 << 20);
   if (cudaMalloc(&m->ws, wsbytes) != cudaSuccess) {
     cudaFree(m->wmem);
@@ -1337,7 +1347,7 @@ int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
     for (int bn : {32, 64, 128, 192, 256}) {
       if (bn == 32 ? N > 32 : N <= bn / 2) continue;
       if (role == 0 && d % bn != 0) continue;
-      for (int sp : {1, 2, 3, 4, 6, -2, -4, 0}) {
+      for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0}) {
         if (sp > 1 && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
         if (sp < 0 && !l2_split_ok(m, *sh, N, bn, -sp)) continue;
         if (sp == 0 && bn < 64) continue;
@@ -1827,7 +1837,7 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   }
   if (bn != 32 && bn != 64 && bn != 128 && bn != 192 && bn != 256) return W2V_EINVAL;
   if (s.splits < 1 || s.splits > 8 || s.splits > K / 64) return W2V_EINVAL;
-  if (s.split_l2 && ((s.splits != 2 && s.splits != 4) || bn < 64)) return W2V_EINVAL;
+  if (s.split_l2 && (s.splits < 2 || s.splits > 4 || bn < 64 || !gemm_l2_split_fits(bn, s.splits))) return W2V_EINVAL;
   if (s.pair && bn < 64) return W2V_EINVAL;
   CUtensorMap ta, tb;
   if (map_a(&ta, A, K, M, K, 1, 0) != cudaSuccess) return W2V_ECUDA;
@@ -1845,9 +1855,15 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   if (s.split_l2) {
     e.ws_rows = 128L * ((M + 127) / 128);
     e.ws_ld = (N + 3) / 4 * 4;
-    if (cudaMallocAsync(&ws, static_cast<size_t>(s.splits) * e.ws_rows * e.ws_ld * 4, st) != cudaSuccess)
-      return W2V_ENOMEM;
+    const size_t part = static_cast<size_t>(s.splits) * e.ws_rows * e.ws_ld * 4;
+    e.ticket_cap = static_cast<int64_t>((M + 127) / 128) * ((N + bn - 1) / bn);
+    if (cudaMallocAsync(&ws, part + static_cast<size_t>(e.ticket_cap) * 4, st) != cudaSuccess) return W2V_ENOMEM;
     e.part_ws = static_cast<float*>(ws);
+    e.split_tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + part);
+    if (cudaMemsetAsync(e.split_tickets, 0, static_cast<size_t>(e.ticket_cap) * 4, st) != cudaSuccess) {
+      cudaFreeAsync(ws, st);
+      return W2V_ECUDA;
+    }
   }
   const cudaError_t r = launch_gemm(ta, tb, s, bn, e, err_dev, st);
   if (ws) cudaFreeAsync(ws, st);

@@ -96,6 +96,10 @@ struct GemmEpilogue : GemmEpiArgs {
   float* part_ws = nullptr;
   int64_t ws_rows = 0;
   int64_t ws_ld = 0;
+  // one arrival counter per output tile for the same form, zero before the
+  // first launch (each launch leaves them zero); ticket_cap counters
+  int* split_tickets = nullptr;
+  int64_t ticket_cap = 0;
 };
 
 // Streaming multiprocessors of a B200: the grid of the persistent kernels.
@@ -114,8 +118,9 @@ struct GemmDims {
 };
 
 struct GemmShape : GemmDims {
-  bool split_l2 = false;  // or, with splits 2 or 4, through the L2 scratch of
-                          // GemmEpilogue (TMA stores and loads of fp32 boxes)
+  bool split_l2 = false;  // or, with splits 2..4, through the L2 scratch of
+                          // GemmEpilogue (TMA stores and loads of fp32 boxes,
+                          // the last split to arrive finishing the tile)
   bool pair = false;      // CTA pairs on 256-row tiles (2-CTA tensor-core
                           // instructions); then tmB's box is {64, bn/2}, no split
 };
@@ -125,6 +130,8 @@ struct GemmShape : GemmDims {
 // QKV projection needs tiles that do not straddle Q/K/V).
 // tmA: {cols, rows, batch}, box {64,128,1}; tmB: {K, N}, box {64, bn}.
 int gemm_pick(GemmShape* s, int bn_divides);
+// Whether the split-K-through-L2 form fits tile width bn with `splits` splits.
+bool gemm_l2_split_fits(int bn, int splits);
 // Raise the dynamic shared-memory limits of the tcgen05 kernels (idempotent;
 // called before any launch or stream capture).
 cudaError_t gemm_prepare();

@@ -41,13 +41,15 @@ GEMM_CASES = [
     (130, 96, 512, (64, 8), 2, None, 0),
     (1, 2341, 1024, (256, 5), 0, None, 1),
     (799, 512, 1024, (192, 3), 1, "f16", 0),
-    # split-K through the L2 scratch (splits -2 / -4)
-    (799, 768, 3072, (128, -4), 0, "f16", 1),
-    (799, 768, 3072, (256, -2), 0, "f32", 1),
+    # split-K through the L2 scratch, finished by the last split to arrive
+    # (splits -2..-4; the tile widths whose staging fits)
+    (799, 768, 3072, (128, -3), 0, "f16", 1),
+    (799, 768, 3072, (192, -2), 0, "f32", 1),
     (799, 768, 768, (64, -2), 0, "f16", 1),
     (130, 96, 512, (64, -4), 2, None, 0),
-    (257, 512, 1536, (192, -4), 1, "f16", 0),
-    (1, 640, 1024, (256, -2), 0, None, 1),
+    (257, 512, 1536, (192, -2), 1, "f16", 0),
+    (1, 640, 1024, (64, -3), 0, None, 1),
+    (799, 768, 3072, (128, -2), 0, "f16", 0),
     # CTA pairs on 256-row tiles (splits 0): odd M (the last pair half or
     # wholly past M), N tails, every tile width, residuals, both outputs
     (799, 2304, 768, (128, 0), 0, None, 0),
@@ -95,8 +97,8 @@ def test_gemm_every_tile_width_same_result():
     A = torch.randn(M, K, generator=g).half().cuda()
     W = (torch.randn(N, K, generator=g) * 0.05).half().cuda()
     outs = []
-    for bn, sp in ((32, 1), (64, 1), (128, 1), (192, 1), (256, 1), (256, 2), (128, 8), (64, 3), (256, -2),
-                   (128, -4), (192, -4), (64, 0), (128, 0), (192, 0), (256, 0)):
+    for bn, sp in ((32, 1), (64, 1), (128, 1), (192, 1), (256, 1), (256, 2), (128, 8), (64, 3), (64, -3),
+                   (128, -3), (192, -2), (64, 0), (128, 0), (192, 0), (256, 0)):
         out = torch.empty(M, N, dtype=torch.float32, device="cuda")
         assert B.w2v_op_gemm(A, W, M, N, K, None, None, 0, out, 1, 0, _err(), bn=bn, splits=sp) == 0
         outs.append(out)
