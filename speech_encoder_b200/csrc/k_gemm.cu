@@ -58,12 +58,19 @@ struct GemmCfg {
   static constexpr int ROWLN_OFF = VEC_OFF + 2 * BN * 4;  // per-row LN factors, 128 float2
   static constexpr int BAR_OFF = ROWLN_OFF + 128 * 8;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  // An fp16 residual tile (128 rows x BN) staged by TMA during the mainloop
+  // takes the ring's last RES_STAGES stages.
+  static constexpr int RES_BYTES = BM * BN * 2;
+  static constexpr int RES_STAGES = (RES_BYTES + STAGE - 1) / STAGE;
   static_assert(BM * BN * 4 <= RING, "parked tile must fit in the operand ring");
   static_assert(ROW_CHUNKS >= 8, "row swizzle needs >= 8 chunks");
 };
 
 constexpr int kGemmThreads = 320;
 constexpr int kEpiThreads = 256;
+// Flag in the kernel's mode word: the fp16 residual tile is staged in shared
+// memory by TMA (its map in tmO2's slot, which only the QKV split uses).
+constexpr int kModeResTma = 16;
 static_assert(sizeof(GemmEpiArgs) <= 128, "the GEMM kernel's parameter block must stay within 808 bytes");
 
 // fp32 tile rows of `row_chunks` 16-byte chunks; chunk j of row r lives at
@@ -77,26 +84,95 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Epilogue chunk helpers.  Each tests its uniform condition once, outside the
+// unrolled loop over the chunk, so that the code a launch executes is one
+// compact straight run (it runs once per CTA, from a cold instruction cache).
+// v += bias (tile columns lcol..lcol+N-1, 16-byte aligned in shared memory)
+template <int N>
+__device__ __forceinline__ void add_cols(float (&v)[N], const float* col_s) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 b = *reinterpret_cast<const float4*>(col_s + i);
+    v[i] += b.x;
+    v[i + 1] += b.y;
+    v[i + 2] += b.z;
+    v[i + 3] += b.w;
+  }
+}
+
+// Folded LayerNorm of the A rows (ln_mode 1): v = rstd * v - mean * rstd * colsum
+template <int N>
+__device__ __forceinline__ void ln1_cols(float (&v)[N], const float* cs_s, float2 lnr) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 cs = *reinterpret_cast<const float4*>(cs_s + i);
+    v[i] = fmaf(lnr.x, v[i], lnr.y * cs.x);
+    v[i + 1] = fmaf(lnr.x, v[i + 1], lnr.y * cs.y);
+    v[i + 2] = fmaf(lnr.x, v[i + 2], lnr.y * cs.z);
+    v[i + 3] = fmaf(lnr.x, v[i + 3], lnr.y * cs.w);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void act_inplace(float (&v)[N], int act) {
+  if (act == 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = gelu_erf(v[i]);
+  } else if (act == 2) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = gelu_tanh(v[i]);
+  }
+}
+
+// v += residual f, normalised first when ln_mode == 2:
+// (f * rstd - mean * rstd) * gamma + beta (gamma at g_s, beta at g_s + bn)
+template <int N>
+__device__ __forceinline__ void add_residual(float (&v)[N], const float (&f)[N], int ln_mode, const float* g_s,
+                                             int bn, float2 lnr) {
+  if (ln_mode == 2) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const float4 g = *reinterpret_cast<const float4*>(g_s + i);
+      const float4 b = *reinterpret_cast<const float4*>(g_s + bn + i);
+      v[i] += fmaf(fmaf(f[i], lnr.x, lnr.y), g.x, b.x);
+      v[i + 1] += fmaf(fmaf(f[i + 1], lnr.x, lnr.y), g.y, b.y);
+      v[i + 2] += fmaf(fmaf(f[i + 2], lnr.x, lnr.y), g.z, b.z);
+      v[i + 3] += fmaf(fmaf(f[i + 3], lnr.x, lnr.y), g.w, b.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] += f[i];
+  }
+}
+
 // Final epilogue for 4 consecutive columns [col, col+4) of row grow: bias
 // (from shared memory), GELU, residual, store.  `vec` selects 16-/8-byte
 // accesses (row starts and pointers 16-byte aligned, full 4-vector in range).
 // lnr: the row's LayerNorm factors (rstd, -mean * rstd) when e.ln_mode != 0;
 // vec_s: the LN column vectors of this tile (ln_mode 1: column sums; 2: gamma,
 // then beta at vec_s + BN).
+// res_s: the staged fp16 residual tile (boxes of 32 columns x 128 rows,
+// 64-byte rows, 64-byte swizzle; zeros outside the matrix) or null to read
+// the residual from global memory; lrow: the tile row.
 __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, const float* vec_s, int bn, float2 lnr,
                                         int lcol, int grow, int col, int nv, int bzb, const GemmEpiArgs& e,
-                                        void* outp, int ocol0, bool vec) {
+                                        void* outp, int ocol0, bool vec, const uint8_t* res_s = nullptr,
+                                        int lrow = 0) {
   const int ln_mode = e.ln_cfg & 255;
-  if (ln_mode == 1) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = fmaf(lnr.x, x[i], lnr.y * vec_s[lcol + i]);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) x[i] = apply_act(x[i] + bias_s[lcol + i], e.act);
+  if (ln_mode == 1) ln1_cols<4>(x, vec_s + lcol, lnr);
+  add_cols<4>(x, bias_s + lcol);
+  act_inplace<4>(x, e.act);
   if (e.residual) {
     const int64_t roff = static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
     float rv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (e.res_f32) {
+    if (res_s) {
+      const int cc = lcol & 31;
+      const uint2 u = *reinterpret_cast<const uint2*>(res_s + (lcol >> 5) * 8192 + lrow * 64 +
+                                                      (((cc >> 3) ^ ((lrow >> 1) & 3)) << 4) + (cc & 7) * 2);
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+      rv[0] = a.x; rv[1] = a.y; rv[2] = b.x; rv[3] = b.y;
+    } else if (e.res_f32) {
       const float* rp = static_cast<const float*>(e.residual) + roff;
       if (vec && nv == 4) {
         const float4 t = *reinterpret_cast<const float4*>(rp);
@@ -115,12 +191,7 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, cons
         for (int i = 0; i < nv; ++i) rv[i] = __half2float(rp[i]);
       }
     }
-    if (ln_mode == 2) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) rv[i] = fmaf(fmaf(rv[i], lnr.x, lnr.y), vec_s[lcol + i], vec_s[bn + lcol + i]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] += rv[i];
+    add_residual<4>(x, rv, ln_mode, vec_s + lcol, bn, lnr);
   }
   const int64_t ooff = static_cast<int64_t>(bzb) * e.out_batch_stride + static_cast<int64_t>(grow) * e.ldo + (col - ocol0);
   if (e.out_f32) {
@@ -139,8 +210,10 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, cons
 }
 
 // mode: 0 generic, 1 direct (TMA store), 2 split-K through distributed shared
-// memory, 3 split-K through an L2 scratch (with the direct stores)
-// SPLIT: the instantiation for split-K launches (modes 2 and 3); the other one
+// memory (each cluster CTA finishing a band of rows), 3 split-K through an L2
+// scratch, 4 split-K through distributed shared memory (each cluster CTA
+// finishing a group of columns); 3 and 4 with the direct stores.
+// SPLIT: the instantiation for split-K launches (modes 2-4); the other one
 // runs modes 0 and 1 only.
 // PAIR: CTA pairs (clusters of 2 along M) on 256-row tiles with the 2-CTA
 // tensor-core instructions, mode 1 only.  The pair halves the B operand bytes
@@ -151,9 +224,14 @@ template <int BN, bool SPLIT, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
-               const __grid_constant__ CUtensorMap tmV, GemmDims s, GemmEpiArgs e, int vec_ok, int mode, int* err) {
+               const __grid_constant__ CUtensorMap tmV, GemmDims s, GemmEpiArgs e, int vec_ok, int mode_word,
+               int* err) {
   static_assert(!(SPLIT && PAIR), "pairs do not split K");
   using C = GemmCfg<BN, PAIR>;
+  const int mode = mode_word & 15;
+  const bool res_tma = (mode_word & kModeResTma) != 0;
+  // ring stages in use (the staged residual takes the last ones)
+  const int nst = res_tma ? C::STAGES - C::RES_STAGES : C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + C::BIAS_OFF);
@@ -163,7 +241,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
   uint64_t* peer_bar = accf + 1;  // [8] mode 3: one per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_bar + 8);
+  uint64_t* res_bar = peer_bar + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_bar + 1);
+  const uint8_t* res_s = smem + nst * C::STAGE;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -175,7 +255,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int bzb = S > 1 ? 0 : static_cast<int>(blockIdx.z);  // batch index
   const int kb0 = split * nk / S;
   const int nkl = (split + 1) * nk / S - kb0;  // K blocks of this CTA (>= 1)
-  const int pre = nkl < C::STAGES ? nkl : C::STAGES;
+  const int pre = nkl < nst ? nkl : nst;
   // pair rank (0: the CTA that issues the MMAs), cluster rank of that CTA,
   // the first B row this CTA loads, and the pair's CTA mask
   const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
@@ -191,6 +271,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     mbar_init(accf, 1);
     for (int i = 0; i < 8; ++i) mbar_init(&peer_bar[i], 1);
+    mbar_init(res_bar, 1);
     fence_mbar_init();
     pdl_launch_dependents();
     tma_prefetch_desc(&tmA);
@@ -220,6 +301,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The fp16 residual tile of this CTA's 128 rows, as BN/32 boxes of 32
+  // columns, into the ring's tail on this CTA's own barrier (pairs too); the
+  // epilogue waits for it.
+  auto stage_residual = [&]() {
+    mbar_arrive_expect_tx(res_bar, C::RES_BYTES);
+    for (int cb = 0; cb < BN / 32; ++cb)
+      tma_load_3d(smem + nst * C::STAGE + cb * 8192, &tmO2, res_bar, n0 + cb * 32, m0, bzb);
+  };
 
   if (PAIR && warp == 0) {
     if (lane == 0) {
@@ -235,10 +324,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int k = (kb0 + i) * C::BK;
         tma_load_3d_pair(smem + i * C::STAGE, &tmA, fbar(i), k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
       }
+      if (res_tma) stage_residual();
       bool ok = true;
       for (int i = pre; i < nkl; ++i) {
-        const int st = i % C::STAGES;
-        if (!mbar_wait(&empty[st], ((i / C::STAGES) & 1) ^ 1)) {
+        const int st = i % nst;
+        if (!mbar_wait(&empty[st], ((i / nst) & 1) ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
           break;
@@ -253,8 +343,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // CTA has landed and every release the MMA issuer sent here has
       // arrived, before this CTA may leave.
       if (ok) {
-        for (int i = (nkl > C::STAGES ? nkl - C::STAGES : 0); i < nkl; ++i)
-          if (!mbar_wait(&empty[i % C::STAGES], (i / C::STAGES) & 1)) {
+        for (int i = (nkl > nst ? nkl - nst : 0); i < nkl; ++i)
+          if (!mbar_wait(&empty[i % nst], (i / nst) & 1)) {
             atomicOr(err, kErrWaitProducer);
             break;
           }
@@ -280,7 +370,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kk = 0; kk < 4; ++kk)
           umma_f16_pair(tmem, dA0 + off + 2 * kk, dB0 + off + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
         umma_commit_pair(&empty[st], pmask);
-        if (++st == C::STAGES) {
+        if (++st == nst) {
           st = 0;
           ph ^= 1u;
         }
@@ -294,11 +384,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int k = (kb0 + i) * C::BK;
         tma_load_3d(smem + i * C::STAGE, &tmA, &full[i], k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
       }
+      if (res_tma) stage_residual();
       int issued = pre;
       bool ok = true;
       for (int i = pre; i < nkl; ++i) {
-        const int st = i % C::STAGES;
-        const uint32_t ph = (i / C::STAGES) & 1;
+        const int st = i % nst;
+        const uint32_t ph = (i / nst) & 1;
         if (!mbar_wait(&empty[st], ph ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
@@ -313,8 +404,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA exits.
-        for (int i = (issued > C::STAGES ? issued - C::STAGES : 0); i < issued; ++i)
-          mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1);
+        for (int i = (issued > nst ? issued - nst : 0); i < issued; ++i)
+          mbar_wait(&full[i % nst], (i / nst) & 1);
       }
     }
   } else if (warp == 1) {
@@ -341,7 +432,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kk = 0; kk < 4; ++kk)
           umma_f16(tmem, dA0 + off + 2 * kk, dB0 + off + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
         umma_commit(&empty[st]);
-        if (++st == C::STAGES) {
+        if (++st == nst) {
           st = 0;
           ph ^= 1u;
         }
@@ -405,18 +496,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
     if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+    if (res_tma) {  // waited for even after a failure: no copy may land after the CTA leaves
+      const bool rok = __all_sync(0xffffffffu, mbar_wait(res_bar, 0));
+      if (!rok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+      ok = ok && rok;
+    }
     tc_fence_after();
   }
   // The LayerNorm factors (rstd, -mean * rstd) of tile row lrow.
   auto row_lnr = [&](int lrow) -> float2 { return ln_mode != 0 ? rowln_s[lrow] : make_float2(1.f, 0.f); };
   // Modes 0 and 2 with partial row sums to store: each epilogue warp takes
   // whole rows (lr0 + lr, lr < nrows, tile rows r0 + lr) and its lanes the
-  // rows' 16-byte chunks, so that a row's two half-tile sums reduce inside the
-  // warp in a fixed order.  fetch4(lr, j) gives chunk j of the row's fp32 sums.
+  // rows' 16-byte chunks, so that the sums of each 32-column group (8 chunks,
+  // 8 neighbouring lanes) reduce inside the warp in a fixed order; they go to
+  // partial (n0 + col) / 32, as in every form.  fetch4(lr, j) gives chunk j of
+  // the row's fp32 sums.
   auto finish_rows_stats = [&](int r0, int nrows, void* outp, int ocol0, auto&& fetch4) {
     constexpr int RC = C::ROW_CHUNKS;
     constexpr int RPW = RC >= 32 ? 1 : 32 / RC;  // rows per warp pass
     constexpr int JSTEP = RC >= 32 ? 32 : RC;
+    constexpr int NJ = RC >= 32 ? RC / 32 : 1;   // chunks per lane and row
     const int ew = et >> 5;
     const int sub = RC >= 32 ? 0 : lane / RC;
     const int j0 = RC >= 32 ? lane : lane % RC;
@@ -425,40 +524,41 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int lr = lb + sub;
       const int grow = m0 + r0 + lr;
       const bool live = lr < nrows && grow < s.M;
-      float a1 = 0.f, a2 = 0.f, b1 = 0.f, b2 = 0.f;
+      float p1[NJ], p2[NJ];
+#pragma unroll
+      for (int t = 0; t < NJ; ++t) p1[t] = p2[t] = 0.f;
       if (live) {
         const float2 lnr = row_lnr(r0 + lr);
-        for (int j = j0; j < RC; j += JSTEP) {
+#pragma unroll
+        for (int t = 0; t < NJ; ++t) {
+          const int j = j0 + t * JSTEP;
           const int col = n0 + 4 * j;
           if (col >= s.N) continue;
           const int nv = min(4, s.N - col);
           const float4 v = fetch4(lr, j);
           float x[4] = {v.x, v.y, v.z, v.w};
-          finish4(x, bias_s, vec_s, BN, lnr, 4 * j, grow, col, nv, bzb, e, outp, ocol0, vec);
-          float p1 = 0.f, p2 = 0.f;
+          finish4(x, bias_s, vec_s, BN, lnr, 4 * j, grow, col, nv, bzb, e, outp, ocol0, vec,
+                  res_tma ? res_s : nullptr, r0 + lr);
           for (int i = 0; i < nv; ++i) {
-            p1 += x[i];
-            p2 = fmaf(x[i], x[i], p2);
-          }
-          if (4 * j < BN / 2) {
-            a1 += p1;
-            a2 += p2;
-          } else {
-            b1 += p1;
-            b2 += p2;
+            p1[t] += x[i];
+            p2[t] = fmaf(x[i], x[i], p2[t]);
           }
         }
       }
 #pragma unroll
-      for (int o = (RC >= 32 ? 16 : RC / 2); o > 0; o >>= 1) {
-        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-        b1 += __shfl_xor_sync(0xffffffffu, b1, o);
-        b2 += __shfl_xor_sync(0xffffffffu, b2, o);
+      for (int t = 0; t < NJ; ++t) {
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+          p1[t] += __shfl_xor_sync(0xffffffffu, p1[t], o);
+          p2[t] += __shfl_xor_sync(0xffffffffu, p2[t], o);
+        }
       }
-      if (live && j0 == 0) {
-        e.ln_out[static_cast<int64_t>(2 * blockIdx.y) * s.M + grow] = make_float2(a1, a2);
-        e.ln_out[static_cast<int64_t>(2 * blockIdx.y + 1) * s.M + grow] = make_float2(b1, b2);
+      if (live && (j0 & 7) == 0) {
+#pragma unroll
+        for (int t = 0; t < NJ; ++t) {
+          const int col = n0 + 4 * (j0 + t * JSTEP);
+          if (col < s.N) e.ln_out[static_cast<int64_t>(col >> 5) * s.M + grow] = make_float2(p1[t], p2[t]);
+        }
       }
     }
   };
@@ -487,12 +587,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
         float v[32];
         if (ok) tmem_ld32(trow + c, v);
-        if (ln_mode == 1) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = fmaf(lnr.x, v[i], lnr.y * vec_s[c + i]);
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i] + bias_s[c + i], e.act);
+        if (ln_mode == 1) ln1_cols<32>(v, vec_s + c, lnr);
+        add_cols<32>(v, bias_s + c);
+        act_inplace<32>(v, e.act);
         const int cc = n0 + c - 2 * e.qkv_d;  // column within V: head * 64 + dim
         if (boxed) {
           uint8_t* box = stage + nbox * 4096;
@@ -520,7 +617,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     tc_fence_before();
     __syncthreads();
-  } else if (mode == 1 || (SPLIT && mode == 3)) {
+  } else if (mode == 1 || (SPLIT && (mode == 3 || mode == 4))) {
     // ------------------------------------------------------------- direct
     // mode 3 = split-K through L2, finished by the last arrival: the S CTAs
     // of a tile (grid z, no cluster) each TMA-store their fp32 partial boxes
@@ -531,14 +628,56 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // its place) and finishes as in the direct form; it resets the counter.
     // No CTA waits for another: the others are done once their partial and
     // ticket are out.
+    //
+    // mode 4 = split-K through the cluster (grid z, cluster of S along z),
+    // each CTA finishing a group of columns: the tile's columns form S groups
+    // of W = BN / S (a multiple of 64); cluster CTA k, which also computed K
+    // split k, finishes group k.  After a cluster barrier (every ring is
+    // drained) each warp writes its rows of the other groups' columns, fp32,
+    // into the owners' shared memory (slot of this sender, 4 KB boxes of 32
+    // rows x 32 columns); after a second barrier each owner adds the S partials
+    // in split order 0..S-1 (its own from TMEM in its place) and finishes its
+    // columns as in the direct form, every epilogue warp on W / 2 of them.
     constexpr int kChunks = BN / 2 / 32;  // 32-column boxes per warp
     const bool m3 = SPLIT && mode == 3;
+    const bool m4 = SPLIT && mode == 4;
     bool owner = true;
+    const int gw = m4 ? BN / S : BN;  // width of the column group this CTA finishes
+    const int kc4 = gw / 64;          // boxes per warp in mode 4
+    // this warp's columns of the tile in the finishing loop
+    const int cbeg = (m4 ? split * gw : 0) + half * (gw / 2);
+    const int cend = cbeg + gw / 2;
     // Staging of the boxes of the other splits for warp w (0..7), split slot
-    // pi (0..S-2): after the eight warps' own output staging.
+    // pi (0..S-2): mode 3 after the eight warps' own output staging; mode 4 at
+    // the start of the ring, the output staging after it.
     auto peer_region = [&](int pi) -> uint8_t* {
+      if (m4) return smem + ((pi * 8 + (warp - 2)) * kc4) * 4096;
       return smem + (8 * kChunks + ((warp - 2) * (S - 1) + pi) * kChunks) * 4096;
     };
+    if (m4) {
+      cluster_sync();  // every accumulator of the cluster is final: all rings are free
+      if (epi && ok) {
+#pragma unroll 1
+        for (int g = 0; g < S; ++g) {
+          if (g == split) continue;
+          const int si = split < g ? split : split - 1;  // this CTA's slot at owner g
+#pragma unroll 1
+          for (int cb = 0; cb < kc4; ++cb) {
+            float v[32];
+            tmem_ld32(trow + g * gw + half * (gw / 2) + cb * 32, v);
+            const uint32_t dst =
+                mapa_shared(smem_u32(smem) + static_cast<uint32_t>(((si * 8 + (warp - 2)) * kc4 + cb) * 4096 + lane * 128),
+                            static_cast<uint32_t>(g));
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              st_dsmem_f4(dst + ((k ^ (lane & 7)) << 4), make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      cluster_sync();  // every partial has landed in its owner's shared memory
+      tc_fence_after();
+    }
     if (m3) {
       int* tickets = static_cast<int*>(e.out_k);
       const int tile = static_cast<int>(blockIdx.y) * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
@@ -599,17 +738,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int ocol0 = region > 0 ? region * e.qkv_d : 0;
       const CUtensorMap* om = region == 1 ? &tmO2 : &tmO;
       // Staging: this warp's boxes of 32 rows x 32 columns, 4 KB apart.
-      uint8_t* stage = smem + (warp - 2) * (BN / 2 / 32) * 4096;
+      uint8_t* stage = smem + ((m4 ? (S - 1) * 8 * kc4 : 0) + (warp - 2) * ((cend - cbeg) / 32)) * 4096;
       int nbox = 0;
       const float2 lnr = row_lnr(r);
-      float st1 = 0.f, st2 = 0.f;
 #pragma unroll 1
-      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+      for (int c = cbeg; c < cend; c += 32) {
         float v[32];
         if (ok) tmem_ld32(trow + c, v);
-        if (m3 && ok) {
+        if ((m3 || m4) && ok) {
           // partials in split order 0..S-1, this CTA's own (TMEM) in its place
-          const int cb = (c - half * (BN / 2)) / 32;
+          const int cb = (c - cbeg) / 32;
           float acc[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) acc[i] = 0.f;
@@ -631,71 +769,71 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = acc[i];
         }
-        if (ln_mode == 1) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = fmaf(lnr.x, v[i], lnr.y * vec_s[c + i]);
-        }
+        if (ln_mode == 1) ln1_cols<32>(v, vec_s + c, lnr);
+        add_cols<32>(v, bias_s + c);
+        act_inplace<32>(v, e.act);
         const int col = n0 + c;
+        const int nv = min(32, s.N - col);
         if (e.residual && grow < s.M) {
           const int64_t roff =
               static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
-          const int nv = min(32, s.N - col);
+          float f[32];
           if (e.res_f32) {
             const float* rp = static_cast<const float*>(e.residual) + roff;
             if (nv == 32) {
 #pragma unroll
               for (int i = 0; i < 32; i += 4) {
                 const float4 rv = *reinterpret_cast<const float4*>(rp + i);
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + rv.x;
-                v[i + 1] = apply_act(v[i + 1] + bias_s[c + i + 1], e.act) + rv.y;
-                v[i + 2] = apply_act(v[i + 2] + bias_s[c + i + 2], e.act) + rv.z;
-                v[i + 3] = apply_act(v[i + 3] + bias_s[c + i + 3], e.act) + rv.w;
+                f[i] = rv.x;
+                f[i + 1] = rv.y;
+                f[i + 2] = rv.z;
+                f[i + 3] = rv.w;
               }
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + (i < nv ? rp[i] : 0.f);
+              for (int i = 0; i < 32; ++i) f[i] = i < nv ? rp[i] : 0.f;
             }
           } else {
             const __half* rp = static_cast<const __half*>(e.residual) + roff;
-            if (nv == 32) {
+            // staged: this row's 64 bytes of the column box c / 32 (zeros past N)
+            const uint8_t* rb = res_s + (c >> 5) * 8192 + r * 64;
+            if (res_tma || nv == 32) {
 #pragma unroll
               for (int i = 0; i < 32; i += 8) {
-                const uint4 u = *reinterpret_cast<const uint4*>(rp + i);
+                const uint4 u = res_tma ? *reinterpret_cast<const uint4*>(rb + (((i >> 3) ^ ((r >> 1) & 3)) << 4))
+                                        : *reinterpret_cast<const uint4*>(rp + i);
                 const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                  float2 f = __half22float2(h[k]);
-                  if (ln_mode == 2) {
-                    const int cc = c + i + 2 * k;
-                    f.x = fmaf(fmaf(f.x, lnr.x, lnr.y), vec_s[cc], vec_s[BN + cc]);
-                    f.y = fmaf(fmaf(f.y, lnr.x, lnr.y), vec_s[cc + 1], vec_s[BN + cc + 1]);
-                  }
-                  v[i + 2 * k] = apply_act(v[i + 2 * k] + bias_s[c + i + 2 * k], e.act) + f.x;
-                  v[i + 2 * k + 1] = apply_act(v[i + 2 * k + 1] + bias_s[c + i + 2 * k + 1], e.act) + f.y;
+                  const float2 t = __half22float2(h[k]);
+                  f[i + 2 * k] = t.x;
+                  f[i + 2 * k + 1] = t.y;
                 }
               }
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float f = i < nv ? __half2float(rp[i]) : 0.f;
-                if (ln_mode == 2) f = fmaf(fmaf(f, lnr.x, lnr.y), vec_s[c + i], vec_s[BN + c + i]);
-                v[i] = apply_act(v[i] + bias_s[c + i], e.act) + f;
-              }
+              for (int i = 0; i < 32; ++i) f[i] = i < nv ? __half2float(rp[i]) : 0.f;
             }
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = apply_act(v[i] + bias_s[c + i], e.act);
+          add_residual<32>(v, f, ln_mode, vec_s + c, BN, lnr);
         }
-        if (e.ln_out) {  // this row's partial sums over this warp's half of the tile
-          const int nvs = min(32, s.N - col);
+        if (e.ln_out) {  // this row's partial sums over these 32 columns
+          float st1 = 0.f, st2 = 0.f;
+          if (nv == 32) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nvs) {
+            for (int i = 0; i < 32; ++i) {
               st1 += v[i];
               st2 = fmaf(v[i], v[i], st2);
             }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nv) {
+                st1 += v[i];
+                st2 = fmaf(v[i], v[i], st2);
+              }
+          }
+          if (ok && grow < s.M && nv > 0) e.ln_out[static_cast<int64_t>(col >> 5) * s.M + grow] = make_float2(st1, st2);
         }
         uint8_t* box = stage + nbox * 4096;
         if (e.out_f32) {
@@ -717,8 +855,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (lane == 0 && ok && col < s.N) tma_store_3d(om, box, col - ocol0, m0 + q * 32, bzb);
         ++nbox;
       }
-      if (e.ln_out && ok && grow < s.M)
-        e.ln_out[static_cast<int64_t>(2 * blockIdx.y + half) * s.M + grow] = make_float2(st1, st2);
       if (lane == 0) {  // as above: wait until the boxes have been read
         bulk_commit_group();
         bulk_wait_read_all();
@@ -777,15 +913,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const int col = n0 + 4 * j;
           if (grow >= s.M || col >= s.N) continue;
           const float4 v = fetch(lr, j);
-          const float x[4] = {v.x, v.y, v.z, v.w};
+          float x[4] = {v.x, v.y, v.z, v.w};
+          if (ln_mode == 1) ln1_cols<4>(x, vec_s + 4 * j, row_lnr(r0 + lr));
+          add_cols<4>(x, bias_s + 4 * j);
+          act_inplace<4>(x, e.act);
           const int cc = col - 2 * e.qkv_d;
           const int clip = grow / e.t_len;
           const int t = grow - clip * e.t_len;
           __half* dst = static_cast<__half*>(e.vt) +
                         (static_cast<int64_t>(clip * e.n_heads + (cc >> 6)) * 64 + (cc & 63)) * e.t_pad + t;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(apply_act(x[i] + bias_s[4 * j + i], e.act));
+          for (int i = 0; i < 4; ++i) dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(x[i]);
         }
       } else {
         void* outp = region == 1 ? e.out_k : e.out;
@@ -802,7 +940,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const float4 v = fetch(lr, j);
           float x[4] = {v.x, v.y, v.z, v.w};
           finish4(x, bias_s, vec_s, BN, row_lnr(r0 + lr), 4 * j, grow, col, min(4, s.N - col), bzb, e, outp,
-                  ocol0, vec);
+                  ocol0, vec, res_tma ? res_s : nullptr, r0 + lr);
         }
       }
     }
@@ -843,19 +981,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (grow >= s.M || col >= s.N) continue;
           const float4 v = *reinterpret_cast<const float4*>(park + swz_off(C::ROW_CHUNKS, rr, j));
           float x[4] = {v.x, v.y, v.z, v.w};
-          if (ln_mode == 1) {
-            const float2 lnr = rowln_s[rr];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) x[i] = fmaf(lnr.x, x[i], lnr.y * vec_s[4 * j + i]);
-          }
+          if (ln_mode == 1) ln1_cols<4>(x, vec_s + 4 * j, rowln_s[rr]);
+          add_cols<4>(x, bias_s + 4 * j);
+          act_inplace<4>(x, e.act);
           const int cc = col - 2 * e.qkv_d;
           const int clip = grow / e.t_len;
           const int t = grow - clip * e.t_len;
           __half* dst = static_cast<__half*>(e.vt) +
                         (static_cast<int64_t>(clip * e.n_heads + (cc >> 6)) * 64 + (cc & 63)) * e.t_pad + t;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(apply_act(x[i] + bias_s[4 * j + i], e.act));
+          for (int i = 0; i < 4; ++i) dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(x[i]);
         }
       } else {
         void* outp = region == 1 ? e.out_k : e.out;
@@ -940,6 +1075,35 @@ int gemm_pick(GemmShape* s, int bn_divides) {
   return best_bn;
 }
 
+// Whether a staged residual tile leaves at least two ring stages and room in
+// front of it for the epilogue's staging of this form: the output boxes
+// (mode 1, 8 warps x BN/64 boxes of 4 KB), the cluster partials (mode 2,
+// S slots of ceil(128/S) fp32 rows; mode 4, S - 1 slots of 128 rows x BN/S
+// columns and the output boxes) or the L2 form's boxes (mode 3).
+template <int BN, bool PAIR>
+static bool res_stage_fits_cfg(int mode, int splits) {
+  using C = GemmCfg<BN, PAIR>;
+  if (BN < 64 || BN > 192) return false;
+  const int nst = C::STAGES - C::RES_STAGES;
+  if (nst < 2) return false;
+  const int room = nst * C::STAGE;
+  const int chunks = BN / 64;
+  if (mode == 1) return 8 * chunks * 4096 <= room;
+  if (mode == 2) return splits * ((C::BM + splits - 1) / splits) * (BN / 4) * 16 <= room;
+  if (mode == 3) return 8 * splits * chunks * 4096 <= room;
+  if (mode == 4) return 8 * BN / 64 * 4096 <= room;  // the S - 1 senders' slots and the output staging
+  return false;
+}
+
+bool gemm_res_stage_fits(int bn, bool pair, int mode, int splits) {
+  switch (bn) {
+    case 64: return pair ? res_stage_fits_cfg<64, true>(mode, splits) : res_stage_fits_cfg<64, false>(mode, splits);
+    case 128: return pair ? res_stage_fits_cfg<128, true>(mode, splits) : res_stage_fits_cfg<128, false>(mode, splits);
+    case 192: return pair ? res_stage_fits_cfg<192, true>(mode, splits) : res_stage_fits_cfg<192, false>(mode, splits);
+    default: return false;
+  }
+}
+
 // The L2 split form's last arrival keeps its own output staging plus the
 // other S-1 splits' boxes of its rows in the drained operand ring.
 bool gemm_l2_split_fits(int bn, int splits) {
@@ -999,15 +1163,16 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = pair ? 2 : 1;
   attr[1].val.clusterDim.y = 1;
-  const bool cluster_split = S > 1 && mode == 2;  // the L2 form (mode 3) needs no cluster
+  // the cluster forms (modes 2 and 4); the L2 form (mode 3) needs no cluster
+  const bool cluster_split = S > 1 && ((mode & 15) == 2 || (mode & 15) == 4);
   attr[1].val.clusterDim.z = cluster_split ? S : 1;
   cfg.attrs = attr;
   cfg.numAttrs = (cluster_split || pair) ? 2 : 1;
   const GemmDims sd = s;      // the kernel's parameter block holds only
   GemmEpiArgs ea = e;         // what it reads
-  if (mode == 3) ea.out_k = e.split_tickets;  // the L2 form's tickets (out_k is a QKV-only field)
+  if ((mode & 15) == 3) ea.out_k = e.split_tickets;  // the L2 form's tickets (out_k is a QKV-only field)
   if (pair) {
-    if (BN < 64 || S > 1 || mode != 1) return cudaErrorInvalidValue;
+    if (BN < 64 || S > 1 || (mode & 15) != 1) return cudaErrorInvalidValue;
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, (BN >= 64)>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
                               mode, err);
   }
@@ -1057,7 +1222,11 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
                        s.N <= e.ws_ld && e.ws_ld % 4 == 0 && e.ws_rows >= 128L * ((s.M + 127) / 128) &&
                        (reinterpret_cast<uintptr_t>(e.part_ws) % 16) == 0;
   if (s.split_l2 && !l2split) return cudaErrorInvalidValue;
-  const bool tma_ok = (s.splits == 1 || l2split) && bn >= 64 && vec && (e.ldo * esz_out) % 16 == 0 &&
+  // split-K through the cluster with column groups (mode 4): groups of a
+  // multiple of 64 columns, the direct epilogue's stores
+  const bool colsplit = s.splits > 1 && !s.split_l2 && e.qkv_d == 0 && bn % s.splits == 0 &&
+                        (bn / s.splits) % 64 == 0;
+  const bool tma_ok = (s.splits == 1 || l2split || colsplit) && bn >= 64 && vec && (e.ldo * esz_out) % 16 == 0 &&
                       (e.residual == nullptr || (e.ldr * esz_res) % 16 == 0);
   if (tma_ok) {
     const uint64_t cols = e.qkv_d > 0 ? static_cast<uint64_t>(e.qkv_d) : static_cast<uint64_t>(s.N);
@@ -1085,10 +1254,23 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
       const uint64_t ws[2] = {static_cast<uint64_t>(e.ws_ld) * 4, static_cast<uint64_t>(e.ws_rows * e.ws_ld) * 4};
       built = make_tmap(&tmV, e.part_ws, 3, wd, ws, box, 4, 128) == cudaSuccess;
     }
-    if (built) mode = l2split ? 3 : 1;
+    if (built) mode = l2split ? 3 : (colsplit ? 4 : 1);
   }
   if (l2split && mode != 3) return cudaErrorInvalidValue;
   if (s.pair && mode != 1) return cudaErrorInvalidValue;
+  // An fp16 residual is staged in shared memory by TMA while the mainloop
+  // runs (boxes of 32 columns x 128 rows, 64-byte swizzle), when the ring's
+  // remaining stages still hold the epilogue's own staging.
+  if (mode >= 1 && e.residual && !e.res_f32 && e.qkv_d == 0 && (e.ldr * 2) % 16 == 0 &&
+      reinterpret_cast<uintptr_t>(e.residual) % 16 == 0 && (s.batch == 1 || (e.res_batch_stride * 2) % 16 == 0) &&
+      gemm_res_stage_fits(bn, s.pair, mode, s.splits)) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.N), static_cast<uint64_t>(s.M), static_cast<uint64_t>(s.batch)};
+    const uint64_t bstride = s.batch > 1 ? static_cast<uint64_t>(e.res_batch_stride) * 2
+                                         : static_cast<uint64_t>(s.M) * e.ldr * 2;
+    const uint64_t str[2] = {static_cast<uint64_t>(e.ldr) * 2, bstride};
+    const uint32_t box[3] = {32, 128, 1};
+    if (make_tmap(&tmO2, e.residual, 3, dims, str, box, 2, 64) == cudaSuccess) mode |= kModeResTma;
+  }
   switch (bn) {
     case 32: return launch_bn<32>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);
     case 64: return launch_bn<64>(tmA, tmB, tmO, tmO2, tmV, s, e, vec, mode, err, st);

@@ -320,9 +320,13 @@ GemmEpilogue epi_proj(const w2v_model* m) {
   return e;
 }
 
-// Partial row sums stored by a GEMM of N columns in tiles of bn (two per
-// column tile), and the ln_cfg word of a GEMM that reads them.
-int ln_parts(int N, int bn) { return 2 * ((N + bn - 1) / bn); }
+// Partial row sums stored by a GEMM of N columns (one per 32-column group,
+// whatever its tile width and form), and the ln_cfg word of a GEMM that
+// reads them.
+int ln_parts(int N, int bn) {
+  (void)bn;
+  return (N + 31) / 32;
+}
 int ln_cfg(int mode, int parts) { return mode | (parts << 8); }
 
 GemmEpilogue epi_qkv(const w2v_model* m, const Plan& p, int l) {
@@ -1233,7 +1237,7 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
   wtake(reinterpret_cast<void**>(&m->r), rows * d * 4);
   wtake(reinterpret_cast<void**>(&m->ra), rows * d * 2);
   // partial row sums of the folded LayerNorms: up to 2 per 32 columns
-  const size_t ln_parts_max = 2 * static_cast<size_t>((d + 31) / 32);
+  const size_t ln_parts_max = static_cast<size_t>((d + 31) / 32);
   wtake(reinterpret_cast<void**>(&m->stats_a), ln_parts_max * rows * 8);
   wtake(reinterpret_cast<void**>(&m->stats_f), ln_parts_max * rows * 8);
   wtake(reinterpret_cast<void**>(&m->gn_partial), static_cast<size_t>(B) * 296 * 65 * 8);

@@ -72,8 +72,9 @@ struct GemmEpiArgs {
   int t_len = 0;                   // frames per clip (rows are clip-major)
   // LayerNorm folded into the GEMMs (post-norm encoder blocks).  Row
   // statistics travel as partial sums: a GEMM with ln_out set stores, for each
-  // output row and each half of each column tile (2 N / BN partials), the sum
-  // and the sum of squares of its final values at ln_out[p * M + row].  A GEMM
+  // output row and each 32-column group p (ceil(N / 32) partials, whatever the
+  // tile width or split form), the sum and the sum of squares of its final
+  // values at ln_out[p * M + row].  A GEMM
   // reading such rows gets (ln_cfg >> 8) partials per row at ln_in and
   //  ln_mode 1 (ln_cfg & 255): A holds the un-normalised rows x and B holds
   //    W diag(gamma); the epilogue turns the accumulator into LN(x) W^T + bias
@@ -132,6 +133,8 @@ struct GemmShape : GemmDims {
 int gemm_pick(GemmShape* s, int bn_divides);
 // Whether the split-K-through-L2 form fits tile width bn with `splits` splits.
 bool gemm_l2_split_fits(int bn, int splits);
+// Whether a GEMM of this form can stage its fp16 residual tile in shared memory.
+bool gemm_res_stage_fits(int bn, bool pair, int mode, int splits);
 // Raise the dynamic shared-memory limits of the tcgen05 kernels (idempotent;
 // called before any launch or stream capture).
 cudaError_t gemm_prepare();

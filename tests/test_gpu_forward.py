@@ -328,6 +328,31 @@ def test_plan_file_pins_the_gemm_choices_across_models(tmp_path, monkeypatch):
     m3.close()
 
 
+@pytest.mark.parametrize("forms", [("128:2", "64:-2", "128:0", "64:4"), ("128:1", "128:2", "256:2", "128:2")])
+def test_every_split_form_in_the_encoder_matches_oracle(tmp_path, monkeypatch, forms):
+    # A pinned plan puts each encoder GEMM of the post-norm model (folded
+    # LayerNorms, partial row sums) on another form.  First: QKV split 2 ways
+    # through the cluster by row bands (its V^T columns normalised too), the
+    # out-projection split 2 ways through the L2 scratch with its fp16 residual
+    # staged, FFN1 on CTA pairs, FFN2 split 4 ways by row bands.  Second: the
+    # out-projection, FFN1 and FFN2 split through the cluster by column
+    # groups.  The logits still match the oracle.
+    shape = S.small_shape()
+    pcm = S.synth_pcm(30000, 9)
+    path = tmp_path / "plans.txt"
+    monkeypatch.setenv("W2V_PLAN_FILE", str(path))
+    m1 = U.make_model(shape, 48000, 1, seed=3, affine_noise=True)
+    _run(m1, pcm[None])
+    m1.close()
+    key, *choices = path.read_text().split()
+    choices[7:11] = list(forms)
+    path.write_text(" ".join([key] + choices) + "\n")
+    m2 = U.make_model(shape, 48000, 1, seed=3, affine_noise=True)
+    got = _run(m2, pcm[None])
+    m2.close()
+    print(U.compare_logits(got[0], U.oracle_logits(shape, pcm, seed=3, affine_noise=True), "split forms"))
+
+
 def test_model_from_safetensors_equals_model_from_blob(tmp_path, monkeypatch):
     # The loader's blob (checkpoint names, fp16 tensors, weight-normalised
     # positional conv) gives the same logits as the same blob handed to

@@ -61,6 +61,21 @@ GEMM_CASES = [
     (12799, 512, 1536, (256, 0), 1, None, 0),
     (300, 2304, 1024, (256, 0), 0, None, 1),
     (257, 200, 192, (128, 0), 1, "f32", 0),
+    # fp16 residual tiles staged in shared memory by TMA: ragged N (zero fill
+    # past N) and M in every form that stages them; rows of 100 halves are not
+    # 16-byte multiples and take the global-load path
+    (130, 200, 192, 64, 0, "f16", 0),
+    (257, 200, 256, (128, 2), 0, "f16", 1),
+    (799, 200, 768, (128, 0), 0, "f16", 0),
+    (300, 456, 1024, (192, 0), 1, "f16", 1),
+    (799, 328, 3072, (64, -4), 0, "f16", 0),
+    (130, 100, 128, 64, 0, "f16", 0),
+    # split-K through the cluster with each CTA finishing a group of columns
+    # (splits dividing the tile into groups of 64 or 128 columns)
+    (799, 768, 3072, (128, 2), 0, "f16", 0),
+    (799, 768, 3072, (256, 4), 0, "f16", 1),
+    (300, 456, 1024, (192, 3), 2, "f32", 1),
+    (1, 256, 512, (128, 2), 0, None, 0),
 ]
 
 
