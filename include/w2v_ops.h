@@ -34,8 +34,13 @@ extern "C" {
  * the scratch on the stream); splits 0 (bn >= 64) runs CTA pairs: clusters of
  * two CTAs on 256-row tiles with the 2-CTA tensor-core instructions, each CTA
  * loading its 128 rows of A and half of the tile's B columns (needs a
- * 16-byte-aligned output row pitch: the direct TMA-store epilogue).  Invalid
- * combinations return W2V_EINVAL. */
+ * 16-byte-aligned output row pitch: the direct TMA-store epilogue); splits 9
+ * (bn >= 64) runs the persistent form: one CTA per SM walking the output
+ * tiles, two TMEM accumulators so that each tile's epilogue overlaps the next
+ * tile's mainloop (needs 16-byte-aligned output and residual row pitches).
+ * With splits 2..8 and bn / splits a multiple of 64 each cluster CTA
+ * finishes a group of the tile's columns, otherwise a band of its rows.
+ * Invalid combinations return W2V_EINVAL. */
 int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, const float* bias, const void* residual,
                 int res_f32, void* out, int out_f32, int act, int bn, int splits, int* err_dev, void* stream);
 

@@ -1031,6 +1031,317 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
+// ---------------------------------------------------------------- persistent
+// Persistent form for GEMMs with more output tiles than SMs: one CTA per SM
+// walks the tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... (row tile
+// fastest, then column tile, then batch item).  Operand stages flow through
+// one ring across tiles, and the accumulator is double-buffered in TMEM: the
+// MMA thread fills one buffer while the epilogue warps drain the other, so a
+// tile's epilogue runs under the next tile's mainloop.  The epilogue is the
+// direct form's arithmetic (folded LayerNorm, bias, activation, residual,
+// partial row sums) with plain vector stores from registers (no staging);
+// the bias, LN vectors and row factors are reloaded for each tile.
+template <int BN>
+struct GemmPCfg {
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int RING_MAX = 200 * 1024;
+  static constexpr int STAGES = (RING_MAX / STAGE) > 8 ? 8 : (RING_MAX / STAGE);
+  static constexpr int RING = STAGES * STAGE;
+  static constexpr int ACC_COLS = BN <= 64 ? 64 : (BN <= 128 ? 128 : 256);  // one accumulator
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int BIAS_OFF = RING;
+  static constexpr int VEC_OFF = BIAS_OFF + BN * 4;
+  static constexpr int ROWLN_OFF = VEC_OFF + 2 * BN * 4;
+  static constexpr int BAR_OFF = ROWLN_OFF + 128 * 8;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static_assert(BN >= 64 && BN % 32 == 0, "persistent tiles are 64..256 wide");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmDims s,
+                    GemmEpiArgs e, int n_mt, int n_nt, int vec_ok, int* err) {
+  using C = GemmPCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* bias_s = reinterpret_cast<float*>(smem + C::BIAS_OFF);
+  float* vec_s = reinterpret_cast<float*>(smem + C::VEC_OFF);
+  float2* rowln_s = reinterpret_cast<float2*>(smem + C::ROWLN_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;  // [2] accumulator b complete
+  uint64_t* tempty = tfull + 2;         // [2] accumulator b drained (one arrival per epilogue warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nk = s.K / C::BK;
+  const int n_tiles = n_mt * n_nt * s.batch;
+  auto tile_of = [&](int t, int& m0, int& n0, int& bz) {
+    const int mt = t % n_mt;
+    const int rest = t / n_mt;
+    m0 = mt * C::BM;
+    n0 = (rest % n_nt) * BN;
+    bz = rest / n_nt;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(&tfull[0], 1);
+    mbar_init(&tfull[1], 1);
+    mbar_init(&tempty[0], kEpiThreads / 32);
+    mbar_init(&tempty[1], kEpiThreads / 32);
+    fence_mbar_init();
+    pdl_launch_dependents();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();
+      int st = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        int m0, n0, bz;
+        tile_of(t, m0, n0, bz);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[st], ph ^ 1)) {
+            atomicOr(err, kErrWaitProducer);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + st * C::STAGE;
+          mbar_arrive_expect_tx(&full[st], C::STAGE);
+          const int k = kb * C::BK;
+          tma_load_3d(sa, &tmA, &full[st], k % s.a_kwrap, m0 + k / s.a_kwrap, bz);
+          tma_load_2d(sa + C::A_BYTES, &tmB, &full[st], k, n0);
+          ++issued;
+          if (++st == C::STAGES) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already in flight land before the CTA exits.
+        for (int i = (issued > C::STAGES ? issued - C::STAGES : 0); i < issued; ++i)
+          mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(128, BN);
+      const uint64_t dA0 = desc_sw128(smem_u32(smem));
+      const uint64_t dB0 = desc_sw128(smem_u32(smem) + C::A_BYTES);
+      int st = 0;
+      uint32_t ph = 0;
+      int i = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+        const int b = i & 1;
+        if (!mbar_wait(&tempty[b], ((i >> 1) & 1) ^ 1)) {
+          atomicOr(err, kErrWaitMma);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(b * C::ACC_COLS);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[st], ph)) {
+            atomicOr(err, kErrWaitMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t off = static_cast<uint64_t>(st * (C::STAGE >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16(d, dA0 + off + 2 * kk, dB0 + off + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(&empty[st]);
+          if (++st == C::STAGES) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[b]);
+      }
+    }
+  } else {
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = q * 32 + lane;
+    const int ln_mode = e.ln_cfg & 255;
+    const bool vec = vec_ok != 0;
+    bool ok = true;
+    pdl_wait();  // row partial sums and residuals come from earlier kernels
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      int m0, n0, bz;
+      tile_of(t, m0, n0, bz);
+      // this tile's column vectors and row factors (the previous tile's
+      // readers are past the barrier)
+      named_barrier_sync(1, kEpiThreads);
+      for (int c = et; c < BN; c += kEpiThreads) {
+        const bool in = n0 + c < s.N;
+        bias_s[c] = (e.bias && in) ? e.bias[n0 + c] : 0.f;
+        if (ln_mode != 0) vec_s[c] = in ? e.ln_vec[n0 + c] : 0.f;
+        if (ln_mode == 2) vec_s[BN + c] = in ? e.ln_vec[s.N + n0 + c] : 0.f;
+      }
+      if (ln_mode != 0 && et < C::BM) {
+        const int grow = m0 + et;
+        float2 f = make_float2(1.f, 0.f);
+        if (grow < s.M) {
+          const int parts = e.ln_cfg >> 8;
+          float s1 = 0.f, s2 = 0.f;
+          for (int p0 = 0; p0 < parts; p0 += 8) {
+            float2 tv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              tv[k] = p0 + k < parts ? e.ln_in[static_cast<int64_t>(p0 + k) * s.M + grow] : make_float2(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              s1 += tv[k].x;
+              s2 += tv[k].y;
+            }
+          }
+          const float inv = 1.f / static_cast<float>(ln_mode == 1 ? s.K : s.N);
+          const float mean = s1 * inv;
+          const float rstd = rsqrtf(fmaxf(fmaf(s2, inv, -mean * mean), 0.f) + e.ln_eps);
+          f = make_float2(rstd, -mean * rstd);
+        }
+        rowln_s[et] = f;
+      }
+      named_barrier_sync(1, kEpiThreads);
+      const int b = i & 1;
+      if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[b], (i >> 1) & 1));
+        if (!ok && lane == 0) atomicOr(err, kErrWaitEpilogue);
+      }
+      tc_fence_after();
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * C::ACC_COLS);
+      const int grow = m0 + r;
+      const float2 lnr = ln_mode != 0 ? rowln_s[r] : make_float2(1.f, 0.f);
+#pragma unroll 1
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2) && ok; c += 32) {
+        float v[32];
+        tmem_ld32(tacc + c, v);
+        if (c + 32 >= (half + 1) * (BN / 2)) {
+          // the last read of this accumulator: hand it back to the MMA thread
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[b]);
+        }
+        if (ln_mode == 1) ln1_cols<32>(v, vec_s + c, lnr);
+        add_cols<32>(v, bias_s + c);
+        act_inplace<32>(v, e.act);
+        const int col = n0 + c;
+        const int nv = min(32, s.N - col);
+        if (grow >= s.M || nv <= 0) continue;
+        if (e.residual) {
+          const int64_t roff =
+              static_cast<int64_t>(bz) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+          float f[32];
+          if (e.res_f32) {
+            const float* rp = static_cast<const float*>(e.residual) + roff;
+            if (vec && nv == 32) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 4) {
+                const float4 rv = *reinterpret_cast<const float4*>(rp + k);
+                f[k] = rv.x;
+                f[k + 1] = rv.y;
+                f[k + 2] = rv.z;
+                f[k + 3] = rv.w;
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) f[k] = k < nv ? rp[k] : 0.f;
+            }
+          } else {
+            const __half* rp = static_cast<const __half*>(e.residual) + roff;
+            if (vec && nv == 32) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 8) {
+                const uint4 u = *reinterpret_cast<const uint4*>(rp + k);
+                const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float2 tf = __half22float2(h[j]);
+                  f[k + 2 * j] = tf.x;
+                  f[k + 2 * j + 1] = tf.y;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) f[k] = k < nv ? __half2float(rp[k]) : 0.f;
+            }
+          }
+          add_residual<32>(v, f, ln_mode, vec_s + c, BN, lnr);
+        }
+        if (e.ln_out) {
+          float st1 = 0.f, st2 = 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k < nv) {
+              st1 += v[k];
+              st2 = fmaf(v[k], v[k], st2);
+            }
+          e.ln_out[static_cast<int64_t>(col >> 5) * s.M + grow] = make_float2(st1, st2);
+        }
+        const int64_t ooff = static_cast<int64_t>(bz) * e.out_batch_stride + static_cast<int64_t>(grow) * e.ldo + col;
+        if (e.out_f32) {
+          float* op = static_cast<float*>(e.out) + ooff;
+          if (vec && nv == 32) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+              *reinterpret_cast<float4*>(op + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k < nv) op[k] = v[k];
+          }
+        } else {
+          __half* op = static_cast<__half*>(e.out) + ooff;
+          if (vec && nv == 32) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 8)
+              *reinterpret_cast<uint4*>(op + k) = make_uint4(pack_h2(v[k], v[k + 1]), pack_h2(v[k + 2], v[k + 3]),
+                                                             pack_h2(v[k + 4], v[k + 5]), pack_h2(v[k + 6], v[k + 7]));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k < nv) op[k] = __float2half_rn(v[k]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 // Tile width and split-K factor: the candidate whose launch should finish
 // first under a simple model of this kernel on B200 (148 SMs):
 //  * MMA time per CTA: per 64-deep K block the larger of the MMA time
@@ -1129,6 +1440,11 @@ static cudaError_t prepare_bn() {
   if (r == cudaSuccess && BN >= 64)
     r = cudaFuncSetAttribute(gemm_tc_kernel<BN, false, (BN >= 64)>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<BN, (BN >= 64)>::SMEM);
+  if constexpr (BN >= 64) {
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(gemm_persist_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               GemmPCfg<BN>::SMEM);
+  }
   return r;
 }
 
@@ -1182,6 +1498,56 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
                                     mode, err);
 }
 
+// The persistent form: no split, pair or QKV split; 16-byte vector stores of
+// the output rows and loads of the residual rows.
+template <int BN>
+static cudaError_t launch_persist_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s,
+                                     const GemmEpilogue& e, int* err, cudaStream_t st) {
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
+      return cudaErrorInvalidValue;
+  }
+  const int n_mt = (s.M + 127) / 128, n_nt = (s.N + BN - 1) / BN;
+  const long tiles = static_cast<long>(n_mt) * n_nt * s.batch;
+  if (tiles <= 0 || tiles > (1L << 30)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < n_sm ? tiles : n_sm));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = GemmPCfg<BN>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const GemmDims sd = s;
+  const GemmEpiArgs ea = e;
+  return cudaLaunchKernelEx(&cfg, gemm_persist_kernel<BN>, tmA, tmB, sd, ea, n_mt, n_nt, 1, err);
+}
+
+static cudaError_t launch_persist(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
+                                  const GemmEpilogue& e, int* err, cudaStream_t st) {
+  if (s.splits != 1 || s.split_l2 || s.pair || e.qkv_d > 0 || !e.out) return cudaErrorInvalidValue;
+  const int esz_out = e.out_f32 ? 4 : 2;
+  const int esz_res = e.res_f32 ? 4 : 2;
+  const bool out_ok = reinterpret_cast<uintptr_t>(e.out) % 16 == 0 && (e.ldo * esz_out) % 16 == 0 &&
+                      (s.batch == 1 || (e.out_batch_stride * esz_out) % 16 == 0);
+  const bool res_ok = e.residual == nullptr ||
+                      (reinterpret_cast<uintptr_t>(e.residual) % 16 == 0 && (e.ldr * esz_res) % 16 == 0 &&
+                       (s.batch == 1 || (e.res_batch_stride * esz_res) % 16 == 0));
+  if (!out_ok || !res_ok) return cudaErrorInvalidValue;
+  switch (bn) {
+    case 64: return launch_persist_bn<64>(tmA, tmB, s, e, err, st);
+    case 128: return launch_persist_bn<128>(tmA, tmB, s, e, err, st);
+    case 192: return launch_persist_bn<192>(tmA, tmB, s, e, err, st);
+    case 256: return launch_persist_bn<256>(tmA, tmB, s, e, err, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
                         const GemmEpilogue& e, int* err, cudaStream_t st) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0) return cudaSuccess;
@@ -1190,6 +1556,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
     return cudaErrorInvalidValue;
   // pairs: no split, tiles at least 64 wide, the direct (TMA-store) epilogue
   if (s.pair && (s.splits != 1 || s.split_l2 || bn < 64)) return cudaErrorInvalidValue;
+  if (s.persist) return launch_persist(tmA, tmB, s, bn, e, err, st);
   if (e.qkv_d > 0 && (e.qkv_d % bn != 0 || s.N != 3 * e.qkv_d || e.t_len <= 0)) return cudaErrorInvalidValue;
   // Folded LayerNorm: row statistics come as partial sums indexed by row
   // (one clip batch); the normalised residual must be fp16.

@@ -429,12 +429,26 @@ bool l2_split_ok(const w2v_model* m, const GemmShape& s, int N, int bn, int sp) 
 // A GEMM role's launch form as one integer (plan files, refinement): 0 = CTA
 // pairs on 256-row tiles, 1 = one CTA per 128-row tile, s > 1 = s K splits
 // reduced through distributed shared memory, -s = s K splits through L2.
-int form_code(const GemmShape& s) { return s.pair ? 0 : (s.split_l2 ? -s.splits : s.splits); }
+// Form codes (plan files, tuner): 1 one CTA per tile; 2..8 K split through
+// the cluster; -2..-4 K split through the L2 scratch; 0 CTA pairs; 9
+// persistent CTAs with double-buffered accumulators.
+constexpr int kFormPersist = 9;
+
+int form_code(const GemmShape& s) {
+  return s.persist ? kFormPersist : (s.pair ? 0 : (s.split_l2 ? -s.splits : s.splits));
+}
 
 void set_form(GemmShape* s, int code) {
+  s->persist = code == kFormPersist;
   s->pair = code == 0;
-  s->splits = code == 0 ? 1 : (code < 0 ? -code : code);
+  s->splits = (code == 0 || code == kFormPersist) ? 1 : (code < 0 ? -code : code);
   s->split_l2 = code < 0;
+}
+
+// The persistent form pays off once the tiles outnumber the SMs.
+bool persist_worth(const GemmShape& s, int N, int bn) {
+  const long tiles = static_cast<long>((s.M + 127) / 128) * ((N + bn - 1) / bn) * s.batch;
+  return bn >= 64 && tiles > 148;
 }
 
 // The B operand map of a GEMM with tile width bn in form `code` (pairs load
@@ -453,7 +467,8 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     const bool bn_ok = (bn == 32 || bn == 64 || bn == 128 || bn == 192 || bn == 256) &&
                        (bn_divides <= 0 || bn_divides % bn == 0);
     const bool sp_ok = sp == 1 || (sp > 1 && sp <= 8 && s->batch == 1 && sp <= nk) ||
-                       ((sp >= -4 && sp <= -2) && l2_split_ok(m, *s, N, bn, -sp)) || (sp == 0 && bn >= 64);
+                       ((sp >= -4 && sp <= -2) && l2_split_ok(m, *s, N, bn, -sp)) || (sp == 0 && bn >= 64) ||
+                       (sp == kFormPersist && bn >= 64 && e.qkv_d == 0);
     if (!bn_ok || !sp_ok) return fail(m, W2V_EINVAL, "plan file: bn=%d splits=%d invalid for N=%d K=%d", bn, sp, N, K);
     (void)splits;
     set_form(s, sp);
@@ -478,15 +493,17 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     CUDA_OR(m, map_matrix(&tmB, W, N, K, bn));
     if (bn >= 64) CUDA_OR(m, map_b(&tmBp, W, N, K, bn, 0));
     // sp > 1: K splits reduced through distributed shared memory; sp < 0:
-    // -sp splits reduced through the L2 scratch; sp 0: CTA pairs
-    for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0}) {
-      if (sp > 1 && (s->batch != 1 || nk < 16 || sp > nk)) continue;
+    // -sp splits reduced through the L2 scratch; sp 0: CTA pairs; 9: persistent
+    for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0, kFormPersist}) {
+      if (sp > 1 && sp != kFormPersist && (s->batch != 1 || nk < 16 || sp > nk)) continue;
       if (sp < 0 && !l2_split_ok(m, *s, N, bn, -sp)) continue;
       if (sp == 0 && bn < 64) continue;
+      if (sp == kFormPersist && (e.qkv_d > 0 || !persist_worth(*s, N, bn))) continue;
       GemmShape c = *s;
       set_form(&c, sp);
       const cudaError_t lr = launch_gemm(tmA, sp == 0 ? tmBp : tmB, c, bn, e, m->err_word, st);
-      if (sp == 0 && lr == cudaErrorInvalidValue) continue;  // pairs need the direct epilogue
+      // pairs need the direct epilogue, the persistent form 16-byte rows
+      if ((sp == 0 || sp == kFormPersist) && lr == cudaErrorInvalidValue) continue;
       CUDA_OR(m, lr);
       CUDA_OR(m, cudaEventRecord(e0, st));
       for (int it = 0; it < 3; ++it) CUDA_OR(m, launch_gemm(tmA, sp == 0 ? tmBp : tmB, c, bn, e, m->err_word, st));
@@ -1351,10 +1368,11 @@ int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
     for (int bn : {32, 64, 128, 192, 256}) {
       if (bn == 32 ? N > 32 : N <= bn / 2) continue;
       if (role == 0 && d % bn != 0) continue;
-      for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0}) {
-        if (sp > 1 && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
+      for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0, kFormPersist}) {
+        if (sp > 1 && sp != kFormPersist && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
         if (sp < 0 && !l2_split_ok(m, *sh, N, bn, -sp)) continue;
         if (sp == 0 && bn < 64) continue;
+        if (sp == kFormPersist && (role == 0 || !persist_worth(*sh, N, bn))) continue;
         if (bn == cur_bn && sp == cur_s) continue;
         int rc = apply_role(m, p, role, bn, sp);
         if (rc != W2V_OK) return rc;
@@ -1835,6 +1853,8 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
     bn = gemm_pick(&s, 0);
   } else if (splits == 0) {
     s.pair = true;
+  } else if (splits == kFormPersist) {
+    s.persist = true;
   } else {
     s.splits = splits < 0 ? -splits : splits;
     s.split_l2 = splits < 0;
@@ -1842,7 +1862,7 @@ extern "C" int w2v_op_gemm(const void* A, const void* B, int M, int N, int K, co
   if (bn != 32 && bn != 64 && bn != 128 && bn != 192 && bn != 256) return W2V_EINVAL;
   if (s.splits < 1 || s.splits > 8 || s.splits > K / 64) return W2V_EINVAL;
   if (s.split_l2 && (s.splits < 2 || s.splits > 4 || bn < 64 || !gemm_l2_split_fits(bn, s.splits))) return W2V_EINVAL;
-  if (s.pair && bn < 64) return W2V_EINVAL;
+  if ((s.pair || s.persist) && bn < 64) return W2V_EINVAL;
   CUtensorMap ta, tb;
   if (map_a(&ta, A, K, M, K, 1, 0) != cudaSuccess) return W2V_ECUDA;
   if (map_matrix(&tb, B, N, K, s.pair ? bn / 2 : bn) != cudaSuccess) return W2V_ECUDA;

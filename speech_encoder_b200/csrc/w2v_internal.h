@@ -124,6 +124,9 @@ struct GemmShape : GemmDims {
                           // the last split to arrive finishing the tile)
   bool pair = false;      // CTA pairs on 256-row tiles (2-CTA tensor-core
                           // instructions); then tmB's box is {64, bn/2}, no split
+  bool persist = false;   // persistent CTAs (one per SM) walking the output tiles
+                          // with double-buffered TMEM accumulators; no split,
+                          // pair or QKV split, 16-byte aligned rows
 };
 
 // Chooses the N tile width (returned) and the split-K factor (s->splits) for

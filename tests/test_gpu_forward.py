@@ -328,7 +328,8 @@ def test_plan_file_pins_the_gemm_choices_across_models(tmp_path, monkeypatch):
     m3.close()
 
 
-@pytest.mark.parametrize("forms", [("128:2", "64:-2", "128:0", "64:4"), ("128:1", "128:2", "256:2", "128:2")])
+@pytest.mark.parametrize("forms", [("128:2", "64:-2", "128:0", "64:4"), ("128:1", "128:2", "256:2", "128:2"),
+                                   ("128:1", "64:9", "128:9", "64:9")])
 def test_every_split_form_in_the_encoder_matches_oracle(tmp_path, monkeypatch, forms):
     # A pinned plan puts each encoder GEMM of the post-norm model (folded
     # LayerNorms, partial row sums) on another form.  First: QKV split 2 ways
@@ -336,7 +337,8 @@ def test_every_split_form_in_the_encoder_matches_oracle(tmp_path, monkeypatch, f
     # out-projection split 2 ways through the L2 scratch with its fp16 residual
     # staged, FFN1 on CTA pairs, FFN2 split 4 ways by row bands.  Second: the
     # out-projection, FFN1 and FFN2 split through the cluster by column
-    # groups.  The logits still match the oracle.
+    # groups.  Third: the same three on persistent CTAs.  The logits still
+    # match the oracle.
     shape = S.small_shape()
     pcm = S.synth_pcm(30000, 9)
     path = tmp_path / "plans.txt"

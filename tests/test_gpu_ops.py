@@ -76,6 +76,14 @@ GEMM_CASES = [
     (799, 768, 3072, (256, 4), 0, "f16", 1),
     (300, 456, 1024, (192, 3), 2, "f32", 1),
     (1, 256, 512, (128, 2), 0, None, 0),
+    # persistent CTAs with double-buffered accumulators (splits 9): more tiles
+    # than SMs, ragged M and N, every tile width, residuals, both outputs
+    (7984, 768, 768, (128, 9), 0, "f16", 0),
+    (7984, 3072, 768, (192, 9), 2, None, 0),
+    (25599, 512, 1536, (256, 9), 1, None, 0),
+    (3001, 456, 512, (64, 9), 1, "f32", 1),
+    (1000, 200, 256, (128, 9), 0, "f16", 1),
+    (130, 96, 128, (64, 9), 2, None, 0),
 ]
 
 
@@ -113,7 +121,7 @@ def test_gemm_every_tile_width_same_result():
     W = (torch.randn(N, K, generator=g) * 0.05).half().cuda()
     outs = []
     for bn, sp in ((32, 1), (64, 1), (128, 1), (192, 1), (256, 1), (256, 2), (128, 8), (64, 3), (64, -3),
-                   (128, -3), (192, -2), (64, 0), (128, 0), (192, 0), (256, 0)):
+                   (128, -3), (192, -2), (64, 0), (128, 0), (192, 0), (256, 0), (64, 9), (256, 9)):
         out = torch.empty(M, N, dtype=torch.float32, device="cuda")
         assert B.w2v_op_gemm(A, W, M, N, K, None, None, 0, out, 1, 0, _err(), bn=bn, splits=sp) == 0
         outs.append(out)
