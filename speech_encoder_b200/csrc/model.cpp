@@ -495,7 +495,7 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     // sp > 1: K splits reduced through distributed shared memory; sp < 0:
     // -sp splits reduced through the L2 scratch; sp 0: CTA pairs; 9: persistent
     for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0, kFormPersist}) {
-      if (sp > 1 && sp != kFormPersist && (s->batch != 1 || nk < 16 || sp > nk)) continue;
+      if (sp > 1 && sp != kFormPersist && (s->batch != 1 || nk < 8 || sp > nk / 2)) continue;
       if (sp < 0 && !l2_split_ok(m, *s, N, bn, -sp)) continue;
       if (sp == 0 && bn < 64) continue;
       if (sp == kFormPersist && (e.qkv_d > 0 || !persist_worth(*s, N, bn))) continue;
@@ -1369,7 +1369,7 @@ int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
       if (bn == 32 ? N > 32 : N <= bn / 2) continue;
       if (role == 0 && d % bn != 0) continue;
       for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0, kFormPersist}) {
-        if (sp > 1 && sp != kFormPersist && (sh->batch != 1 || nk < 16 || sp > nk)) continue;
+        if (sp > 1 && sp != kFormPersist && (sh->batch != 1 || nk < 8 || sp > nk / 2)) continue;
         if (sp < 0 && !l2_split_ok(m, *sh, N, bn, -sp)) continue;
         if (sp == 0 && bn < 64) continue;
         if (sp == kFormPersist && (role == 0 || !persist_worth(*sh, N, bn))) continue;
