@@ -326,18 +326,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       if (res_tma) stage_residual();
       bool ok = true;
+      // Stage, phase and A coordinates advance incrementally: this thread's
+      // own instruction latency is on the mainloop's critical path.
+      int st = pre == nst ? 0 : pre;
+      uint32_t ph = pre == nst ? 1u : 0u;
+      int k = (kb0 + pre) * C::BK;
+      int kx = k % s.a_kwrap, ky = k / s.a_kwrap;
       for (int i = pre; i < nkl; ++i) {
-        const int st = i % nst;
-        if (!mbar_wait(&empty[st], ((i / nst) & 1) ^ 1)) {
+        if (!mbar_wait(&empty[st], ph ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
           break;
         }
         uint8_t* sa = smem + st * C::STAGE;
         if (prank == 0) mbar_arrive_expect_tx(&full[st], 2 * C::STAGE);
-        const int k = (kb0 + i) * C::BK;
-        tma_load_3d_pair(sa, &tmA, fbar(st), k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
+        tma_load_3d_pair(sa, &tmA, fbar(st), kx, m0 + ky, bzb);
         tma_load_2d_pair(sa + C::A_BYTES, &tmB, fbar(st), k, nb0);
+        k += C::BK;
+        kx += C::BK;
+        if (kx == s.a_kwrap) {
+          kx = 0;
+          ++ky;
+        }
+        if (++st == nst) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
       // Wait until the last stages have been consumed: every copy into this
       // CTA has landed and every release the MMA issuer sent here has
@@ -387,9 +401,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (res_tma) stage_residual();
       int issued = pre;
       bool ok = true;
+      // Stage, phase and A coordinates advance incrementally: this thread's
+      // own instruction latency is on the mainloop's critical path.
+      int st = pre == nst ? 0 : pre;
+      uint32_t ph = pre == nst ? 1u : 0u;
+      int k = (kb0 + pre) * C::BK;
+      int kx = k % s.a_kwrap, ky = k / s.a_kwrap;
       for (int i = pre; i < nkl; ++i) {
-        const int st = i % nst;
-        const uint32_t ph = (i / nst) & 1;
         if (!mbar_wait(&empty[st], ph ^ 1)) {
           atomicOr(err, kErrWaitProducer);
           ok = false;
@@ -397,10 +415,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         uint8_t* sa = smem + st * C::STAGE;
         mbar_arrive_expect_tx(&full[st], C::STAGE);
-        const int k = (kb0 + i) * C::BK;
-        tma_load_3d(sa, &tmA, &full[st], k % s.a_kwrap, m0 + k / s.a_kwrap, bzb);
+        tma_load_3d(sa, &tmA, &full[st], kx, m0 + ky, bzb);
         tma_load_2d(sa + C::A_BYTES, &tmB, &full[st], k, n0);
         issued = i + 1;
+        k += C::BK;
+        kx += C::BK;
+        if (kx == s.a_kwrap) {
+          kx = 0;
+          ++ky;
+        }
+        if (++st == nst) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA exits.
@@ -1122,6 +1149,7 @@ gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         int m0, n0, bz;
         tile_of(t, m0, n0, bz);
+        int kx = 0, ky = 0;  // A coordinates, advanced incrementally
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[st], ph ^ 1)) {
             atomicOr(err, kErrWaitProducer);
@@ -1130,9 +1158,13 @@ gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
           uint8_t* sa = smem + st * C::STAGE;
           mbar_arrive_expect_tx(&full[st], C::STAGE);
-          const int k = kb * C::BK;
-          tma_load_3d(sa, &tmA, &full[st], k % s.a_kwrap, m0 + k / s.a_kwrap, bz);
-          tma_load_2d(sa + C::A_BYTES, &tmB, &full[st], k, n0);
+          tma_load_3d(sa, &tmA, &full[st], kx, m0 + ky, bz);
+          tma_load_2d(sa + C::A_BYTES, &tmB, &full[st], kb * C::BK, n0);
+          kx += C::BK;
+          if (kx == s.a_kwrap) {
+            kx = 0;
+            ++ky;
+          }
           ++issued;
           if (++st == C::STAGES) {
             st = 0;
