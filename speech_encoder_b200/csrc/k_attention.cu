@@ -9,8 +9,9 @@
 //               K=64) into one of three TMEM score buffers and, once P_j is in
 //               shared memory, O += P_j [V_j | 1] (M=128, N=80, K=128) into a
 //               TMEM accumulator that lives across all key tiles.  The scores
-//               run two tiles ahead (S_{j+2} is issued before waiting for
-//               P_j), so the softmax never waits behind a P V product: every
+//               run up to two tiles ahead (S_{j+2} is issued as soon as its
+//               K/V tile lands, polled together with P_j), so neither the
+//               softmax nor P V waits behind the other's operands: every
 //               tcgen05.mma of M=128, K=16 occupies the tensor pipe about the
 //               same ~100-140 cycles whatever its N up to 192, which makes the
 //               eight P V instructions per tile the longer of the two chains.
@@ -93,7 +94,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
       mbar_init(&s_full[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&p_full[i], 32 * kSoftWarps);
+      mbar_init(&p_full[i], kSoftWarps);  // one arrival per softmax warp
       mbar_init(&pv_done[i], 1);
     }
     fence_mbar_init();
@@ -180,18 +181,32 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
           }
         }
       }
+      // S_m may be issued once its K/V stage has landed and P_{m-3} was seen
+      // (S_m reuses the score buffer of S_{m-3}, whose softmax finished reading
+      // it before publishing P_{m-3}): m <= j + 2 while waiting for P_j.  The
+      // thread polls both, so P_j V_j never waits behind a K/V tile that is
+      // still in flight (that tile's stage is only refilled after an earlier
+      // P V completes).
+      int next_s = nkv > 1 ? 2 : 1;
       for (int j = 0; ok && j < nkv; ++j) {
-        // S_{j+2} reuses the score buffer of S_{j-1}, whose softmax finished
-        // reading it before P_{j-1} was published.
-        if (j + 2 < nkv) {
-          if (!mbar_wait(&kv_full[(j + 2) % kKvStages], ((j + 2) / kKvStages) & 1)) {
-            ok = false;
+        bool have_p = false;
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 1;; ++it) {
+          // test_wait: a try_wait on a phase still open may suspend the
+          // thread for a while, delaying the other barrier's detection
+          if (next_s < nkv && next_s <= j + 2 &&
+              mbar_test_wait(&kv_full[next_s % kKvStages], (next_s / kKvStages) & 1)) {
+            tc_fence_after();
+            issue_s(next_s);
+            ++next_s;
+          }
+          if (mbar_test_wait(&p_full[j & 1], (j >> 1) & 1)) {
+            have_p = true;
             break;
           }
-          tc_fence_after();
-          issue_s(j + 2);
+          if ((it & 255u) == 0 && globaltimer_ns() - t0 > W2V_WAIT_LIMIT_NS) break;
         }
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) {
+        if (!have_p) {
           ok = false;
           break;
         }
@@ -294,7 +309,9 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
             make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      // one arrival per warp: 512 arrivals on one barrier word serialise
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[j & 1]);
     }
     const int last = nkv - 1;
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[last & 1], (last >> 1) & 1));
