@@ -953,21 +953,109 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int i = 0; i < 4; ++i) dst[static_cast<int64_t>(i) * e.t_pad] = __float2half_rn(x[i]);
         }
       } else {
+        // Every partial, this CTA's own included, is in shared memory, so any
+        // warp can finish any row: lane = row (band rows 32 g .. 32 g + 31,
+        // g = epilogue warp / 4), and the warp's 32-column chunks are
+        // (epilogue warp % 4) + 4 k.  The direct form's chunk arithmetic, the
+        // partial sums in split order 0..S-1, 16-byte stores from registers.
         void* outp = region == 1 ? e.out_k : e.out;
         const int ocol0 = region > 0 ? region * e.qkv_d : 0;
-        const int total = e.ln_out ? 0 : nrows * C::ROW_CHUNKS;
-        if (e.ln_out) finish_rows_stats(r0, nrows, outp, ocol0, fetch);
-#pragma unroll 2
-        for (int idx = et; idx < total; idx += kEpiThreads) {
-          const int lr = idx / C::ROW_CHUNKS;
-          const int j = idx - lr * C::ROW_CHUNKS;
-          const int grow = m0 + r0 + lr;
-          const int col = n0 + 4 * j;
-          if (grow >= s.M || col >= s.N) continue;
-          const float4 v = fetch(lr, j);
-          float x[4] = {v.x, v.y, v.z, v.w};
-          finish4(x, bias_s, vec_s, BN, row_lnr(r0 + lr), 4 * j, grow, col, min(4, s.N - col), bzb, e, outp,
-                  ocol0, vec, res_tma ? res_s : nullptr, r0 + lr);
+        const int ew = warp - 2;
+        const int lr = (ew >> 2) * 32 + lane;
+        const int rt = r0 + lr;  // tile row
+        const int grow = m0 + rt;
+        const bool live = lr < nrows && grow < s.M;
+        const float2 lnr = live ? row_lnr(rt) : make_float2(1.f, 0.f);
+        const bool vec16 = vec && ((e.ldo * (e.out_f32 ? 4 : 2)) % 16 == 0);
+#pragma unroll 1
+        for (int cb = ew & 3; cb < BN / 32 && (ew >> 2) * 32 < nrows; cb += 4) {
+          const int c = cb * 32;
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          if (live) {
+            for (int p = 0; p < S; ++p) {
+              const uint8_t* src = smem + p * slot_bytes;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float4 pv = *reinterpret_cast<const float4*>(src + swz_off(C::ROW_CHUNKS, lr, (c >> 2) + k));
+                v[4 * k] += pv.x;
+                v[4 * k + 1] += pv.y;
+                v[4 * k + 2] += pv.z;
+                v[4 * k + 3] += pv.w;
+              }
+            }
+          }
+          if (ln_mode == 1) ln1_cols<32>(v, vec_s + c, lnr);
+          add_cols<32>(v, bias_s + c);
+          act_inplace<32>(v, e.act);
+          const int col = n0 + c;
+          const int nv = min(32, s.N - col);
+          if (!live || nv <= 0) continue;
+          if (e.residual) {
+            const int64_t roff =
+                static_cast<int64_t>(bzb) * e.res_batch_stride + static_cast<int64_t>(grow) * e.ldr + col;
+            float f[32];
+            if (res_tma) {
+              const uint8_t* rb = res_s + cb * 8192 + rt * 64;
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                const uint4 u = *reinterpret_cast<const uint4*>(rb + (((i >> 3) ^ ((rt >> 1) & 3)) << 4));
+                const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float2 t = __half22float2(h[k]);
+                  f[i + 2 * k] = t.x;
+                  f[i + 2 * k + 1] = t.y;
+                }
+              }
+            } else if (e.res_f32) {
+              const float* rp = static_cast<const float*>(e.residual) + roff;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) f[i] = i < nv ? rp[i] : 0.f;
+            } else {
+              const __half* rp = static_cast<const __half*>(e.residual) + roff;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) f[i] = i < nv ? __half2float(rp[i]) : 0.f;
+            }
+            add_residual<32>(v, f, ln_mode, vec_s + c, BN, lnr);
+          }
+          if (e.ln_out) {
+            float st1 = 0.f, st2 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nv) {
+                st1 += v[i];
+                st2 = fmaf(v[i], v[i], st2);
+              }
+            e.ln_out[static_cast<int64_t>(col >> 5) * s.M + grow] = make_float2(st1, st2);
+          }
+          const int64_t ooff =
+              static_cast<int64_t>(bzb) * e.out_batch_stride + static_cast<int64_t>(grow) * e.ldo + (col - ocol0);
+          if (e.out_f32) {
+            float* op = static_cast<float*>(outp) + ooff;
+            if (vec16 && nv == 32) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<float4*>(op + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (k < nv) op[k] = v[k];
+            }
+          } else {
+            __half* op = static_cast<__half*>(outp) + ooff;
+            if (vec16 && nv == 32) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 8)
+                *reinterpret_cast<uint4*>(op + k) = make_uint4(pack_h2(v[k], v[k + 1]), pack_h2(v[k + 2], v[k + 3]),
+                                                               pack_h2(v[k + 4], v[k + 5]), pack_h2(v[k + 6], v[k + 7]));
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (k < nv) op[k] = __float2half_rn(v[k]);
+            }
+          }
         }
       }
     }
