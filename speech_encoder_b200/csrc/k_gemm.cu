@@ -58,6 +58,14 @@ struct GemmCfg {
   static constexpr int ROWLN_OFF = VEC_OFF + 2 * BN * 4;  // per-row LN factors, 128 float2
   static constexpr int BAR_OFF = ROWLN_OFF + 128 * 8;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  // Row LayerNorm over a cluster of column tiles (ln_mode 3): per row the two
+  // half-tile (count, mean, M2) and one slot per cluster CTA (up to 8),
+  // outside the ring so that peers may write before this CTA's ring drains.
+  // Only those launches request it (a larger request shrinks the SM's L1).
+  static constexpr int LN3_OFF = BAR_OFF + 256;
+  static constexpr int LN3_BYTES = (2 + 8) * 128 * 16;
+  static constexpr int SMEM_LN3 = SMEM + LN3_BYTES;
+  static_assert(SMEM_LN3 <= 227 * 1024, "a CTA's dynamic shared memory is at most 227 KB");
   // An fp16 residual tile (128 rows x BN) staged by TMA during the mainloop
   // takes the ring's last RES_STAGES stages.
   static constexpr int RES_BYTES = BM * BN * 2;
@@ -213,8 +221,9 @@ __device__ __forceinline__ void finish4(float (&x)[4], const float* bias_s, cons
 // memory (each cluster CTA finishing a band of rows), 3 split-K through an L2
 // scratch, 4 split-K through distributed shared memory (each cluster CTA
 // finishing a group of columns); 3 and 4 with the direct stores.
-// SPLIT: the instantiation for split-K launches (modes 2-4); the other one
-// runs modes 0 and 1 only.
+// SPLIT: the instantiation with cluster code, for split-K launches (modes
+// 2-4) and the row-LayerNorm epilogue (mode 1, ln_mode 3); the other one runs
+// modes 0 and 1 only.
 // PAIR: CTA pairs (clusters of 2 along M) on 256-row tiles with the 2-CTA
 // tensor-core instructions, mode 1 only.  The pair halves the B operand bytes
 // each SM takes in per output, which bounds the mainloop (an SM receives
@@ -299,6 +308,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   // pairs: both CTAs' barriers are initialised before either signals the other
   if (PAIR) cluster_sync();
+  // row LayerNorm over a cluster: announce that this CTA runs; the epilogue
+  // waits for every peer's announcement before writing into their memory
+  // (the cluster instantiation only: the plain one carries no cluster code)
+  const bool ln3_cluster = SPLIT && !PAIR && mode == 1 && (e.ln_cfg & 255) == 3;
+  if (ln3_cluster) cluster_arrive_relaxed();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // The fp16 residual tile of this CTA's 128 rows, as BN/32 boxes of 32
@@ -482,13 +496,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (e.bias && n0 + i < s.N) ? e.bias[n0 + i] : 0.f;
     if (ln_mode == 1) {
       for (int i = et; i < BN; i += kEpiThreads) vec_s[i] = n0 + i < s.N ? e.ln_vec[n0 + i] : 0.f;
-    } else if (ln_mode == 2) {
+    } else if (ln_mode == 2 || ln_mode == 3) {
       for (int i = et; i < BN; i += kEpiThreads) {
         vec_s[i] = n0 + i < s.N ? e.ln_vec[n0 + i] : 0.f;
         vec_s[BN + i] = n0 + i < s.N ? e.ln_vec[s.N + n0 + i] : 0.f;
       }
     }
-    if (ln_mode != 0) {
+    if (ln_mode == 1 || ln_mode == 2) {
       // Row statistics from the partial sums the producing GEMM stored (it is
       // a previous kernel: wait for it here, while the mainloop runs), added
       // in partial order: rowln_s[row] = (rstd, -mean * rstd).  The width is
@@ -758,8 +772,77 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (et == 0) tickets[tile] = 0;  // ready for the next launch
       }
     }
+    if (ln3_cluster) {
+      // LayerNorm of each output row over all N columns, held by the CY =
+      // gridDim.y CTAs of this cluster (BN each), applied to acc + bias before
+      // the activation.  Each thread takes (count, mean, centred sum of
+      // squares) of its row's half tile (two passes over TMEM), and the parts
+      // combine by Chan's formula in a fixed order: the two halves in shared
+      // memory, then one slot per cluster CTA through distributed shared
+      // memory (every CTA writes its row parts into every CTA's slot).
+      float4* half_s = reinterpret_cast<float4*>(smem + C::LN3_OFF);      // [2][128]
+      float4* slot_s = half_s + 2 * 128;                                 // [CY][128]
+      const int cy = static_cast<int>(gridDim.y);
+      const uint32_t crank = cluster_ctarank();
+      cluster_wait();  // every CTA of the cluster is running
+      auto chan = [](float4 a, float4 b) -> float4 {
+        const float n = a.x + b.x;
+        if (n == 0.f) return a;
+        const float d = b.y - a.y;
+        return make_float4(n, a.y + d * (b.x / n), a.z + b.z + d * d * (a.x * b.x / n), 0.f);
+      };
+      if (epi) {
+        named_barrier_sync(1, kEpiThreads);  // bias staged
+        float cnt = 0.f, sum = 0.f;
+#pragma unroll 1
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+          float v[32];
+          if (ok) tmem_ld32(trow + c, v);
+          add_cols<32>(v, bias_s + c);
+          const int nv = min(32, s.N - (n0 + c));
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) sum += v[i];
+          cnt += static_cast<float>(max(nv, 0));
+        }
+        const float mu = cnt > 0.f ? sum / cnt : 0.f;
+        float m2 = 0.f;
+#pragma unroll 1
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+          float v[32];
+          if (ok) tmem_ld32(trow + c, v);
+          add_cols<32>(v, bias_s + c);
+          const int nv = min(32, s.N - (n0 + c));
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) {
+              const float dv = v[i] - mu;
+              m2 = fmaf(dv, dv, m2);
+            }
+        }
+        half_s[half * 128 + r] = make_float4(cnt, mu, m2, 0.f);
+        named_barrier_sync(1, kEpiThreads);
+        if (half == 0) {
+          const float4 part = chan(half_s[r], half_s[128 + r]);
+          const uint32_t dst = smem_u32(slot_s + crank * 128 + r);
+          for (int p = 0; p < cy; ++p)
+            st_dsmem_f4(mapa_shared(dst, static_cast<uint32_t>(p)), part);
+        }
+      }
+      cluster_sync();  // every CTA's row parts are in every CTA's slots
+      if (epi) {
+        if (half == 0) {
+          float4 tot = slot_s[r];
+          for (int p = 1; p < cy; ++p) tot = chan(tot, slot_s[p * 128 + r]);
+          const float var = tot.x > 0.f ? tot.z / tot.x : 0.f;
+          const float rstd = rsqrtf(var + e.ln_eps);
+          rowln_s[r] = make_float2(rstd, -tot.y * rstd);
+        }
+        named_barrier_sync(1, kEpiThreads);
+      }
+    }
     if (epi && owner) {
-      if (mode == 1) named_barrier_sync(1, kEpiThreads);  // bias staged (mode 3: the ticket barriers)
+      if (mode == 1 && !ln3_cluster) named_barrier_sync(1, kEpiThreads);  // bias staged (mode 3: the ticket barriers)
       const int grow = m0 + r;
       void* outp = region == 1 ? e.out_k : e.out;
       const int ocol0 = region > 0 ? region * e.qkv_d : 0;
@@ -798,6 +881,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         if (ln_mode == 1) ln1_cols<32>(v, vec_s + c, lnr);
         add_cols<32>(v, bias_s + c);
+        if (ln3_cluster) {  // (v - mean) * rstd * gamma + beta (cluster instantiation only)
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 g = *reinterpret_cast<const float4*>(vec_s + c + i);
+            const float4 b = *reinterpret_cast<const float4*>(vec_s + BN + c + i);
+            v[i] = fmaf(fmaf(v[i], lnr.x, lnr.y), g.x, b.x);
+            v[i + 1] = fmaf(fmaf(v[i + 1], lnr.x, lnr.y), g.y, b.y);
+            v[i + 2] = fmaf(fmaf(v[i + 2], lnr.x, lnr.y), g.z, b.z);
+            v[i + 3] = fmaf(fmaf(v[i + 3], lnr.x, lnr.y), g.w, b.w);
+          }
+        }
         act_inplace<32>(v, e.act);
         const int col = n0 + c;
         const int nv = min(32, s.N - col);
@@ -1556,7 +1650,7 @@ static cudaError_t prepare_bn() {
                                        GemmCfg<BN>::SMEM);
   if (r == cudaSuccess)
     r = cudaFuncSetAttribute(gemm_tc_kernel<BN, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<BN>::SMEM);
+                             GemmCfg<BN>::SMEM_LN3);
   if (r == cudaSuccess && BN >= 64)
     r = cudaFuncSetAttribute(gemm_tc_kernel<BN, false, (BN >= 64)>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<BN, (BN >= 64)>::SMEM);
@@ -1591,7 +1685,8 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = pair ? GemmCfg<BN, (BN >= 64)>::SMEM : GemmCfg<BN>::SMEM;
+  cfg.dynamicSmemBytes = pair ? GemmCfg<BN, (BN >= 64)>::SMEM
+                              : ((e.ln_cfg & 255) == 3 ? GemmCfg<BN>::SMEM_LN3 : GemmCfg<BN>::SMEM);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1601,9 +1696,15 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
   attr[1].val.clusterDim.y = 1;
   // the cluster forms (modes 2 and 4); the L2 form (mode 3) needs no cluster
   const bool cluster_split = S > 1 && ((mode & 15) == 2 || (mode & 15) == 4);
+  // row LayerNorm: the column tiles of a row block form one cluster along y
+  const bool cluster_ln = (e.ln_cfg & 255) == 3;
+  if (cluster_ln) {
+    attr[1].val.clusterDim.y = grid.y;
+    if (pair || S > 1 || (mode & 15) != 1) return cudaErrorInvalidValue;
+  }
   attr[1].val.clusterDim.z = cluster_split ? S : 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (cluster_split || pair) ? 2 : 1;
+  cfg.numAttrs = (cluster_split || pair || cluster_ln) ? 2 : 1;
   const GemmDims sd = s;      // the kernel's parameter block holds only
   GemmEpiArgs ea = e;         // what it reads
   if ((mode & 15) == 3) ea.out_k = e.split_tickets;  // the L2 form's tickets (out_k is a QKV-only field)
@@ -1612,10 +1713,12 @@ static cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, con
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, (BN >= 64)>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
                               mode, err);
   }
-  return S > 1 ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, true, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
-                                    mode, err)
-               : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok,
-                                    mode, err);
+  // the cluster instantiation for split-K and for the row LayerNorm
+  return (S > 1 || cluster_ln)
+             ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, true, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok, mode,
+                                  err)
+             : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, false, false>, tmA, tmB, tmO, tmO2, tmV, sd, ea, vec_ok, mode,
+                                  err);
 }
 
 // The persistent form: no split, pair or QKV split; 16-byte vector stores of
@@ -1650,7 +1753,8 @@ static cudaError_t launch_persist_bn(const CUtensorMap& tmA, const CUtensorMap& 
 
 static cudaError_t launch_persist(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmShape& s, int bn,
                                   const GemmEpilogue& e, int* err, cudaStream_t st) {
-  if (s.splits != 1 || s.split_l2 || s.pair || e.qkv_d > 0 || !e.out) return cudaErrorInvalidValue;
+  if (s.splits != 1 || s.split_l2 || s.pair || e.qkv_d > 0 || !e.out || (e.ln_cfg & 255) > 2)
+    return cudaErrorInvalidValue;
   const int esz_out = e.out_f32 ? 4 : 2;
   const int esz_res = e.res_f32 ? 4 : 2;
   const bool out_ok = reinterpret_cast<uintptr_t>(e.out) % 16 == 0 && (e.ldo * esz_out) % 16 == 0 &&
@@ -1681,7 +1785,12 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   // Folded LayerNorm: row statistics come as partial sums indexed by row
   // (one clip batch); the normalised residual must be fp16.
   const int ln_mode = e.ln_cfg & 255;
-  if (ln_mode > 2 || (ln_mode != 0 && (!e.ln_vec || !e.ln_in || (e.ln_cfg >> 8) < 1 || s.batch != 1)))
+  if (ln_mode > 3 || ((ln_mode == 1 || ln_mode == 2) && (!e.ln_vec || !e.ln_in || (e.ln_cfg >> 8) < 1 || s.batch != 1)))
+    return cudaErrorInvalidValue;
+  // Row LayerNorm of the output (ln_mode 3): the N / bn column tiles of a row
+  // block form a cluster (at most 8), one CTA per tile, the direct epilogue.
+  if (ln_mode == 3 && (!e.ln_vec || s.N % bn != 0 || s.N / bn > 8 || s.splits != 1 || s.split_l2 || s.pair ||
+                       s.persist || e.qkv_d > 0 || e.residual || e.ln_out || bn < 64))
     return cudaErrorInvalidValue;
   if (ln_mode == 2 && (!e.residual || e.res_f32)) return cudaErrorInvalidValue;
   if (e.ln_out && (s.batch != 1 || e.qkv_d > 0)) return cudaErrorInvalidValue;
@@ -1745,6 +1854,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   }
   if (l2split && mode != 3) return cudaErrorInvalidValue;
   if (s.pair && mode != 1) return cudaErrorInvalidValue;
+  if (ln_mode == 3 && mode != 1) return cudaErrorInvalidValue;
   // An fp16 residual is staged in shared memory by TMA while the mainloop
   // runs (boxes of 32 columns x 128 rows, 64-byte swizzle), when the ring's
   // remaining stages still hold the epilogue's own staging.

@@ -148,6 +148,9 @@ struct Plan {
   CUtensorMap convA[7], convB[7];
   GemmShape convS[7];
   int convBN[7] = {};
+  // layer layout: conv layer i's LayerNorm runs in its GEMM's epilogue (the
+  // column tiles of a row block in one cluster) rather than as its own kernel
+  bool convLn3[7] = {};
   CUtensorMap projA, projB;
   GemmShape projS;
   int projBN = 0;
@@ -177,6 +180,7 @@ struct w2v_model {
   float* cb[7] = {};
   float* cg[7] = {};
   float* cbeta[7] = {};
+  float* cgb[7] = {};  // layer layout: [gamma; beta] of conv layer i's LayerNorm, for the GEMM epilogue
   float *fpg = nullptr, *fpb = nullptr;
   __half* wp = nullptr;
   float* bp = nullptr;
@@ -308,7 +312,15 @@ GemmEpilogue epi_conv(const w2v_model* m, const Plan& p, int i) {
   e.out = (i % 2 == 0) ? m->act_a : m->act_b;
   e.ldo = kC;
   e.out_batch_stride = static_cast<int64_t>(p.Tpad[i]) * kC;
-  e.act = (m->cfg.conv_norm == 0) ? (m->cfg.gelu_tanh ? 2 : 1) : 0;
+  // GELU after the LayerNorm: in this epilogue, or in the LayerNorm kernel
+  e.act = (m->cfg.conv_norm == 0 || p.convLn3[i]) ? (m->cfg.gelu_tanh ? 2 : 1) : 0;
+  if (m->cfg.conv_norm == 1 && p.convLn3[i]) {
+    // layer layout: bias, LayerNorm over the 512 channels of each frame (the
+    // column tiles of a row block form a cluster), then GELU
+    e.ln_cfg = 3;
+    e.ln_vec = m->cgb[i];
+    e.ln_eps = m->cfg.ln_eps;
+  }
   return e;
 }
 
@@ -469,7 +481,10 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
     const bool sp_ok = sp == 1 || (sp > 1 && sp <= 8 && s->batch == 1 && sp <= nk) ||
                        ((sp >= -4 && sp <= -2) && l2_split_ok(m, *s, N, bn, -sp)) || (sp == 0 && bn >= 64) ||
                        (sp == kFormPersist && bn >= 64 && e.qkv_d == 0);
-    if (!bn_ok || !sp_ok) return fail(m, W2V_EINVAL, "plan file: bn=%d splits=%d invalid for N=%d K=%d", bn, sp, N, K);
+    // a row-LayerNorm epilogue needs one CTA per column tile, 2..8 tiles a row
+    const bool ln3_ok = (e.ln_cfg & 255) != 3 || (sp == 1 && bn >= 64 && N % bn == 0 && N / bn <= 8);
+    if (!bn_ok || !sp_ok || !ln3_ok)
+      return fail(m, W2V_EINVAL, "plan file: bn=%d splits=%d invalid for N=%d K=%d", bn, sp, N, K);
     (void)splits;
     set_form(s, sp);
     *bn_out = bn;
@@ -486,9 +501,11 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
   CUDA_OR(m, cudaEventCreate(&e1));
   float best = 1e30f;
   int best_bn = 0, best_s = 1;
+  const bool ln3 = (e.ln_cfg & 255) == 3;
   for (int bn : {32, 64, 128, 192, 256}) {
     if (bn == 32 ? N > 32 : N <= bn / 2) continue;
     if (bn_divides > 0 && bn_divides % bn != 0) continue;
+    if (ln3 && (bn < 64 || N % bn != 0 || N / bn > 8)) continue;
     CUtensorMap tmB, tmBp;
     CUDA_OR(m, map_matrix(&tmB, W, N, K, bn));
     if (bn >= 64) CUDA_OR(m, map_b(&tmBp, W, N, K, bn, 0));
@@ -499,6 +516,7 @@ int tune_gemm(w2v_model* m, GemmShape* s, const CUtensorMap& tmA, const __half* 
       if (sp < 0 && !l2_split_ok(m, *s, N, bn, -sp)) continue;
       if (sp == 0 && bn < 64) continue;
       if (sp == kFormPersist && (e.qkv_d > 0 || !persist_worth(*s, N, bn))) continue;
+      if (ln3 && sp != 1) continue;
       GemmShape c = *s;
       set_form(&c, sp);
       const cudaError_t lr = launch_gemm(tmA, sp == 0 ? tmBp : tmB, c, bn, e, m->err_word, st);
@@ -551,8 +569,20 @@ int build_frontend(w2v_model* m, int n, int batch, Plan* p, bool analytic) {
     s.K = K;
     s.a_kwrap = 2 * kC;
     s.batch = batch;
+    // Layer layout: the analytic plans (one per clip length of a varlen call,
+    // whose short clips make the frontend launch-bound) fuse the LayerNorm
+    // into the GEMM (a cluster per row block: one launch per layer instead of
+    // two, true-length clips 11 679 -> 12 767 audio-s/s).  Tuned plans keep a
+    // LayerNorm kernel after the GEMM: their conv layers take the persistent
+    // and other forms the fused epilogue cannot use, and measured the fused
+    // form slower on the 16 s window of the large model (2.05 vs 1.96 ms).
+    p->convLn3[i] = m->cfg.conv_norm == 1 && analytic;
     if (analytic) {
       p->convBN[i] = gemm_pick(&s, 0);
+      if (p->convLn3[i]) {  // the row-LayerNorm epilogue: one CTA per column tile
+        s.splits = 1;
+        if (p->convBN[i] < 64 || kC % p->convBN[i] != 0) p->convBN[i] = 256;
+      }
     } else {
       const int rc = tune_gemm(m, &s, p->convA[i], m->cw[i], kC, K, epi_conv(m, *p, i), 0, &p->convBN[i]);
       if (rc != W2V_OK) return rc;
@@ -843,7 +873,7 @@ int enqueue_frontend(w2v_model* m, const Plan& p, const float* pcm, __half* out6
     LAUNCH(W2V_K_CONV_GEMM, 2.0 * p.T[i] * kC * K * B,
            2.0 * kC * (p.T[i - 1] + p.T[i]) * B + 2.0 * kC * K,
            launch_gemm(p.convA[i], p.convB[i], p.convS[i], p.convBN[i], e, m->err_word, st));
-    if (c.conv_norm == 1)
+    if (c.conv_norm == 1 && !p.convLn3[i])
       LAUNCH(W2V_K_CONV_LN, 0.0, 4.0 * kC * p.Tpad[i] * B,
              launch_layernorm(e.out, 0, static_cast<__half*>(e.out), B * p.Tpad[i], kC, m->cg[i], m->cbeta[i], eps,
                               act, st));
@@ -1126,6 +1156,12 @@ extern "C" int w2v_create(const w2v_config* cfg, const float* host_weights, size
     if (c.conv_norm == 1) {
       put_f32(reinterpret_cast<void**>(&m->cg[i]), src(p + ".norm.weight"), kC);
       put_f32(reinterpret_cast<void**>(&m->cbeta[i]), src(p + ".norm.bias"), kC);
+      if (i > 0) {  // [gamma; beta] for the conv GEMM's row-LayerNorm epilogue
+        const size_t o = take(2 * kC * 4);
+        std::memcpy(host.data() + o, src(p + ".norm.weight"), kC * 4);
+        std::memcpy(host.data() + o + kC * 4, src(p + ".norm.bias"), kC * 4);
+        fix.push_back({o, reinterpret_cast<void**>(&m->cgb[i])});
+      }
     }
   }
   put_f32(reinterpret_cast<void**>(&m->fpg), src("fp.norm.weight"), kC);

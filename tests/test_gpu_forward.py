@@ -47,6 +47,26 @@ def test_small_model_matches_oracle(layout, n):
     model.close()
 
 
+@pytest.mark.parametrize("layout", ["layer_stable", "layer_stable_tanh"])
+def test_layer_layout_conv_layernorms_both_forms(layout):
+    # Two full 48000-sample clips through the tuned plan (each conv layer's
+    # LayerNorm a kernel after its GEMM), then the same clips through the
+    # varlen entry point, whose analytic plan normalises inside the conv GEMMs
+    # (a cluster per row block).  Both match the oracle.
+    shape = S.small_shape(**LAYOUTS[layout])
+    model = U.make_model(shape, max_samples=48000, max_batch=2, seed=3, affine_noise=True)
+    pcm = np.stack([S.synth_pcm(48000, 23), S.synth_pcm(48000, 24)])
+    got = _run(model, pcm)
+    logits, frames = model.forward_varlen([torch.from_numpy(pcm[0]).cuda(), torch.from_numpy(pcm[1]).cuda()])
+    model.sync()
+    vl = logits.cpu().numpy()
+    for b in range(2):
+        ref = U.oracle_logits(shape, pcm[b], seed=3, affine_noise=True)
+        U.compare_logits(got[b], ref, f"{layout} n=48000 clip {b}")
+        U.compare_logits(vl[b * frames[0]:(b + 1) * frames[0]], ref, f"{layout} n=48000 varlen clip {b}")
+    model.close()
+
+
 @pytest.mark.parametrize("layout", ["group_post", "group_post_tanh"])
 def test_unfolded_post_norm_matches_oracle(layout, monkeypatch):
     # W2V_LN_FOLD=0 at create time keeps the post-norm LayerNorms as their own
