@@ -57,7 +57,7 @@ constexpr int kSubs = kSoftWarps / 4;    // warps per TMEM lane quarter
 constexpr int kSCols = 128 / kSubs;      // score columns per warp
 constexpr int kOCols = 64 / kSubs;       // output columns per warp
 constexpr float kLazyLimit = 8.0f;       // log2 of the largest P value allowed (256)
-constexpr int kPolyPairs = 6;            // exponential pairs per warp and tile computed by polynomial
+constexpr int kPolyPairs = 6 * (kSCols / 32);  // exponential pairs per warp and tile computed by polynomial
 
 __device__ __forceinline__ void quarter_barrier(int q) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kSubs) : "memory");
@@ -226,14 +226,16 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
     }
   } else {
     const int q = warp & 3;
-    const int sub = (warp - 2) >> 2;  // score columns [32 sub, 32 sub + 32), output columns [16 sub, 16 sub + 16)
+    const int sub = (warp - 2) >> 2;  // score columns [kSCols sub, +kSCols), output columns [kOCols sub, +kOCols)
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float c = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
     float m_ref = -INFINITY;                        // reference maximum, log2 units
-    // This warp's 32 keys are half of a 64-key swizzle atom (sub >> 1).
-    const int prow_off = AttnSmem::P + (sub >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
-    const int ch0 = (sub & 1) * 4;
+    // This warp's keys within the 64-key swizzle atoms of P: 32 keys are half
+    // of atom sub >> 1 (chunks from ch0), 64 keys are atom sub.
+    const int atom = kSCols >= 64 ? sub : (sub >> 1);
+    const int prow_off = AttnSmem::P + atom * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+    const int ch0 = kSCols >= 64 ? 0 : (sub & 1) * 4;
     bool ok = true;
     // Every iteration runs the quarter barrier and the p_full arrival even
     // after a failed wait (the work is skipped), so no thread is left waiting
@@ -245,7 +247,10 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
       float mx = -INFINITY;
       if (ok) {
         tc_fence_after();
-        tmem_ld32(tmem + (j % kKvStages) * 128 + sub * kSCols + lane_base, s);
+#pragma unroll
+        for (int h32 = 0; h32 < kSCols; h32 += 32)
+          tmem_ld32(tmem + (j % kKvStages) * 128 + sub * kSCols + h32 + lane_base,
+                    *reinterpret_cast<float(*)[32]>(s + h32));
         if (nvalid < kSCols) {
 #pragma unroll
           for (int i = 0; i < kSCols; ++i)
@@ -263,10 +268,12 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
       float* slot = red_max + (j & 1) * (kSubs * 128);
       slot[sub * 128 + r] = mx;
       quarter_barrier(q);
-      mx = fmaxf(fmaxf(slot[r], slot[128 + r]), fmaxf(slot[256 + r], slot[384 + r]));
+      mx = slot[r];
+#pragma unroll
+      for (int k = 1; k < kSubs; ++k) mx = fmaxf(mx, slot[k * 128 + r]);
       const float mt = mx * c;  // finite: every key tile has a valid column
       // Move the reference when the tile's maximum is more than 2^8 above it.
-      // The four warps of a row see the same mt and m_ref and decide alike.
+      // The warps of a row see the same mt and m_ref and decide alike.
       const bool move = mt > m_ref + kLazyLimit;
       if (__any_sync(0xffffffffu, move)) {
         const float m_new = move ? mt : m_ref;
@@ -278,10 +285,13 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
             tc_fence_after();
             const float alpha = ex2_approx(m_ref - m_new);
             float v[16];
-            tmem_ld16(tO + lane_base + sub * kOCols, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= alpha;
-            tmem_st16(tO + lane_base + sub * kOCols, v);
+            for (int h16 = 0; h16 < kOCols; h16 += 16) {
+              tmem_ld16(tO + lane_base + sub * kOCols + h16, v);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] *= alpha;
+              tmem_st16(tO + lane_base + sub * kOCols + h16, v);
+            }
             if (sub == 0) {
               tmem_ld16(tO + lane_base + 64, v);
 #pragma unroll
@@ -304,7 +314,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
       if (j >= 2 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1));
       uint8_t* prow = smem + prow_off + (j & 1) * 32768;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
+      for (int ch = 0; ch < kSCols / 8; ++ch)
         *reinterpret_cast<uint4*>(prow + (((ch0 + ch) ^ (r & 7)) << 4)) =
             make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       fence_proxy_async_smem();
@@ -318,8 +328,10 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
     const int t = qt * 128 + r;
     if (ok) {
       tc_fence_after();
-      float o[16];
-      tmem_ld16(tO + lane_base + sub * kOCols, o);
+      float o[kOCols];
+#pragma unroll
+      for (int h16 = 0; h16 < kOCols; h16 += 16)
+        tmem_ld16(tO + lane_base + sub * kOCols + h16, *reinterpret_cast<float(*)[16]>(o + h16));
       const float l = tmem_ld1(tO + lane_base + 64);
       if (t < T) {
         const float inv = 1.0f / l;
