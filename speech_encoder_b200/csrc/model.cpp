@@ -1370,7 +1370,7 @@ float time_forward_us(w2v_model* m, const Plan& p, const float* pcm, float* logi
   cudaEvent_t e0, e1;
   if (cudaEventCreate(&e0) == cudaSuccess && cudaEventCreate(&e1) == cudaSuccess) {
     cudaGraphLaunch(ge, st);
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 5; ++i) {
       cudaEventRecord(e0, st);
       cudaGraphLaunch(ge, st);
       cudaEventRecord(e1, st);
@@ -1424,7 +1424,52 @@ int refine_plan(w2v_model* m, Plan* p, const float* pcm, float* logits) {
     if (rc != W2V_OK) return rc;
     if (log) std::fprintf(stderr, "w2v tune: %s -> bn=%d splits=%d, forward %.1f us\n", names[role], cur_bn, cur_s, best);
   }
-  return W2V_OK;
+  // The conv layers, the projection and the CTC head: their choices were
+  // timed alone, which misses what a launch costs in the forward (the
+  // overlap with its neighbours); time their candidates in the forward too.
+  auto refine_one = [&](const char* name, GemmShape* sh, int* bn_field, CUtensorMap* bmap, const __half* W, int N,
+                        int K) -> int {
+    const int nk = K / 64;
+    int cur_bn = *bn_field, cur_s = form_code(*sh);
+    auto apply = [&](int bn, int sp) -> int {
+      set_form(sh, sp);
+      *bn_field = bn;
+      CUDA_OR(m, map_b(bmap, W, N, K, bn, sp));
+      return W2V_OK;
+    };
+    for (int bn : {32, 64, 128, 192, 256}) {
+      if (bn == 32 ? N > 32 : N <= bn / 2) continue;
+      for (int sp : {1, 2, 3, 4, 6, -2, -3, -4, 0, kFormPersist}) {
+        if (sp > 1 && sp != kFormPersist && (sh->batch != 1 || nk < 8 || sp > nk / 2)) continue;
+        if (sp < 0 && !l2_split_ok(m, *sh, N, bn, -sp)) continue;
+        if (sp == 0 && bn < 64) continue;
+        if (sp == kFormPersist && !persist_worth(*sh, N, bn)) continue;
+        if (bn == cur_bn && sp == cur_s) continue;
+        int rc = apply(bn, sp);
+        if (rc != W2V_OK) return rc;
+        const float t = time_forward_us(m, *p, pcm, logits);
+        if (t < best * 0.995f) {
+          best = t;
+          cur_bn = bn;
+          cur_s = sp;
+        }
+      }
+    }
+    const int rc = apply(cur_bn, cur_s);
+    if (log) std::fprintf(stderr, "w2v tune: %s -> bn=%d splits=%d, forward %.1f us\n", name, cur_bn, cur_s, best);
+    return rc;
+  };
+  static const char* conv_names[7] = {"", "conv1", "conv2", "conv3", "conv4", "conv5", "conv6"};
+  for (int i = 1; i < 7; ++i) {
+    if (p->convLn3[i]) continue;  // the row-LayerNorm epilogue has its own constraints
+    const int rc = refine_one(conv_names[i], &p->convS[i], &p->convBN[i], &p->convB[i], m->cw[i], kC, p->convS[i].K);
+    if (rc != W2V_OK) return rc;
+  }
+  {
+    const int rc = refine_one("projection", &p->projS, &p->projBN, &p->projB, m->wp, d, kC);
+    if (rc != W2V_OK) return rc;
+  }
+  return refine_one("lm_head", &p->lmS, &p->lmBN, &p->lmB, m->wlm, m->cfg.vocab, d);
 }
 }  // namespace
 
