@@ -6,15 +6,16 @@
 //   warp 0      TMA: the Q tile once, then K and V^T tiles of 128 keys into a
 //               3-deep ring
 //   warp 1      TMEM owner; one thread issues S_j = Q K_j^T (M=128, N=128,
-//               K=64) into one of three TMEM score buffers and, once P_j is in
-//               shared memory, O += P_j [V_j | 1] (M=128, N=80, K=128) into a
-//               TMEM accumulator that lives across all key tiles.  The scores
-//               run up to two tiles ahead (S_{j+2} is issued as soon as its
-//               K/V tile lands, polled together with P_j), so neither the
-//               softmax nor P V waits behind the other's operands: every
-//               tcgen05.mma of M=128, K=16 occupies the tensor pipe about the
-//               same ~100-140 cycles whatever its N up to 192, which makes the
-//               eight P V instructions per tile the longer of the two chains.
+//               K=64) into one of three TMEM score buffers and, once P_j is
+//               written, O += P_j [V_j | 1] (M=128, N=80, K=128) into a TMEM
+//               accumulator that lives across all key tiles.  P_j is the A
+//               operand straight from tensor memory (it overwrites the first
+//               half of each warp's own columns of S_j), so only V crosses the
+//               shared-memory port for P V.  The scores run up to two tiles
+//               ahead (S_{j+2} is issued as soon as its K/V tile lands and
+//               P_{j-1} V_{j-1}, the last reader of its buffer, has completed;
+//               polled together with P_j), so the softmax rarely waits for its
+//               scores.
 //   warps 2-17  softmax: four warps per TMEM lane quarter, each owning 32 of
 //               the 128 key columns (and 16 of the 64 output columns) of its
 //               32 query rows; the tile's row maximum is combined through
@@ -25,8 +26,9 @@
 // the TMEM accumulator (wait for the previous P V, load, scale, store) is rare;
 // otherwise no softmax step waits for the tensor core.  P is formed as packed
 // fp16 pairs (packed fp32 FMA, rounding, then the fp16x2 exponent instruction
-// or, for a share of the pairs, a cubic on the FMA pipe) and written in the
-// 128-byte-swizzled K-major layout the MMA reads, double-buffered.  The row sum
+// or, for a share of the pairs, a cubic on the FMA pipe) and stored to tensor
+// memory in the layout of a K-major A operand (lane = query row, one 32-bit
+// column per two keys).  The row sum
 // is not accumulated by the threads: V^T carries a 65th row of ones, so column
 // 64 of the accumulator is sum_k P[r][k] computed from the same fp16 P that
 // multiplies V.
@@ -45,8 +47,7 @@ struct AttnSmem {
   static constexpr int K0 = 16384;                        // [stages] 128 keys x 64 dims, SW128
   static constexpr int kVHalf = 10240;                    // 80 rows (64 dims + ones + zeros) x 64 keys
   static constexpr int V0 = K0 + kKvStages * 16384;       // [stages][2 key halves] kVHalf
-  static constexpr int P = V0 + kKvStages * 2 * kVHalf;   // [2 buffers] 128 rows x 128 keys fp16, SW128
-  static constexpr int RED = P + 2 * 32768;        // float red_max[2][4][128]
+  static constexpr int RED = V0 + kKvStages * 2 * kVHalf;  // float red_max[2][4][128]
   static constexpr int BAR = RED + 4096;
   static constexpr int TOTAL = BAR + 256 + 1024;
 };
@@ -159,7 +160,6 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
       // start-address field (16-byte units; addresses stay below 256 KB).
       const uint64_t dQ = desc_sw128(smem_u32(smem + AttnSmem::Q));
       const uint64_t dK0 = desc_sw128(smem_u32(smem + AttnSmem::K0));
-      const uint64_t dP0 = desc_sw128(smem_u32(smem + AttnSmem::P));
       const uint64_t dV0 = desc_sw128(smem_u32(smem + AttnSmem::V0));
       auto issue_s = [&](int j) {
         const int b = j % kKvStages;
@@ -181,43 +181,54 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
           }
         }
       }
-      // S_m may be issued once its K/V stage has landed and P_{m-3} was seen
-      // (S_m reuses the score buffer of S_{m-3}, whose softmax finished reading
-      // it before publishing P_{m-3}): m <= j + 2 while waiting for P_j.  The
-      // thread polls both, so P_j V_j never waits behind a K/V tile that is
-      // still in flight (that tile's stage is only refilled after an earlier
-      // P V completes).
+      // S_m may be issued once its K/V stage has landed and P_{m-3} V_{m-3},
+      // the last reader of its score buffer (P_{m-3} lives there), has
+      // completed; m <= j + 2 while waiting for P_j.  Completed P V products
+      // are confirmed strictly in order (pv_seen), and P_j V_j is issued only
+      // after P_{j-2} V_{j-2} was confirmed, so the phase tested on a pv_done
+      // barrier is always the latest one it can have reached: a parity test
+      // would otherwise pass or fail wrongly once the barrier had moved two
+      // phases on.  The thread polls everything with test_wait (a try_wait on
+      // an open phase may suspend it and delay the other barriers), so P_j V_j
+      // never waits behind a K/V tile that is still in flight (that tile's
+      // stage is only refilled after an earlier P V completes).
       int next_s = nkv > 1 ? 2 : 1;
+      int pv_seen = 0;  // P V products known complete
       for (int j = 0; ok && j < nkv; ++j) {
-        bool have_p = false;
-        const uint64_t t0 = globaltimer_ns();
+        bool have_p = false, ready = false;
+        uint64_t t0 = globaltimer_ns();
         for (uint32_t it = 1;; ++it) {
-          // test_wait: a try_wait on a phase still open may suspend the
-          // thread for a while, delaying the other barrier's detection
-          if (next_s < nkv && next_s <= j + 2 &&
+          while (pv_seen < j && mbar_test_wait(&pv_done[pv_seen & 1], (pv_seen >> 1) & 1)) ++pv_seen;
+          if (next_s < nkv && next_s <= j + 2 && (next_s < 3 || pv_seen >= next_s - 2) &&
               mbar_test_wait(&kv_full[next_s % kKvStages], (next_s / kKvStages) & 1)) {
             tc_fence_after();
             issue_s(next_s);
             ++next_s;
+            t0 = globaltimer_ns();
           }
-          if (mbar_test_wait(&p_full[j & 1], (j >> 1) & 1)) {
-            have_p = true;
+          if (!have_p) have_p = mbar_test_wait(&p_full[j & 1], (j >> 1) & 1);
+          if (have_p && (j < 2 || pv_seen >= j - 1)) {
+            ready = true;
             break;
           }
           if ((it & 255u) == 0 && globaltimer_ns() - t0 > W2V_WAIT_LIMIT_NS) break;
         }
-        if (!have_p) {
+        if (!ready) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t dP = dP0 + static_cast<uint64_t>((j & 1) * (32768 >> 4));
+        // P_j: keys kSCols w .. kSCols (w + 1) - 1 (softmax warp w of a lane
+        // quarter) at columns kSCols w .. kSCols w + kSCols / 2 - 1 of score
+        // buffer j % 3, so K step kk (16 keys) starts at column
+        // kSCols (16 kk / kSCols) + 8 (kk % (kSCols / 16)).
+        const uint32_t tP = tmem + static_cast<uint32_t>((j % kKvStages) * 128);
         const uint64_t dV = dV0 + static_cast<uint64_t>((j % kKvStages) * (2 * AttnSmem::kVHalf >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = dP + static_cast<uint64_t>((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
+          const uint32_t a = tP + static_cast<uint32_t>(kSCols * (16 * kk / kSCols) + 8 * (kk % (kSCols / 16)));
           const uint64_t bv = dV + static_cast<uint64_t>((kk >> 2) * (AttnSmem::kVHalf >> 4) + (kk & 3) * 2);
-          umma_f16(tO, a, bv, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tO, a, bv, idO, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[j & 1]);
         umma_commit(&kv_empty[j % kKvStages]);
@@ -231,11 +242,6 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float c = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
     float m_ref = -INFINITY;                        // reference maximum, log2 units
-    // This warp's keys within the 64-key swizzle atoms of P: 32 keys are half
-    // of atom sub >> 1 (chunks from ch0), 64 keys are atom sub.
-    const int atom = kSCols >= 64 ? sub : (sub >> 1);
-    const int prow_off = AttnSmem::P + atom * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
-    const int ch0 = kSCols >= 64 ? 0 : (sub & 1) * 4;
     bool ok = true;
     // Every iteration runs the quarter barrier and the p_full arrival even
     // after a failed wait (the work is skipped), so no thread is left waiting
@@ -310,19 +316,25 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
       for (int i = 0; i < kSCols; i += 2)
         pk[i / 2] = (i / 2 < kPolyPairs) ? exp2_affine_poly_f16x2(s[i], s[i + 1], c, nb)
                                          : exp2_affine_f16x2(s[i], s[i + 1], c, nb);
-      // P buffer j & 1 was last read by P_{j-2} V_{j-2}.
+      // This warp's arrival for P_j goes to the barrier that carried P_{j-2}:
+      // that phase must be complete first, which P_{j-2} V_{j-2} having run
+      // shows (no warp of another lane quarter may still owe it an arrival).
       if (j >= 2 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1));
-      uint8_t* prow = smem + prow_off + (j & 1) * 32768;
+      // P over the first half of this warp's own score columns (read above):
+      // packed key pairs, the A operand layout of P V.
+      if (ok) {
 #pragma unroll
-      for (int ch = 0; ch < kSCols / 8; ++ch)
-        *reinterpret_cast<uint4*>(prow + (((ch0 + ch) ^ (r & 7)) << 4)) =
-            make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-      fence_proxy_async_smem();
+        for (int h16 = 0; h16 < kSCols / 2; h16 += 16)
+          tmem_st16_u32(tmem + (j % kKvStages) * 128 + sub * kSCols + h16 + lane_base,
+                        *reinterpret_cast<const uint32_t(*)[16]>(pk + h16));
+      }
       tc_fence_before();
       // one arrival per warp: 512 arrivals on one barrier word serialise
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[j & 1]);
     }
+    // The last product (P_{last-2} V_{last-2}, the previous phase of its
+    // barrier, was waited for above, so the parity is unambiguous).
     const int last = nkv - 1;
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[last & 1], (last >> 1) & 1));
     const int t = qt * 128 + r;
