@@ -64,6 +64,20 @@ __device__ __forceinline__ void quarter_barrier(int q) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kSubs) : "memory");
 }
 
+// The same barrier, returning whether any thread of the quarter passed true.
+__device__ __forceinline__ bool quarter_barrier_any(int q, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"(v ? 1u : 0u), "r"(1 + q), "r"(32 * kSubs)
+      : "memory");
+  return out != 0;
+}
+
 // One CTA's work: query tile qt (local rows qt*128 ..) of one clip of T frames
 // and head h.  The clip's queries start at row qrow of the Q map (batch
 // coordinate bz), its keys at row krow0 of the K map and column krow0 of the V^T
@@ -271,16 +285,25 @@ __device__ __forceinline__ void attention_body(const CUtensorMap& tmQ, const CUt
         mx = fmax3(m0, m1, s[kSCols - 2]);
         mx = fmaxf(mx, s[kSCols - 1]);
       }
-      float* slot = red_max + (j & 1) * (kSubs * 128);
-      slot[sub * 128 + r] = mx;
-      quarter_barrier(q);
-      mx = slot[r];
+      // Move a row's reference when the tile's maximum is more than 2^8 above
+      // it.  Usually no row of the lane quarter moves: one barrier whose
+      // predicate reduction says so replaces the exchange of the row maxima
+      // (exact: a row's maximum exceeds the limit only if one of its warps'
+      // column maxima does).  Otherwise the maxima are combined through shared
+      // memory and the warps of a row see the same mt and m_ref and decide
+      // alike.
+      bool move = false;
+      float mt = 0.f;
+      if (quarter_barrier_any(q, mx * c > m_ref + kLazyLimit)) {
+        float* slot = red_max + (j & 1) * (kSubs * 128);
+        slot[sub * 128 + r] = mx;
+        quarter_barrier(q);
+        mx = slot[r];
 #pragma unroll
-      for (int k = 1; k < kSubs; ++k) mx = fmaxf(mx, slot[k * 128 + r]);
-      const float mt = mx * c;  // finite: every key tile has a valid column
-      // Move the reference when the tile's maximum is more than 2^8 above it.
-      // The warps of a row see the same mt and m_ref and decide alike.
-      const bool move = mt > m_ref + kLazyLimit;
+        for (int k = 1; k < kSubs; ++k) mx = fmaxf(mx, slot[k * 128 + r]);
+        mt = mx * c;  // finite: every key tile has a valid column
+        move = mt > m_ref + kLazyLimit;
+      }
       if (__any_sync(0xffffffffu, move)) {
         const float m_new = move ? mt : m_ref;
         if (j > 0 && ok) {
