@@ -18,8 +18,10 @@
 //               scores.
 //   warps 2-17  softmax: four warps per TMEM lane quarter, each owning 32 of
 //               the 128 key columns (and 16 of the 64 output columns) of its
-//               32 query rows; the tile's row maximum is combined through
-//               shared memory with a 128-thread named barrier per quarter.
+//               32 query rows; a 128-thread named barrier per quarter
+//               tells whether any row's reference must move (an OR-reduced
+//               predicate), and only then are the row maxima combined
+//               through shared memory.
 // Online softmax with a lazily moved reference: a row's reference maximum m
 // (log2 units, 1/8 scale folded in) moves only when the tile's maximum exceeds
 // it by more than 8, so P = 2^(s/8 log2 e - m) stays <= 256 and the rescale of
